@@ -1,0 +1,220 @@
+"""fp64 CPU oracle for attention with an additive rank-factorised bias.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library
+never calls it and shares no code with it.
+
+What it computes (per batch-head, scale ``s``)::
+
+    S   = s * Q @ K.T + U @ W.T        # bias matrix formed explicitly
+    P   = softmax(S, axis=-1)
+    O   = P @ V
+    LSE = log(sum(exp(S), axis=-1))    # natural log
+
+following "FlashBias: Fast Computation of Attention with Bias" (Abstract: a
+bias matrix added to the query-key scores) and "Rank-Factorized Implicit Neural
+Bias" (Abstract: a low-rank bias U W^T).  The backward is the plain chain rule
+through the same definition (see ``rfb_oracle.c``).
+
+The arithmetic lives in ``rfb_oracle.c`` (plain C, fp64, OpenMP over output
+rows).  This module only compiles it with gcc and marshals numpy arrays.
+
+Every function is pinned by ``tests/test_oracle_*.py`` against library special
+cases (torch SDPA and autograd in fp64), brute force with ``math.fsum``,
+closed forms, invariants and finite differences.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rfb_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "librfb_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_lp = ctypes.POINTER(ctypes.c_long)
+
+
+def _compile(src: str, out: str) -> str:
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+           "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, IEEE semantics kept, OpenMP)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    return _compile(_SRC, _LIB_PATH)
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    L, D, I = ctypes.c_long, ctypes.c_double, ctypes.c_int
+    lib.rfb_oracle_fwd.argtypes = [_dp] * 7 + [L] * 4 + [D, L, L, _lp, L, I]
+    lib.rfb_oracle_fwd.restype = I
+    lib.rfb_oracle_bwd.argtypes = [_dp] * 12 + [L] * 4 + [D, L, L, I]
+    lib.rfb_oracle_bwd.restype = I
+    lib.rfb_oracle_bwd_query_rows.argtypes = [_dp] * 9 + [L] * 4 + [D, L, _lp, L, I]
+    lib.rfb_oracle_bwd_query_rows.restype = I
+    lib.rfb_oracle_max_threads.argtypes = []
+    lib.rfb_oracle_max_threads.restype = I
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(build())
+    return _lib
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+class Variant:
+    """The same Python API bound to a separately compiled copy of the oracle
+    source (used by the mutation tests to plant mistakes in a copy)."""
+
+    def __init__(self, src_text: str, workdir: str):
+        os.makedirs(workdir, exist_ok=True)
+        src = os.path.join(workdir, "variant.c")
+        with open(src, "w") as f:
+            f.write(src_text)
+        self._lib = _bind(_compile(src, os.path.join(workdir, "libvariant.so")))
+
+    def fwd(self, *a, **kw):
+        return fwd(*a, _lib_override=self._lib, **kw)
+
+    def bwd(self, *a, **kw):
+        return bwd(*a, _lib_override=self._lib, **kw)
+
+
+def max_threads() -> int:
+    return int(_load().rfb_oracle_max_threads())
+
+
+def _as_f64(x):
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    return a
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(_dp)
+
+
+def _shape(q, u):
+    if q.ndim != 4:
+        raise ValueError("expected [B, H, N, d]")
+    B, H, N, d = q.shape
+    r = 0 if u is None else u.shape[-1]
+    return B, H, N, d, r
+
+
+def _prep(q, k, v, u, w):
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, H, N, d, r = _shape(q, u)
+    if r > 0:
+        u, w = _as_f64(u), _as_f64(w)
+        if u.shape != (B, H, N, r) or w.shape != (B, H, N, r):
+            raise ValueError("U, W must be [B, H, N, r]")
+    else:
+        u = w = None
+    for t in (k, v):
+        if t.shape != q.shape:
+            raise ValueError("Q, K, V must share [B, H, N, d]")
+    return q, k, v, u, w, (B, H, N, d, r)
+
+
+def fwd(q, k, v, u, w, scale, *, nthreads: int = 0, bh_range=None, rows=None,
+        _lib_override=None):
+    """Forward.  Returns ``(O, LSE)`` as float64.
+
+    With ``bh_range=(bh0, bh1)`` and/or ``rows`` (query indices) only those
+    heads / rows are computed; shapes are then ``[bh1-bh0, len(rows), d]`` and
+    ``[bh1-bh0, len(rows)]``.  Without them: ``[B, H, N, d]`` and ``[B, H, N]``.
+    """
+    q, k, v, u, w, (B, H, N, d, r) = _prep(q, k, v, u, w)
+    BH = B * H
+    bh0, bh1 = (0, BH) if bh_range is None else bh_range
+    if rows is None:
+        rows_a, nrows = None, N
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows = int(rows_a.size)
+    nh = bh1 - bh0
+    o = np.empty((nh, nrows, d), dtype=np.float64)
+    lse = np.empty((nh, nrows), dtype=np.float64)
+    rc = (_lib_override or _load()).rfb_oracle_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o), _ptr(lse), BH, N, d, r,
+        float(scale), bh0, bh1,
+        None if rows_a is None else rows_a.ctypes.data_as(_lp), nrows, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle fwd failed ({rc})")
+    if bh_range is None and rows is None:
+        return o.reshape(B, H, N, d), lse.reshape(B, H, N)
+    return o, lse
+
+
+def bwd(q, k, v, u, w, dout, scale, *, nthreads: int = 0, bh_range=None, return_D=False,
+        _lib_override=None):
+    """Full backward.  Returns ``(dQ, dK, dV, dU, dW)`` (dU, dW are None when r == 0),
+    shaped like the inputs, or ``[bh1-bh0, N, c]`` with ``bh_range``."""
+    q, k, v, u, w, (B, H, N, d, r) = _prep(q, k, v, u, w)
+    dout = _as_f64(dout)
+    BH = B * H
+    bh0, bh1 = (0, BH) if bh_range is None else bh_range
+    nh = bh1 - bh0
+    dq = np.empty((nh, N, d))
+    dk = np.empty((nh, N, d))
+    dv = np.empty((nh, N, d))
+    du = np.empty((nh, N, r)) if r else None
+    dw = np.empty((nh, N, r)) if r else None
+    D = np.empty((nh, N))
+    rc = (_lib_override or _load()).rfb_oracle_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(dout), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(du), _ptr(dw), _ptr(D), BH, N, d, r, float(scale), bh0, bh1,
+        int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle bwd failed ({rc})")
+    out = [dq, dk, dv, du, dw]
+    if bh_range is None:
+        out = [None if t is None else t.reshape(B, H, N, t.shape[-1]) for t in out]
+        D = D.reshape(B, H, N)
+    return (tuple(out), D) if return_D else tuple(out)
+
+
+def bwd_query_rows(q, k, v, u, w, dout, scale, bh, rows, *, nthreads: int = 0):
+    """dQ_i, dU_i and D_i for the listed query rows of flat head ``bh``."""
+    q, k, v, u, w, (B, H, N, d, r) = _prep(q, k, v, u, w)
+    dout = _as_f64(dout)
+    rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = int(rows_a.size)
+    dq = np.empty((n, d))
+    du = np.empty((n, r)) if r else None
+    D = np.empty(n)
+    rc = _load().rfb_oracle_bwd_query_rows(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(dout), _ptr(dq), _ptr(du),
+        _ptr(D), B * H, N, d, r, float(scale), int(bh), rows_a.ctypes.data_as(_lp), n,
+        int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle bwd_query_rows failed ({rc})")
+    return dq, du, D
