@@ -1,0 +1,417 @@
+#!/usr/bin/env python3
+"""Throughput of the rank-factorised-bias attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {rfb,reference}]
+                    [--workload train] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path -- forward (O, LSE) and backward
+(dQ, dK, dV, dU, dW) -- over one batch of the training workload: B=2 images of a
+128x128 token map (N=16384), H=8 heads, d=64, bias rank r=32, bf16, seeded
+synthetic inputs (rank_biased_window_b200/inputs.py).  The metric is
+algorithmic bf16 TFLOP/s of that step (forward 2*BH*N^2*(2d+r) plus backward
+2*BH*N^2*(5d+3r) flops, r counted unpadded), with windows/s beside it.
+
+Multi-GPU (launched with torchrun): every rank runs its own full workload on
+its own GPU (independent problems, weak scaling, no data-path collective);
+the step time is the max over ranks and `value` counts the work of all ranks.
+
+`--impl reference` times the fp64 CPU oracle (oracle/) on the host cores on a
+bounded sample of the same workload; it is a deliberately slow reference, not
+a tuned CPU implementation.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "biased-attn fwd+bwd TFLOP/s (bf16) & % of B200 dense-BF16 peak; windows/s"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("rfb", "reference"), default="rfb")
+    ap.add_argument("--workload", default="train")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target wall seconds of the CPU-baseline sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- work model
+def work(wl):
+    BH, N, d, r = wl.B * wl.H, wl.N, wl.d, wl.r
+    fwd = 2.0 * BH * N * N * (2 * d + r)
+    bwd = 2.0 * BH * N * N * (5 * d + 3 * r) if wl.backward else 0.0
+    # bytes that must cross HBM once (inputs read, outputs written), bf16 / fp32
+    fwd_bytes = BH * N * (2 * (3 * d + 2 * r + d) + 4)
+    bwd_bytes = BH * N * (2 * (5 * d + 2 * r) + 12 + 2 * (3 * d + 2 * r)) if wl.backward else 0
+    return fwd, bwd, fwd_bytes, bwd_bytes
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_biased_window_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """Per-launch DRAM bytes from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    return t.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ clock sampling
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device_index)
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - clocks are reported, not required
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                bits = fn(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.05)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        busy = [s for s in self.samples] or [0]
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ CPU reference
+def cpu_sample(wl, seconds, x64=None):
+    """Times the fp64 oracle on a bounded sample of the workload: forward and the
+    query-side backward (dQ, dU) of R query rows of head 0 against all N keys,
+    with R calibrated so the sample takes about `seconds`.  Returns
+    (credited flops, wall seconds, rows, threads)."""
+    import oracle
+    from rank_biased_window_b200.inputs import to_f64, workload_inputs
+    if x64 is None:
+        x = workload_inputs(wl, with_dout=True)
+        # only head 0 is touched: slice it to keep the conversion cheap
+        x64 = {k: to_f64(v[:1, :1].contiguous()) for k, v in x.items()}
+    N, d, r = wl.N, wl.d, wl.r
+    s = wl.scale
+
+    def run(rows):
+        t0 = time.perf_counter()
+        oracle.fwd(x64["q"], x64["k"], x64["v"], x64["u"], x64["w"], s, bh_range=(0, 1),
+                   rows=rows)
+        if wl.backward:
+            oracle.bwd_query_rows(x64["q"], x64["k"], x64["v"], x64["u"], x64["w"], x64["dout"],
+                                  s, 0, rows)
+        return time.perf_counter() - t0
+
+    probe_rows = list(range(min(64, N)))
+    t_probe = run(probe_rows)
+    R = int(max(16, min(N, len(probe_rows) * seconds / max(t_probe, 1e-6))))
+    rows = list(range(R))
+    t = run(rows)
+    flops = 2.0 * R * N * (2 * d + r)
+    if wl.backward:
+        flops += 2.0 * R * N * (3 * d + 2 * r)  # recompute S, dP, [dQ | dU]
+    return flops, t, R, oracle.max_threads(), x64
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return 0
+    per_step = max(1.0, 150.0 / max(args.steps + args.warmup, 1))
+    flops, t, R, cores, x64 = cpu_sample(wl, per_step)
+    times = []
+    for i in range(args.warmup + args.steps):
+        f_i, t_i, _, _, _ = cpu_sample_fixed(wl, R, x64)
+        if i >= args.warmup:
+            times.append(t_i)
+    t_step = statistics.mean(times) if times else t
+    value = flops / t_step / 1e12
+    sample = (f"fp64 oracle, head 0 of {wl.B * wl.H}, {R} of {wl.N} query rows against all keys: "
+              f"forward + query-side backward (dQ, dU)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r,
+                   "parallelism": "cpu", "note": wl.note},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_sample_fixed(wl, R, x64):
+    import oracle
+    rows = list(range(R))
+    t0 = time.perf_counter()
+    oracle.fwd(x64["q"], x64["k"], x64["v"], x64["u"], x64["w"], wl.scale, bh_range=(0, 1),
+               rows=rows)
+    if wl.backward:
+        oracle.bwd_query_rows(x64["q"], x64["k"], x64["v"], x64["u"], x64["w"], x64["dout"],
+                              wl.scale, 0, rows)
+    t = time.perf_counter() - t0
+    flops = 2.0 * R * wl.N * (2 * wl.d + wl.r)
+    if wl.backward:
+        flops += 2.0 * R * wl.N * (3 * wl.d + 2 * wl.r)
+    return flops, t, R, None, x64
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    args = parse_args()
+    from rank_biased_window_b200.inputs import WORKLOADS, workload_inputs
+    wl = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, wl, rank)
+
+    import torch
+    import rank_biased_window_b200 as rfb
+    from rank_biased_window_b200 import build as rfb_build
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if rank == 0 and not rfb_build.up_to_date():
+        rfb_build.build()
+    if dist is not None:
+        dist.barrier()
+    rfb.load_library()
+
+    x = workload_inputs(wl, with_dout=True)
+    g = {k: v.to(dev) for k, v in x.items()}
+    B, H, N, d, r = wl.B, wl.H, wl.N, wl.d, wl.r
+    s = wl.scale
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"]),
+             torch.empty_like(g["u"]), torch.empty_like(g["w"]))
+    ws = torch.empty(rfb.bwd_workspace_size(B, H, N, d, r), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        rfb.attn_fwd(g["q"], g["k"], g["v"], g["u"], g["w"], s, out=o, lse=lse, stream=stream)
+        if wl.backward:
+            rfb.attn_bwd(g["q"], g["k"], g["v"], g["u"], g["w"], o, lse, g["dout"], s,
+                         workspace=ws, grads=grads, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert rfb.last_device_error() == 0
+
+    # ---- device-timed region: inputs resident in HBM (and larger than L2)
+    rfb.profile_read()
+    rfb.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    rfb.profile_enable(False)
+    prof = rfb.profile_read()
+    ms_total = e0.elapsed_time(e1)
+    err = rfb.last_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error word {err:#x} after the timed region")
+
+    # ---- end-to-end through the public API with pinned host buffers
+    host_in = {k: v.pin_memory() for k, v in x.items()}
+    host_out = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
+    names = ("dq", "dk", "dv", "du", "dw")
+    for n_, t_ in zip(names, grads):
+        host_out[n_] = torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def e2e_step():
+        for k_, v_ in host_in.items():
+            g[k_].copy_(v_, non_blocking=True)
+        step()
+        host_out["o"].copy_(o, non_blocking=True)
+        host_out["lse"].copy_(lse, non_blocking=True)
+        for n_, t_ in zip(names, grads):
+            host_out[n_].copy_(t_, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e_total = f0.elapsed_time(f1)
+
+    # ---- max over ranks
+    vals = torch.tensor([ms_total, ms_e2e_total], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, ms_e2e_total = float(vals[0]), float(vals[1])
+
+    fwd_f, bwd_f, fwd_b, bwd_b = work(wl)
+    step_flops = fwd_f + bwd_f
+    ms_step = ms_total / args.steps
+    value = step_flops * world / (ms_step * 1e-3) / 1e12
+    e2e_value = step_flops * world / (ms_e2e_total / e2e_steps * 1e-3) / 1e12
+
+    peaks = read_peaks()
+    # dominant kernel by measured time
+    per = {k: (v[0] / v[1] if v[1] else 0.0, v[1], v[0]) for k, v in prof.items()}
+    dom = max(per, key=lambda k: per[k][2])
+    dom_flops = {"fwd": fwd_f, "bwd_main": bwd_f}.get(dom)
+    launches = sum(v[1] for v in prof.values())
+    if dom_flops is not None:
+        achieved = dom_flops / (per[dom][0] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "peak_kind": f"bf16 sustained, {peaks['source']}",
+                "traffic": ncu_traffic(dom, wl.name),
+                "avg_launch_ms": per[dom][0]}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": None}
+
+    kernels = {k: {"avg_ms": v[0], "launches": v[1], "share": v[2] / max(sum(w[2] for w in
+               per.values()), 1e-9)} for k, v in per.items() if v[1]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops_c, t_c, R, cores, _ = cpu_sample(wl, args.cpu_seconds)
+        cpu = {"value": flops_c / t_c / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"fp64 oracle, head 0 of {wl.B * wl.H}, {R} of {wl.N} query rows "
+                         f"against all keys: forward + query-side backward (dQ, dU), "
+                         f"{t_c:.1f} s"}
+
+    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q,K,V,dO; N(0,1/r) U,W; bf16)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r,
+                   "global_batch": wl.B * world, "seq_len": wl.N,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs exceed L2 ({in_bytes / 2**20:.0f} MiB > 126 MiB), no flush",
+                   "note": wl.note},
+        "windows_per_s": wl.B * world / (ms_step * 1e-3),
+        "pct_of_bf16_peak": value / world / peaks["bf16_tflops"] * 100.0,
+        "roofline": roof,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,154 @@
+/*
+ * rfb_attn.h -- C ABI of the B200 (sm_100a) library for attention with an
+ * additive rank-factorised bias:
+ *
+ *     S   = s * Q K^T + U W^T                    (per batch b, head h)
+ *     O   = softmax_rows(S) V
+ *     LSE = log(sum_j exp(S_ij))                 (natural log, per row i)
+ *
+ * Where the operation comes from:
+ *   - "FlashBias: Fast Computation of Attention with Bias", Abstract: attention
+ *     with bias adds a bias matrix to the query-key scores; a low-rank bias
+ *     lets the fused (FlashAttention-style) pipeline stay intact.
+ *   - "Rank-Factorized Implicit Neural Bias: Scaling Super-Resolution
+ *     Transformer with FlashAttention", Abstract: the positional bias is a
+ *     low-rank product whose factors are concatenated with the content tokens
+ *     along channels, so the element-wise bias addition becomes part of one
+ *     dot product.  Here U, W are those factors; the library evaluates
+ *     [Q | U/s] . [K | W]^T inside one fused kernel and never forms the N x N
+ *     bias.
+ *   - The scale s multiplies Q K^T only (the bias is added after scaling).
+ *
+ * Conventions for every entry point
+ *   - Layout: all tensors are contiguous row-major.  Q, K, V, O, dO and their
+ *     gradients are [B, H, N, d] bf16; U, W, dU, dW are [B, H, N, r] bf16;
+ *     LSE is [B, H, N] fp32.  The bias factors are per (batch, head).
+ *   - Pointers are DEVICE pointers (CUDA global memory of the current device)
+ *     and must be 16-byte aligned.  The caller owns every buffer; the library
+ *     allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream.  Calls are asynchronous on that stream: a return value
+ *     of RFB_OK means the work was enqueued, not that it finished.
+ *   - Supported shapes: d in {32, 64}; r in {0, 8, 16, ..., 64} (a multiple of
+ *     8); B, H, N >= 0.  B*H*N == 0 is a no-op that returns RFB_OK without
+ *     touching any pointer.  When r == 0, u / w / du / dw may be NULL.
+ *   - Outputs must not alias inputs.
+ *   - Errors are reported only through the return code; nothing is thrown
+ *     across the ABI.  Argument checks happen on the host before anything is
+ *     enqueued.
+ */
+#ifndef RFB_ATTN_H_
+#define RFB_ATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define RFB_API __attribute__((visibility("default")))
+#else
+#define RFB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RFB_OK = 0,
+  RFB_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, non-finite scale */
+  RFB_ERR_UNSUPPORTED = 2,    /* d or r outside the supported set, sizes beyond int32 */
+  RFB_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
+  RFB_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+  RFB_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
+  RFB_ERR_DEVICE_TIMEOUT = 6  /* a kernel's bounded wait expired (see rfb_last_device_error) */
+} rfb_status;
+
+/*
+ * Forward.  Computes O and LSE as defined above.
+ *   q, k, v : [B, H, N, d] bf16 inputs.
+ *   u, w    : [B, H, N, r] bf16 bias factors (NULL allowed iff r == 0).
+ *   o       : [B, H, N, d] bf16 output.
+ *   lse     : [B, H, N] fp32 output (natural-log log-sum-exp of each score row,
+ *             consumed by rfb_attn_bwd).
+ *   scale   : s, any finite value (usually 1/sqrt(d)).
+ */
+RFB_API int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, const void* w,
+                 void* o, float* lse, int B, int H, int N, int d, int r, float scale,
+                 void* stream);
+
+/*
+ * Bytes of device workspace rfb_attn_bwd needs for these sizes (fp32 row
+ * statistics and the fp32 dQ | dU accumulator).  Returns 0 for unsupported or
+ * empty shapes.
+ */
+RFB_API size_t rfb_attn_bwd_workspace_size(int B, int H, int N, int d, int r);
+
+/*
+ * Backward.  Given the forward inputs, the forward outputs o and lse, and the
+ * upstream gradient dout = dL/dO, writes
+ *     dq = s dS K,  dk = s dS^T Q,  dv = P^T dO,  du = dS W,  dw = dS^T U,
+ * with P = softmax(S), dS = P o (dO V^T - rowsum(dO o O)).
+ *   dq, dk, dv : [B, H, N, d] bf16 outputs.
+ *   du, dw     : [B, H, N, r] bf16 outputs (NULL allowed iff r == 0).
+ *   workspace  : device buffer of at least rfb_attn_bwd_workspace_size() bytes,
+ *                16-byte aligned, owned by the caller, contents irrelevant on
+ *                entry and scratch afterwards.  It must not be used by another
+ *                call that runs concurrently.
+ */
+RFB_API int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, const void* w,
+                 const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                 void* du, void* dw, void* workspace, size_t workspace_bytes, int B, int H,
+                 int N, int d, int r, float scale, void* stream);
+
+/* Human-readable text for a status code (static storage). */
+RFB_API const char* rfb_strerror(int status);
+
+/*
+ * Reads and clears the current device's error word, which kernels set when a
+ * bounded wait expires (RFB_ERR_DEVICE_TIMEOUT in the low byte, the wait site
+ * in the next byte).  Synchronises the device first.  Returns 0 if no error
+ * was recorded, -RFB_ERR_CUDA if the word could not be read.
+ */
+RFB_API int rfb_last_device_error(void);
+
+/*
+ * Diagnostics for RFB_ERR_CUDA: the error code of the last CUDA runtime /
+ * driver call that failed inside the library (a cudaError_t, or a CUresult
+ * for tensor-map encoding), and in *site (if not NULL) which call it was:
+ * 1 device query, 2 attribute query, 3 symbol address, 4 driver entry point,
+ * 5 tensor-map encoding, 6 kernel attribute, 7 kernel launch, 8 synchronise.
+ * Returns 0 if nothing has failed.
+ */
+RFB_API int rfb_last_cuda_error(int* site);
+
+/*
+ * Failure-detection self test: launches one CTA whose bounded wait is on an
+ * mbarrier that nothing ever arrives at, with a limit of `timeout_us`
+ * microseconds.  The wait expires, the kernel records RFB_ERR_DEVICE_TIMEOUT in
+ * the error word and returns normally, leaving the context usable.  Returns
+ * the launch status; read the outcome with rfb_last_device_error().
+ */
+RFB_API int rfb_selftest_wait_timeout(unsigned int timeout_us, void* stream);
+
+/*
+ * Optional per-kernel timing.  While enabled, every kernel launch made by
+ * rfb_attn_fwd / rfb_attn_bwd is bracketed by two CUDA events recorded on the
+ * call's stream.  rfb_profile_read synchronises on those events and returns,
+ * per kernel id (0 forward, 1 backward row statistics, 2 backward main,
+ * 3 backward gradient cast; RFB_PROFILE_KERNELS ids in all), the summed
+ * milliseconds and the number of launches since the last read, then clears
+ * them.  Arrays must hold RFB_PROFILE_KERNELS entries.  The events are created
+ * by the library (no device memory is allocated).
+ */
+#define RFB_PROFILE_KERNELS 4
+RFB_API int rfb_profile_enable(int on);
+RFB_API int rfb_profile_read(float* ms, int* launches);
+RFB_API const char* rfb_profile_kernel_name(int id);
+
+/* Library version string. */
+RFB_API const char* rfb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RFB_ATTN_H_ */

@@ -1,0 +1,24 @@
+"""rank_biased_window_b200 -- attention with an additive rank-factorised bias
+(O = softmax(s Q K^T + U W^T) V) as hand-written sm_100a CUDA kernels behind a
+C ABI (include/rfb_attn.h), with a thin ctypes binding.
+
+The library is loaded lazily on the first call; importing the package does not
+need a GPU.
+"""
+from .binding import (  # noqa: F401
+    LIB_PATH,
+    RFBAttention,
+    attn_bwd,
+    attn_fwd,
+    bwd_workspace_size,
+    last_device_error,
+    load_library,
+    profile_enable,
+    profile_read,
+    rfb_attention,
+    selftest_wait_timeout,
+    strerror,
+)
+
+__all__ = ["attn_fwd", "attn_bwd", "bwd_workspace_size", "rfb_attention", "RFBAttention",
+           "last_device_error", "selftest_wait_timeout", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]

@@ -1,0 +1,221 @@
+"""ctypes binding of the C ABI in include/rfb_attn.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``librfb_attn.so``.  torch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call fails, a
+``RuntimeError`` is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librfb_attn.so")
+
+RFB_OK = 0
+RFB_ERR_INVALID_ARG = 1
+RFB_ERR_UNSUPPORTED = 2
+RFB_ERR_ALIGNMENT = 3
+RFB_ERR_WORKSPACE = 4
+RFB_ERR_CUDA = 5
+RFB_ERR_DEVICE_TIMEOUT = 6
+
+# Every symbol the header declares, with (restype, argtypes).
+_vp, _fp, _i, _f, _sz = (ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_int,
+                         ctypes.c_float, ctypes.c_size_t)
+SIGNATURES = {
+    "rfb_attn_fwd": (_i, [_vp] * 6 + [_fp] + [_i] * 5 + [_f, _vp]),
+    "rfb_attn_bwd_workspace_size": (_sz, [_i] * 5),
+    "rfb_attn_bwd": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
+    "rfb_strerror": (ctypes.c_char_p, [_i]),
+    "rfb_last_device_error": (_i, []),
+    "rfb_last_cuda_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
+    "rfb_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
+    "rfb_profile_enable": (_i, [_i]),
+    "rfb_profile_read": (_i, [_fp, ctypes.POINTER(ctypes.c_int)]),
+    "rfb_profile_kernel_name": (ctypes.c_char_p, [_i]),
+    "rfb_version": (ctypes.c_char_p, []),
+}
+PROFILE_KERNELS = 4
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and return the ctypes handle; raises if the .so is absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"CUDA library not built: {path} is missing "
+                    "(run `python -m rank_biased_window_b200.build`)")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return load_library().rfb_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != RFB_OK:
+        extra = ""
+        if rc == RFB_ERR_CUDA:
+            site = ctypes.c_int(0)
+            code = load_library().rfb_last_cuda_error(ctypes.byref(site))
+            extra = f"; CUDA error {code} at site {site.value}"
+        raise RuntimeError(f"{what} failed: {strerror(rc)} (status {rc}{extra})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream, device):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_operand(name, t, shape, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must live on {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _dims(q, u):
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = q.shape
+    r = 0 if u is None else int(u.shape[-1])
+    return int(B), int(H), int(N), int(d), r
+
+
+def attn_fwd(q, k, v, u=None, w=None, scale=None, *, out=None, lse=None, stream=None):
+    """O, LSE = softmax(s Q K^T + U W^T) V, log-sum-exp rows (fp32)."""
+    B, H, N, d, r = _dims(q, u)
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_operand(name, t, (B, H, N, d), dev)
+    if r > 0:
+        _check_operand("u", u, (B, H, N, r), dev)
+        _check_operand("w", w, (B, H, N, r), dev)
+    else:
+        u = w = None
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_operand("out", o, (B, H, N, d), dev)
+    if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    with torch.cuda.device(dev):
+        rc = load_library().rfb_attn_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, H, N, d, r, s,
+            _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_fwd")
+    return o, l
+
+
+def bwd_workspace_size(B, H, N, d, r) -> int:
+    return int(load_library().rfb_attn_bwd_workspace_size(B, H, N, d, r))
+
+
+def attn_bwd(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=None, grads=None,
+             stream=None):
+    """dQ, dK, dV, dU, dW of L with dL/dO = dout (dU, dW are None when r == 0)."""
+    B, H, N, d, r = _dims(q, u)
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_operand(name, t, (B, H, N, d), dev)
+    if r > 0:
+        _check_operand("u", u, (B, H, N, r), dev)
+        _check_operand("w", w, (B, H, N, r), dev)
+    else:
+        u = w = None
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    if grads is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        du = torch.empty_like(u) if r else None
+        dw = torch.empty_like(w) if r else None
+    else:
+        dq, dk, dv, du, dw = grads
+    nbytes = bwd_workspace_size(B, H, N, d, r)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = load_library().rfb_attn_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, H, N, d, r, s,
+            _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_bwd")
+    return dq, dk, dv, du, dw
+
+
+def last_device_error() -> int:
+    """Synchronise the current device, read and clear the kernels' error word."""
+    return int(load_library().rfb_last_device_error())
+
+
+def selftest_wait_timeout(timeout_us: int = 1000, stream=None, device=None):
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        rc = load_library().rfb_selftest_wait_timeout(int(timeout_us), _stream_ptr(stream, dev))
+    _check(rc, "rfb_selftest_wait_timeout")
+
+
+def profile_enable(on: bool = True):
+    load_library().rfb_profile_enable(1 if on else 0)
+
+
+def profile_read():
+    """{kernel name: (total ms, launches)} since the last read (synchronises)."""
+    lib = load_library()
+    ms = (ctypes.c_float * PROFILE_KERNELS)()
+    n = (ctypes.c_int * PROFILE_KERNELS)()
+    _check(lib.rfb_profile_read(ms, n), "rfb_profile_read")
+    return {lib.rfb_profile_kernel_name(i).decode(): (float(ms[i]), int(n[i]))
+            for i in range(PROFILE_KERNELS)}
+
+
+class RFBAttention(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run the CUDA kernels."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, u, w, scale):
+        o, lse = attn_fwd(q, k, v, u, w, scale)
+        ctx.save_for_backward(q, k, v, u, w, o, lse)
+        ctx.scale = scale
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, u, w, o, lse = ctx.saved_tensors
+        dq, dk, dv, du, dw = attn_bwd(q, k, v, u, w, o, lse, dout.contiguous(), ctx.scale)
+        return dq, dk, dv, du, dw, None
+
+
+def rfb_attention(q, k, v, u, w, scale=None):
+    s = (1.0 / math.sqrt(q.shape[-1])) if scale is None else float(scale)
+    return RFBAttention.apply(q, k, v, u, w, s)

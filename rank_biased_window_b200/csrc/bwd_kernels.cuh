@@ -1,0 +1,444 @@
+// bwd_kernels.cuh -- backward of O = softmax(s Q K^T + U W^T) V on sm_100a.
+//
+// Chain rule through the same definition (dP = dO V^T, D_i = sum_j P_ij dP_ij,
+// dS = P o (dP - D)):
+//     dQ = s dS K     dU = dS W     dK = s dS^T Q     dW = dS^T U     dV = P^T dO.
+// With U' = U / s staged on chip the bias side rides the same contractions as
+// the content side ("Rank-Factorized Implicit Neural Bias", Abstract:
+// concatenation turns the bias into part of one dot product):
+//     S^T/s = [K | W] . [Q | U']^T         (one accumulation, recompute of P)
+//     [dK | dW] = s dS^T . [Q | U']        (dW = s dS^T U' = dS^T U)
+//     [dQ | dU] = dS . [K | W] with per-column scales (s | 1).
+//
+// Three kernels:
+//   bwd_pre  : D_i = rowsum(dO o O) (equal to sum_j P_ij dP_ij because O = P V),
+//              LSE_i log2(e), and zeroes the fp32 dQ|dU accumulator.
+//   bwd_main : one CTA per (head, 128-key tile); K, W, V stay in shared memory,
+//              dV, dK, dW accumulate in TMEM across all 128-query tiles.  Per
+//              query tile: S^T and dP^T by tcgen05 into TMEM, P^T and dS^T
+//              formed by the compute warps into swizzled shared memory, then
+//              dV, dK, dW (+=) and the partial dQ|dU tile (into the S^T
+//              columns), which the compute warps add into the fp32
+//              accumulator with vector reductions.
+//   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]).
+#pragma once
+#include "fwd_kernels.cuh"
+
+namespace rfb {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdArgs {
+  const __nv_bfloat16* o;     // [BH, N, D]
+  const float* lse;           // [BH, N]
+  const __nv_bfloat16* dout;  // [BH, N, D]
+  float* dvec;                // [BH, Npad]   D_i
+  float* lse2;                // [BH, Npad]   LSE_i * log2(e)
+  float* acc;                 // [BH, N, D + r] fp32 dQ | dU accumulator
+  __nv_bfloat16* dq;          // [BH, N, D]
+  __nv_bfloat16* dk;          // [BH, N, D]
+  __nv_bfloat16* dv;          // [BH, N, D]
+  __nv_bfloat16* du;          // [BH, N, r]
+  __nv_bfloat16* dw;          // [BH, N, r]
+  int* err;
+  int BH, N, Npad, D, r;
+  float scale;       // s
+  float scale_log2;  // s log2(e)
+  float inv_scale;   // 1/s
+  uint64_t timeout_ns;
+};
+
+// ------------------------------------------------------------------ bwd_pre
+// Thread group of G = D/8 lanes per row (16-byte loads); rows grid-strided.
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
+  const int G = a.D / 8;
+  const int rows_per_block = 256 / G;
+  const int sub = threadIdx.x % G;
+  const long total_rows = static_cast<long>(a.BH) * a.Npad;
+  for (long row = static_cast<long>(blockIdx.x) * rows_per_block + threadIdx.x / G; row < total_rows;
+       row += static_cast<long>(gridDim.x) * rows_per_block) {
+    const int bh = static_cast<int>(row / a.Npad);
+    const int i = static_cast<int>(row % a.Npad);
+    float dsum = 0.f, l2 = 0.f;
+    if (i < a.N) {
+      const size_t base = (static_cast<size_t>(bh) * a.N + i) * a.D + sub * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(a.o + base);
+      const uint4 gv = *reinterpret_cast<const uint4*>(a.dout + base);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dsum = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(gw[e] << 16), dsum);
+        dsum = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(gw[e] & 0xFFFF0000u), dsum);
+      }
+      l2 = a.lse[static_cast<size_t>(bh) * a.N + i] * kLog2e;
+    }
+    for (int off = G / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off, G);
+    if (sub == 0) {
+      a.dvec[row] = dsum;
+      a.lse2[row] = l2;
+    }
+  }
+  // Zero the dQ | dU accumulator.
+  const size_t n4 = static_cast<size_t>(a.BH) * a.N * (a.D + a.r) / 4;
+  float4* acc4 = reinterpret_cast<float4*>(a.acc);
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n4;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x)
+    acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ----------------------------------------------------------------- bwd_post
+__global__ void __launch_bounds__(256) bwd_post_kernel(const BwdArgs a) {
+  const int DA = a.D + a.r;
+  const int groups = DA / 8;
+  const long total = static_cast<long>(a.BH) * a.N * groups;
+  for (long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long>(gridDim.x) * blockDim.x) {
+    const long row = t / groups;
+    const int c = static_cast<int>(t % groups) * 8;
+    const float4* src = reinterpret_cast<const float4*>(a.acc + row * DA + c);
+    const float4 x = src[0], y = src[1];
+    uint4 v;
+    v.x = pack_bf16x2(x.x, x.y);
+    v.y = pack_bf16x2(x.z, x.w);
+    v.z = pack_bf16x2(y.x, y.y);
+    v.w = pack_bf16x2(y.z, y.w);
+    if (c < a.D)
+      *reinterpret_cast<uint4*>(a.dq + row * a.D + c) = v;
+    else
+      *reinterpret_cast<uint4*>(a.du + row * a.r + (c - a.D)) = v;
+  }
+}
+
+// Contraction over 128 rows of K-major A (two 64-column blocks, 128-byte
+// swizzle) with an MN-major B whose rows are NN elements wide:
+//     D[128 x NN] (+)= A[128 x 128] . B[128 x NN]
+template <int NN>
+__device__ __forceinline__ void issue_k128(uint32_t d_tmem, uint32_t a, uint32_t b, bool accumulate) {
+  constexpr uint32_t id = idesc_bf16_f32(128, NN, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t ad = desc_kmajor(a + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 128);
+    const uint64_t bd = desc_mnmajor(b + kk * 16 * (NN * 2), NN * 2, 128 * NN * 2);
+    umma_bf16(d_tmem, ad, bd, id, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+// Same contraction with A read transposed: the tile stored for dS^T (rows =
+// keys, queries contiguous) is used as MN-major A = dS (rows = queries).
+template <int NN>
+__device__ __forceinline__ void issue_k128_at(uint32_t d_tmem, uint32_t a, uint32_t b) {
+  constexpr uint32_t id = idesc_bf16_f32(128, NN, true, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t ad = desc_mnmajor(a + kk * 16 * 128, 128, 128 * 128);
+    const uint64_t bd = desc_mnmajor(b + kk * 16 * (NN * 2), NN * 2, 128 * NN * 2);
+    umma_bf16(d_tmem, ad, bd, id, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D, int RP>
+struct BwdCfg {
+  static constexpr int QB = kTile * D * 2;
+  static constexpr int UB = kTile * RP * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = QB;
+  static constexpr int OFF_W = 2 * QB;
+  static constexpr int KVB = 2 * QB + UB;
+  // stage: Q, dO, U, lse2[128], dvec[128]
+  static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UB, S_DV = S_L2 + 512;
+  static constexpr int STAGE = 2 * QB + UB + 1024;
+  static constexpr int PB = kTile * kTile * 2;
+  static constexpr int NS_FIT = (222 * 1024 - KVB - 2 * PB) / STAGE;
+  static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
+  static constexpr int OFF_STAGE = KVB;
+  static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
+  static constexpr int OFF_DS = OFF_P + PB;
+  static constexpr int OFF_BAR = OFF_DS + PB;
+  // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain
+  static constexpr int NBAR = 2 * NS + 6;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  // TMEM columns
+  static constexpr int T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D, T_DW = 256 + 2 * D;
+  static_assert(NS >= 2, "not enough shared memory for two query stages");
+  static_assert(SMEM <= 232448, "shared memory budget exceeded");
+  static_assert(T_DW + RP <= 512 && D + RP <= 128, "TMEM budget");
+};
+
+template <int D, int RP>
+__global__ void __launch_bounds__(192, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                    const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
+                    const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mDO,
+                    const BwdArgs args) {
+  using C = BwdCfg<D, RP>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + C::OFF_BAR;
+  const uint32_t kv_full = bar0;
+  auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto q_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
+  const uint32_t sdp_full = bar0 + 8u * (1 + 2 * NS);
+  const uint32_t ds_full = bar0 + 8u * (2 + 2 * NS);
+  const uint32_t dq_full = bar0 + 8u * (3 + 2 * NS);
+  const uint32_t dq_free = bar0 + 8u * (4 + 2 * NS);
+  const uint32_t drain_bar = bar0 + 8u * (5 + 2 * NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = static_cast<int>(warp_id());
+  const int lane = static_cast<int>(lane_id());
+  const int N = args.N;
+  const int bh = blockIdx.y;
+  const int k0 = blockIdx.x * kTile;
+  const int nq = (N + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+    }
+    mbar_init(sdp_full, 1);
+    mbar_init(ds_full, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch(&mQ);
+    tma_prefetch(&mK);
+    tma_prefetch(&mV);
+    tma_prefetch(&mDO);
+    if constexpr (RP > 0) {
+      tma_prefetch(&mU);
+      tma_prefetch(&mW);
+    }
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard g{abort_flag, args.err, args.timeout_ns};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_expect_tx(kv_full, C::KVB);
+      tma_load_3d(sb + C::OFF_K, &mK, kv_full, 0, k0, bh);
+      tma_load_3d(sb + C::OFF_V, &mV, kv_full, 0, k0, bh);
+      if constexpr (RP > 0) tma_load_3d(sb + C::OFF_W, &mW, kv_full, 0, k0, bh);
+      const float* l2 = args.lse2 + static_cast<size_t>(bh) * args.Npad;
+      const float* dv = args.dvec + static_cast<size_t>(bh) * args.Npad;
+      int i = 0;
+      for (; i < nq; ++i) {
+        const int s = i % NS;
+        if (i >= NS && !wait_bounded(q_empty(s), ((i / NS) + 1) & 1, g, 31)) break;
+        const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+        mbar_expect_tx(q_full(s), C::STAGE);
+        tma_load_3d(st + C::S_Q, &mQ, q_full(s), 0, i * kTile, bh);
+        tma_load_3d(st + C::S_DO, &mDO, q_full(s), 0, i * kTile, bh);
+        if constexpr (RP > 0) tma_load_3d(st + C::S_U, &mU, q_full(s), 0, i * kTile, bh);
+        bulk_load(st + C::S_L2, l2 + i * kTile, 512, q_full(s));
+        bulk_load(st + C::S_DV, dv + i * kTile, 512, q_full(s));
+      }
+      wait_drain(kv_full, 0, args.timeout_ns);
+      for (int j = (i > NS ? i - NS : 0); j < i; ++j)
+        wait_drain(q_full(j % NS), (j / NS) & 1, args.timeout_ns);
+    }
+  } else if (warp == 5) {
+    // ----------------------------------------------------------- MMA issue
+    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+    bool ok = wait_warp(kv_full, 0, g, 32);
+    for (int i = 0; ok && i < nq; ++i) {
+      const int s = i % NS;
+      const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+      if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) break;
+      if constexpr (RP > 0) {
+        scale_tile_bf16(st + C::S_U, C::UB, args.inv_scale);
+        fence_async_smem();
+      }
+      __syncwarp();
+      if (i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        // S^T / s = K Q^T + W U'^T ;  dP^T = V dO^T
+        issue_scores<D, RP>(tmem + C::T_S, sb + C::OFF_K, st + C::S_Q, sb + C::OFF_W, st + C::S_U);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tmem + C::T_DP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2),
+                    desc_kmajor(st + C::S_DO + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
+        umma_commit(sdp_full);
+      }
+      __syncwarp();
+      if (!wait_warp(ds_full, i & 1, g, 35)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t pb = sb + C::OFF_P, dsb = sb + C::OFF_DS;
+        issue_k128<D>(tmem + C::T_DV, pb, st + C::S_DO, i > 0);   // dV += P^T dO
+        issue_k128<D>(tmem + C::T_DK, dsb, st + C::S_Q, i > 0);   // dK += dS^T Q
+        if constexpr (RP > 0) issue_k128<RP>(tmem + C::T_DW, dsb, st + C::S_U, i > 0);  // dW += dS^T U'
+        issue_k128_at<D>(tmem + C::T_S, dsb, sb + C::OFF_K);       // dQ = dS K
+        if constexpr (RP > 0) issue_k128_at<RP>(tmem + C::T_S + D, dsb, sb + C::OFF_W);  // dU = dS W
+        umma_commit(dq_full);
+        umma_commit(q_empty(s));
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      umma_commit(drain_bar);
+      wait_drain(drain_bar, 0, args.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ compute warps
+    const int row = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const bool key_ok = (k0 + row) < N;
+    const float sl2 = args.scale_log2;
+    const int DA = D + args.r;
+    bool ok = true;
+    for (int i = 0; i < nq; ++i) {
+      const int s = i % NS;
+      const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+      if (!wait_warp(q_full(s), (i / NS) & 1, g, 36)) { ok = false; break; }
+      if (!wait_warp(sdp_full, i & 1, g, 37)) { ok = false; break; }
+      tc_fence_after();
+      const float* l2 = reinterpret_cast<const float*>(smem + C::OFF_STAGE + s * C::STAGE + C::S_L2);
+      const float* dvv = reinterpret_cast<const float*>(smem + C::OFF_STAGE + s * C::STAGE + C::S_DV);
+      const int qvalid = N - i * kTile;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {
+        uint32_t x[32], y[32];
+        tmem_ld32(tmem + lane_base + C::T_S + c, x);
+        tmem_ld32(tmem + lane_base + C::T_DP + c, y);
+        float p[32], ds[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int q = c + e;
+          const bool valid = key_ok && (q < qvalid);
+          p[e] = valid ? fast_exp2(fmaf(__uint_as_float(x[e]), sl2, -l2[q])) : 0.f;
+          ds[e] = p[e] * (__uint_as_float(y[e]) - dvv[q]);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          const uint32_t off = sw128_offset(row, c + e, 128);
+          st_shared_v4(sb + C::OFF_P + off, pack_bf16x2(p[e], p[e + 1]), pack_bf16x2(p[e + 2], p[e + 3]),
+                       pack_bf16x2(p[e + 4], p[e + 5]), pack_bf16x2(p[e + 6], p[e + 7]));
+          st_shared_v4(sb + C::OFF_DS + off, pack_bf16x2(ds[e], ds[e + 1]),
+                       pack_bf16x2(ds[e + 2], ds[e + 3]), pack_bf16x2(ds[e + 4], ds[e + 5]),
+                       pack_bf16x2(ds[e + 6], ds[e + 7]));
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+      // Partial dQ | dU of this query tile (TMEM lane = query row).
+      if (!wait_warp(dq_full, i & 1, g, 38)) { ok = false; break; }
+      tc_fence_after();
+      const int q = i * kTile + row;
+      float* accrow = args.acc + (static_cast<size_t>(bh) * N + q) * DA;
+      if constexpr (D == 32) {
+        uint32_t z[32];
+        tmem_ld32(tmem + lane_base + C::T_S, z);
+        if constexpr (RP > 0) {
+          uint32_t zu[RP];
+          tmem_ld_cols<RP>(tmem + lane_base + C::T_S + D, zu);
+          tc_fence_before();
+          mbar_arrive(dq_free);
+          if (q < N) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              red_add_v4(accrow + c, __uint_as_float(z[c]) * args.scale,
+                         __uint_as_float(z[c + 1]) * args.scale, __uint_as_float(z[c + 2]) * args.scale,
+                         __uint_as_float(z[c + 3]) * args.scale);
+#pragma unroll
+            for (int c = 0; c < RP; c += 4)
+              if (c < args.r)
+                red_add_v4(accrow + D + c, __uint_as_float(zu[c]), __uint_as_float(zu[c + 1]),
+                           __uint_as_float(zu[c + 2]), __uint_as_float(zu[c + 3]));
+          }
+        } else {
+          tc_fence_before();
+          mbar_arrive(dq_free);
+          if (q < N) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              red_add_v4(accrow + c, __uint_as_float(z[c]) * args.scale,
+                         __uint_as_float(z[c + 1]) * args.scale, __uint_as_float(z[c + 2]) * args.scale,
+                         __uint_as_float(z[c + 3]) * args.scale);
+          }
+        }
+      } else {
+        // D == 64: two 32-column halves of dQ, then dU.
+        uint32_t z[64];
+        tmem_ld64(tmem + lane_base + C::T_S, z);
+        uint32_t zu[RP > 0 ? RP : 1];
+        if constexpr (RP > 0) tmem_ld_cols<RP>(tmem + lane_base + C::T_S + D, zu);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        if (q < N) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 4)
+            red_add_v4(accrow + c, __uint_as_float(z[c]) * args.scale,
+                       __uint_as_float(z[c + 1]) * args.scale, __uint_as_float(z[c + 2]) * args.scale,
+                       __uint_as_float(z[c + 3]) * args.scale);
+          if constexpr (RP > 0) {
+#pragma unroll
+            for (int c = 0; c < RP; c += 4)
+              if (c < args.r)
+                red_add_v4(accrow + D + c, __uint_as_float(zu[c]), __uint_as_float(zu[c + 1]),
+                           __uint_as_float(zu[c + 2]), __uint_as_float(zu[c + 3]));
+          }
+        }
+      }
+    }
+    if (ok && nq > 0) {
+      // dq_full of the last tile implies all dV, dK, dW MMAs have completed.
+      uint32_t gv[D], gk[D];
+      tmem_ld_cols<D>(tmem + lane_base + C::T_DV, gv);
+      tmem_ld_cols<D>(tmem + lane_base + C::T_DK, gk);
+      if (key_ok) {
+        const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
+        store_o_row<D>(args.dv + r0 * D, gv, 1.0f);
+        store_o_row<D>(args.dk + r0 * D, gk, args.scale);
+      }
+      if constexpr (RP > 0) {
+        uint32_t gw[RP];
+        tmem_ld_cols<RP>(tmem + lane_base + C::T_DW, gw);
+        if (key_ok) {
+          const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
+          uint4* dst = reinterpret_cast<uint4*>(args.dw + r0 * args.r);
+#pragma unroll
+          for (int c = 0; c < RP; c += 8) {
+            if (c < args.r) {
+              const float f = args.scale;
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(gw[c]) * f, __uint_as_float(gw[c + 1]) * f);
+              v.y = pack_bf16x2(__uint_as_float(gw[c + 2]) * f, __uint_as_float(gw[c + 3]) * f);
+              v.z = pack_bf16x2(__uint_as_float(gw[c + 4]) * f, __uint_as_float(gw[c + 5]) * f);
+              v.w = pack_bf16x2(__uint_as_float(gw[c + 6]) * f, __uint_as_float(gw[c + 7]) * f);
+              dst[c >> 3] = v;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace rfb

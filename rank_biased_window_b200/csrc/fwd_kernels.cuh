@@ -1,0 +1,566 @@
+// fwd_kernels.cuh -- forward of attention with an additive rank-factorised bias,
+//
+//     O = softmax(s Q K^T + U W^T) V,   LSE_i = log sum_j exp(S_ij),
+//
+// on sm_100a.  The bias is never materialised: following "Rank-Factorized
+// Implicit Neural Bias" (Abstract: the low-rank bias factors are concatenated
+// with the content channels so the element-wise bias addition becomes part of
+// the dot product), the score tile is ONE tcgen05 accumulation over the
+// concatenated contraction [Q | U'] . [K | W]^T, with U' = U / s staged on chip,
+// so that the accumulator holds S / s and the softmax applies s log2(e).
+// "FlashBias" (Abstract) is the reason this matters: a low-rank bias keeps the
+// fused attention pipeline intact.
+//
+// Two kernels:
+//   * fwd_window_kernel  (N <= 128): persistent CTAs; each 128-row tile packs
+//     128/NP whole windows (NP = 64 or 128 rows per window).  One S tile per
+//     tile, single-pass softmax, block-diagonal P (off-window blocks stay 0).
+//   * fwd_long_kernel    (N > 128): one CTA per (head, 128-query tile); loops
+//     over 128-key tiles with an online softmax (lazy rescale of O in TMEM).
+//
+// Warp roles (192 threads): warps 0-3 softmax + epilogue (thread = row =
+// TMEM lane), warp 4 TMA producer, warp 5 U' scaling + MMA issue (lane 0) +
+// TMEM allocation.  Operands are staged by TMA with the swizzle that matches
+// their row width; P is written by the softmax threads into a 128-byte
+// swizzled K-major tile.
+#pragma once
+#include "sm100.cuh"
+
+namespace rfb {
+
+constexpr int kTile = 128;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct FwdArgs {
+  __nv_bfloat16* o;  // [BH, N, D]
+  float* lse;        // [BH, N]
+  int* err;          // device error word
+  int BH;
+  int N;
+  float scale_log2;  // s * log2(e)
+  float inv_scale;   // 1 / s  (U' = bf16(U / s))
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Bounded wait that ignores the abort flag: used only on the exit path to let
+// in-flight copies and MMAs land before the CTA frees its resources.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) return;
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NC]) {
+  if constexpr (NC == 16) tmem_ld16(taddr, r);
+  else if constexpr (NC == 32) tmem_ld32(taddr, r);
+  else if constexpr (NC == 64) tmem_ld64(taddr, r);
+  else tmem_ld128(taddr, r);
+}
+template <int NC>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[NC]) {
+  if constexpr (NC == 16) tmem_st16(taddr, r);
+  else if constexpr (NC == 32) tmem_st32(taddr, r);
+  else tmem_st64(taddr, r);
+}
+
+// Write one normalised output row (D bf16 values, 16-byte stores).
+template <int D>
+__device__ __forceinline__ void store_o_row(__nv_bfloat16* dst, const uint32_t (&ov)[D], float inv) {
+  uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int c = 0; c < D; c += 8) {
+    uint4 v;
+    v.x = pack_bf16x2(__uint_as_float(ov[c + 0]) * inv, __uint_as_float(ov[c + 1]) * inv);
+    v.y = pack_bf16x2(__uint_as_float(ov[c + 2]) * inv, __uint_as_float(ov[c + 3]) * inv);
+    v.z = pack_bf16x2(__uint_as_float(ov[c + 4]) * inv, __uint_as_float(ov[c + 5]) * inv);
+    v.w = pack_bf16x2(__uint_as_float(ov[c + 6]) * inv, __uint_as_float(ov[c + 7]) * inv);
+    p[c >> 3] = v;
+  }
+}
+
+// Issue the score MMAs  S(tmem) = Q.K^T + U'.W^T  for one 128x128 tile.
+template <int D, int RP>
+__device__ __forceinline__ void issue_scores(uint32_t s_tmem, uint32_t q, uint32_t k, uint32_t u,
+                                             uint32_t w) {
+  constexpr uint32_t id = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    umma_bf16(s_tmem, desc_kmajor(q + kk * 32, D * 2), desc_kmajor(k + kk * 32, D * 2), id,
+              kk > 0 ? 1u : 0u);
+#pragma unroll
+  for (int kk = 0; kk < RP / 16; ++kk)
+    umma_bf16(s_tmem, desc_kmajor(u + kk * 32, RP * 2), desc_kmajor(w + kk * 32, RP * 2), id, 1u);
+}
+
+// Issue O(tmem) (+)= P . V for a 128-key tile; P is K-major in two 64-key
+// column blocks of 128 rows, V is MN-major (rows = keys, D contiguous).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p, uint32_t v, bool accumulate) {
+  constexpr uint32_t id = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t ad = desc_kmajor(p + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 128);
+    const uint64_t bd = desc_mnmajor(v + kk * 16 * (D * 2), D * 2, 128 * D * 2);
+    umma_bf16(o_tmem, ad, bd, id, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// ============================================================ window regime
+template <int D, int RP, int NP>
+struct WinCfg {
+  static constexpr int NW = kTile / NP;       // windows packed per tile
+  static constexpr int QB = kTile * D * 2;    // bytes of a Q / K / V tile
+  static constexpr int UB = kTile * RP * 2;   // bytes of a U / W tile
+  static constexpr int STAGE = 3 * QB + 2 * UB;
+  static constexpr int PB = kTile * kTile * 2;
+  static constexpr int NS_FIT = (224 * 1024 - 2 * PB) / STAGE;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static constexpr int OFF_P = NS * STAGE;
+  static constexpr int OFF_BAR = OFF_P + 2 * PB;
+  // in_full[NS] in_empty[NS] s_full[2] p_full[2] o_full[2] acc_empty[2] drain
+  static constexpr int NBAR = 2 * NS + 9;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static_assert(NS >= 2, "not enough shared memory for two input stages");
+  static_assert(SMEM <= 232448, "shared memory budget exceeded");
+  static_assert(QB % 1024 == 0 && UB % 1024 == 0, "tile alignment");
+};
+
+template <int D, int RP, int NP>
+__global__ void __launch_bounds__(192, 1)
+    fwd_window_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                      const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
+                      const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
+  using C = WinCfg<D, RP, NP>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + C::OFF_BAR;
+  auto in_full = [&](int s) { return bar0 + 8u * s; };
+  auto in_empty = [&](int s) { return bar0 + 8u * (NS + s); };
+  auto s_full = [&](int a) { return bar0 + 8u * (2 * NS + a); };
+  auto p_full = [&](int a) { return bar0 + 8u * (2 * NS + 2 + a); };
+  auto o_full = [&](int a) { return bar0 + 8u * (2 * NS + 4 + a); };
+  auto acc_empty = [&](int a) { return bar0 + 8u * (2 * NS + 6 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * NS + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = static_cast<int>(warp_id());
+  const int lane = static_cast<int>(lane_id());
+  const int num_tiles = (args.BH + C::NW - 1) / C::NW;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(in_full(s), 1);
+      mbar_init(in_empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(s_full(a), 1);
+      mbar_init(p_full(a), 128);
+      mbar_init(o_full(a), 1);
+      mbar_init(acc_empty(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch(&mQ);
+    tma_prefetch(&mK);
+    tma_prefetch(&mV);
+    if constexpr (RP > 0) {
+      tma_prefetch(&mU);
+      tma_prefetch(&mW);
+    }
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp < 4) {
+    // P buffers start at zero: with NP = 64 each row only ever writes its own
+    // window's 64-key block, so the other block stays zero (block-diagonal P).
+    for (int off = threadIdx.x * 16; off < 2 * C::PB; off += 128 * 16)
+      st_shared_v4(sb + C::OFF_P + off, 0u, 0u, 0u, 0u);
+    fence_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard g{abort_flag, args.err, args.timeout_ns};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        const int s = it % NS;
+        if (it >= NS && !wait_bounded(in_empty(s), ((it / NS) + 1) & 1, g, 1)) break;
+        const uint32_t st = sb + s * C::STAGE;
+        mbar_expect_tx(in_full(s), C::STAGE);
+        const int w0 = t * C::NW;
+        tma_load_3d(st, &mQ, in_full(s), 0, 0, w0);
+        tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
+        tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
+        if constexpr (RP > 0) {
+          tma_load_3d(st + 3 * C::QB, &mU, in_full(s), 0, 0, w0);
+          tma_load_3d(st + 3 * C::QB + C::UB, &mW, in_full(s), 0, 0, w0);
+        }
+      }
+      // Let the last copies land before the CTA can exit.
+      for (int j = (it > NS ? it - NS : 0); j < it; ++j)
+        wait_drain(in_full(j % NS), (j / NS) & 1, args.timeout_ns);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------- U' scaling + MMA issue
+    bool ok = true;
+    auto do_pv = [&](int j) -> bool {
+      const int a = j & 1, s = j % NS;
+      if (!wait_warp(p_full(a), (j >> 1) & 1, g, 3)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        issue_pv<D>(tmem + 256 + a * D, sb + C::OFF_P + a * C::PB, sb + s * C::STAGE + 2 * C::QB,
+                    false);
+        umma_commit(o_full(a));
+        umma_commit(in_empty(s));
+      }
+      __syncwarp();
+      return true;
+    };
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int s = it % NS, a = it & 1;
+      if (!wait_warp(in_full(s), (it / NS) & 1, g, 2)) { ok = false; break; }
+      const uint32_t st = sb + s * C::STAGE;
+      if constexpr (RP > 0) {
+        scale_tile_bf16(st + 3 * C::QB, C::UB, args.inv_scale);
+        fence_async_smem();
+      }
+      __syncwarp();
+      if (it >= 2 && !wait_warp(acc_empty(a), ((it >> 1) + 1) & 1, g, 4)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        issue_scores<D, RP>(tmem + a * 128, st, st + C::QB, st + 3 * C::QB, st + 3 * C::QB + C::UB);
+        umma_commit(s_full(a));
+      }
+      __syncwarp();
+      if (it > 0 && !do_pv(it - 1)) { ok = false; break; }
+    }
+    if (ok && it > 0) do_pv(it - 1);
+    if (lane == 0) {
+      umma_commit(drain_bar);
+      wait_drain(drain_bar, 0, args.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int row = threadIdx.x;  // TMEM lane == tile row
+    const int wl = row / NP;      // window inside the tile
+    const int n = row % NP;       // token inside the window
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int N = args.N;
+    const float sl2 = args.scale_log2;
+
+    auto epilogue = [&](int j, int t, float m, float l) -> bool {
+      const int a = j & 1;
+      if (!wait_warp(o_full(a), (j >> 1) & 1, g, 6)) return false;
+      tc_fence_after();
+      uint32_t ov[D];
+      tmem_ld_cols<D>(tmem + lane_base + 256 + a * D, ov);
+      tc_fence_before();
+      mbar_arrive(acc_empty(a));
+      const int win = t * C::NW + wl;
+      if (win < args.BH && n < N) {
+        const size_t r = static_cast<size_t>(win) * N + n;
+        store_o_row<D>(args.o + r * D, ov, 1.0f / l);
+        args.lse[r] = (m + __log2f(l)) * kLn2;
+      }
+      return true;
+    };
+
+    bool ok = true;
+    int it = 0, t_prev = 0;
+    float m_prev = 0.f, l_prev = 1.f;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int a = it & 1;
+      if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[NP];
+      tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j < N) mx = fmaxf(mx, __uint_as_float(sv[j]));
+      const float m = mx * sl2;
+      float l = 0.f;
+      const uint32_t pbuf = sb + C::OFF_P + a * C::PB;
+#pragma unroll
+      for (int c = 0; c < NP; c += 8) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = c + e;
+          p[e] = (j < N) ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -m)) : 0.f;
+          l += p[e];
+        }
+        st_shared_v4(pbuf + sw128_offset(row, wl * NP + c, 128), pack_bf16x2(p[0], p[1]),
+                     pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full(a));
+      if (it > 0 && !epilogue(it - 1, t_prev, m_prev, l_prev)) { ok = false; break; }
+      m_prev = m;
+      l_prev = l;
+      t_prev = t;
+    }
+    if (ok && it > 0) epilogue(it - 1, t_prev, m_prev, l_prev);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================== long regime
+template <int D, int RP>
+struct LongCfg {
+  static constexpr int QB = kTile * D * 2;
+  static constexpr int UB = kTile * RP * 2;
+  static constexpr int STAGE = 2 * QB + UB;  // K, V, W
+  static constexpr int PB = kTile * kTile * 2;
+  static constexpr int NS_FIT = (200 * 1024 - 2 * PB - QB - UB) / STAGE;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_U = QB;
+  static constexpr int OFF_STAGE = QB + UB;
+  static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
+  static constexpr int OFF_BAR = OFF_P + 2 * PB;
+  // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
+  static constexpr int NBAR = 2 * NS + 10;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static_assert(NS >= 2, "not enough shared memory for two KV stages");
+  static_assert(SMEM <= 232448, "shared memory budget exceeded");
+};
+
+template <int D, int RP>
+__global__ void __launch_bounds__(192, 1)
+    fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                    const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
+                    const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
+  using C = LongCfg<D, RP>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + C::OFF_BAR;
+  const uint32_t q_full = bar0;
+  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (1 + 2 * NS + b); };
+  auto s_empty = [&](int b) { return bar0 + 8u * (3 + 2 * NS + b); };
+  auto p_full = [&](int b) { return bar0 + 8u * (5 + 2 * NS + b); };
+  auto pv_done = [&](int b) { return bar0 + 8u * (7 + 2 * NS + b); };
+  const uint32_t drain_bar = bar0 + 8u * (9 + 2 * NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = static_cast<int>(warp_id());
+  const int lane = static_cast<int>(lane_id());
+  const int N = args.N;
+  const int bh = blockIdx.y;
+  const int q0 = blockIdx.x * kTile;
+  const int nkv = (N + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full(b), 1);
+      mbar_init(s_empty(b), 128);
+      mbar_init(p_full(b), 128);
+      mbar_init(pv_done(b), 1);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch(&mQ);
+    tma_prefetch(&mK);
+    tma_prefetch(&mV);
+    if constexpr (RP > 0) {
+      tma_prefetch(&mU);
+      tma_prefetch(&mW);
+    }
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard g{abort_flag, args.err, args.timeout_ns};
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_expect_tx(q_full, C::QB + C::UB);
+      tma_load_3d(sb + C::OFF_Q, &mQ, q_full, 0, q0, bh);
+      if constexpr (RP > 0) tma_load_3d(sb + C::OFF_U, &mU, q_full, 0, q0, bh);
+      int j = 0;
+      for (; j < nkv; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !wait_bounded(kv_empty(s), ((j / NS) + 1) & 1, g, 11)) break;
+        const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+        mbar_expect_tx(kv_full(s), C::STAGE);
+        tma_load_3d(st, &mK, kv_full(s), 0, j * kTile, bh);
+        tma_load_3d(st + C::QB, &mV, kv_full(s), 0, j * kTile, bh);
+        if constexpr (RP > 0) tma_load_3d(st + 2 * C::QB, &mW, kv_full(s), 0, j * kTile, bh);
+      }
+      wait_drain(q_full, 0, args.timeout_ns);
+      for (int i = (j > NS ? j - NS : 0); i < j; ++i)
+        wait_drain(kv_full(i % NS), (i / NS) & 1, args.timeout_ns);
+    }
+  } else if (warp == 5) {
+    bool ok = wait_warp(q_full, 0, g, 12);
+    if (ok) {
+      if constexpr (RP > 0) {
+        scale_tile_bf16(sb + C::OFF_U, C::UB, args.inv_scale);
+        fence_async_smem();
+      }
+      __syncwarp();
+    }
+    auto do_s = [&](int j) -> bool {
+      const int s = j % NS, b = j & 1;
+      if (!wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
+      if (j >= 2 && !wait_warp(s_empty(b), ((j >> 1) + 1) & 1, g, 14)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+        issue_scores<D, RP>(tmem + b * 128, sb + C::OFF_Q, st, sb + C::OFF_U, st + 2 * C::QB);
+        umma_commit(s_full(b));
+      }
+      __syncwarp();
+      return true;
+    };
+    auto do_pv = [&](int j) -> bool {
+      const int s = j % NS, b = j & 1;
+      if (!wait_warp(p_full(b), (j >> 1) & 1, g, 15)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        issue_pv<D>(tmem + 256, sb + C::OFF_P + b * C::PB, sb + C::OFF_STAGE + s * C::STAGE + C::QB,
+                    j > 0);
+        umma_commit(kv_empty(s));
+        umma_commit(pv_done(b));
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ok) ok = do_s(0);
+    for (int j = 0; ok && j < nkv; ++j) {
+      if (j + 1 < nkv && !do_s(j + 1)) break;
+      if (!do_pv(j)) break;
+    }
+    if (lane == 0) {
+      umma_commit(drain_bar);
+      wait_drain(drain_bar, 0, args.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    const int row = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = args.scale_log2;
+    float m_run = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int b = j & 1;
+      if (!wait_warp(s_full(b), (j >> 1) & 1, g, 16)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[128];
+      tmem_ld_cols<128>(tmem + lane_base + b * 128, sv);
+      tc_fence_before();
+      mbar_arrive(s_empty(b));
+      const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (c < kvalid) mx = fmaxf(mx, __uint_as_float(sv[c]));
+      const float m_new = fmaxf(m_run, mx * sl2);
+      // Lazy rescale: keep the running max unless it grew by more than 2^8.
+      const bool need = m_new > m_run + 8.0f;
+      float alpha = 1.f;
+      if (need) {
+        alpha = fast_exp2(m_run - m_new);
+        l *= alpha;
+        m_run = m_new;
+      }
+      const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
+      if (j >= 2 && !wait_warp(pv_done(b), ((j >> 1) + 1) & 1, g, 17)) { ok = false; break; }
+      const uint32_t pbuf = sb + C::OFF_P + b * C::PB;
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = (c + e < kvalid) ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m_run)) : 0.f;
+          l += p[e];
+        }
+        st_shared_v4(pbuf + sw128_offset(row, c, 128), pack_bf16x2(p[0], p[1]),
+                     pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+      }
+      if (fix_o) {
+        // O holds the sum through tile j-1 at the old running max: wait for that
+        // PV to land, then rescale this thread's row in place.
+        if (!wait_warp(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, g, 18)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t ov[D];
+        tmem_ld_cols<D>(tmem + lane_base + 256, ov);
+#pragma unroll
+        for (int c = 0; c < D; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+        tmem_st_cols<D>(tmem + lane_base + 256, ov);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full(b));
+    }
+    if (ok) {
+      const int jl = nkv - 1;
+      if (wait_warp(pv_done(jl & 1), (jl >> 1) & 1, g, 19)) {
+        tc_fence_after();
+        uint32_t ov[D];
+        tmem_ld_cols<D>(tmem + lane_base + 256, ov);
+        const int q = q0 + row;
+        if (q < N) {
+          const size_t r = static_cast<size_t>(bh) * N + q;
+          store_o_row<D>(args.o + r * D, ov, 1.0f / l);
+          args.lse[r] = (m_run + __log2f(l)) * kLn2;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace rfb

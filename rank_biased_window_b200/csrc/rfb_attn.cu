@@ -1,0 +1,517 @@
+// rfb_attn.cu -- host side of the C ABI declared in include/rfb_attn.h:
+// argument checks, TMA tensor-map encoding, kernel selection and launch.
+//
+// The library allocates no device memory and never synchronises on the
+// caller's stream; everything after the argument checks is an asynchronous
+// launch on `stream`.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "rfb_attn.h"
+#include "bwd_kernels.cuh"
+#include "fwd_kernels.cuh"
+
+namespace rfb {
+
+// Device error word, one per device context.
+__device__ int g_err_word = 0;
+
+__global__ void selftest_wait_kernel(int* err, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitGuard g{&abort_flag, err, timeout_ns};
+    wait_bounded(smem_u32(&bar), 0, g, 99);  // nothing ever arrives on this barrier
+  }
+  __syncthreads();
+}
+
+namespace {
+
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr int kMaxDevices = 64;
+
+// Last failing CUDA call (error code and the site that saw it), for diagnostics.
+std::atomic<int> g_last_cuda_err{0};
+std::atomic<int> g_last_cuda_site{0};
+
+enum CudaSite {
+  kSiteGetDevice = 1, kSiteAttribute = 2, kSiteSymbol = 3, kSiteEncoder = 4, kSiteEncode = 5,
+  kSiteFuncAttr = 6, kSiteLaunch = 7, kSiteSync = 8
+};
+
+int cuda_fail(int err, int site) {
+  g_last_cuda_err.store(err);
+  g_last_cuda_site.store(site);
+  return RFB_ERR_CUDA;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int* err_word = nullptr;
+};
+
+int device_info(DeviceInfo* out) {
+  static DeviceInfo cache[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail(e, kSiteGetDevice);
+  // Binds this host thread to the device's primary context in this library's
+  // runtime (a no-op when already bound); callers may come from any thread.
+  if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e, kSiteGetDevice);
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& d = cache[dev];
+  if (d.sms == 0) {
+    int sms = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, kSiteAttribute);
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_err_word)) != cudaSuccess) return cuda_fail(e, kSiteSymbol);
+    d.err_word = static_cast<int*>(p);
+    d.sms = sms;
+  }
+  *out = d;
+  return RFB_OK;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev >= kMaxDevices) return cuda_fail(e, kSiteGetDevice);
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return RFB_OK;
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) !=
+      cudaSuccess)
+    return cuda_fail(e, kSiteFuncAttr);
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return RFB_OK;
+}
+
+CUtensorMapSwizzle swizzle_for(int row_bytes) {
+  switch (row_bytes) {
+    case 128: return CU_TENSOR_MAP_SWIZZLE_128B;
+    case 64: return CU_TENSOR_MAP_SWIZZLE_64B;
+    default: return CU_TENSOR_MAP_SWIZZLE_32B;
+  }
+}
+
+// 3-D bf16 map over a contiguous [BH, N, cols] tensor.  The box is
+// (box_cols, box_rows, box_heads); box_cols may exceed cols (zero fill).
+int encode_3d(CUtensorMap* m, const void* ptr, int cols, int N, int BH, int box_cols, int box_rows,
+              int box_heads) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return cuda_fail(0, kSiteEncoder);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
+                                 static_cast<cuuint64_t>(cols) * 2 * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows),
+                             static_cast<cuuint32_t>(box_heads)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult rc = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle_for(box_cols * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? RFB_OK : cuda_fail(static_cast<int>(rc), kSiteEncode);
+}
+
+int pad_rank(int r) { return r == 0 ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared shape / scalar checks.  Returns RFB_OK, or an error; *empty is set
+// when there is nothing to compute.
+int check_shape(int B, int H, int N, int d, int r, float scale, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0 || d < 0 || r < 0) return RFB_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return RFB_ERR_INVALID_ARG;
+  if (d != 32 && d != 64) return RFB_ERR_UNSUPPORTED;
+  if (r > 64 || (r % 8) != 0) return RFB_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) {
+    *empty = true;
+    return RFB_OK;
+  }
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 0x7fffffffLL) return RFB_ERR_UNSUPPORTED;
+  if (bh * N * (d + r) > (1LL << 40)) return RFB_ERR_UNSUPPORTED;
+  return RFB_OK;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RFB_OK : cuda_fail(e, kSiteLaunch);
+}
+
+// ------------------------------------------------------- per-kernel timing
+enum KernelId { kIdFwd = 0, kIdBwdPre = 1, kIdBwdMain = 2, kIdBwdPost = 3 };
+
+struct Profiler {
+  std::atomic<bool> on{false};
+  std::mutex mu;
+  struct Rec {
+    int id;
+    cudaEvent_t a, b;
+  };
+  Rec recs[8192];
+  int n = 0;
+  cudaEvent_t pool[16384];
+  int pool_n = 0;
+
+  cudaEvent_t get() {
+    if (pool_n > 0) return pool[--pool_n];
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void put(cudaEvent_t e) {
+    if (pool_n < 16384) pool[pool_n++] = e;
+    else cudaEventDestroy(e);
+  }
+};
+Profiler g_prof;
+
+// RAII bracket around one launch; records nothing when profiling is off.
+struct LaunchTimer {
+  int id;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  LaunchTimer(int kid, cudaStream_t s) : id(kid), st(s) {
+    if (!g_prof.on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    a = g_prof.get();
+    if (a) cudaEventRecord(a, st);
+  }
+  ~LaunchTimer() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    cudaEvent_t b = g_prof.get();
+    if (!b) return;
+    cudaEventRecord(b, st);
+    if (g_prof.n < 8192) g_prof.recs[g_prof.n++] = {id, a, b};
+  }
+};
+
+struct Maps {
+  CUtensorMap q, k, v, u, w, g;
+};
+
+// ---------------------------------------------------------------- forward
+template <int D, int RP, int NP>
+int launch_window(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
+  using C = WinCfg<D, RP, NP>;
+  static std::atomic<uint64_t> done{0};
+  if (int rc = ensure_smem(fwd_window_kernel<D, RP, NP>, C::SMEM, done)) return rc;
+  const int tiles = (a.BH + C::NW - 1) / C::NW;
+  const int grid = tiles < sms ? tiles : sms;
+  LaunchTimer timer(kIdFwd, st);
+  fwd_window_kernel<D, RP, NP><<<grid, 192, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  return launch_status();
+}
+
+template <int D, int RP>
+int launch_long(const Maps& m, const FwdArgs& a, cudaStream_t st) {
+  using C = LongCfg<D, RP>;
+  static std::atomic<uint64_t> done{0};
+  if (int rc = ensure_smem(fwd_long_kernel<D, RP>, C::SMEM, done)) return rc;
+  const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
+  LaunchTimer timer(kIdFwd, st);
+  fwd_long_kernel<D, RP><<<grid, 192, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  return launch_status();
+}
+
+template <int D, int RP>
+int dispatch_fwd(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
+  if (a.N <= 64) return launch_window<D, RP, 64>(m, a, sms, st);
+  if (a.N <= 128) return launch_window<D, RP, 128>(m, a, sms, st);
+  return launch_long<D, RP>(m, a, st);
+}
+
+int dispatch_fwd_rp(int d, int rp, const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
+#define RFB_FWD_CASE(DD, RR) \
+  if (d == DD && rp == RR) return dispatch_fwd<DD, RR>(m, a, sms, st);
+  RFB_FWD_CASE(32, 0) RFB_FWD_CASE(32, 16) RFB_FWD_CASE(32, 32) RFB_FWD_CASE(32, 64)
+  RFB_FWD_CASE(64, 0) RFB_FWD_CASE(64, 16) RFB_FWD_CASE(64, 32) RFB_FWD_CASE(64, 64)
+#undef RFB_FWD_CASE
+  return RFB_ERR_UNSUPPORTED;
+}
+
+// --------------------------------------------------------------- backward
+struct WsLayout {
+  size_t dvec, lse2, acc, total;
+  int npad;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(int B, int H, int N, int d, int r) {
+  WsLayout L{};
+  const size_t bh = static_cast<size_t>(B) * H;
+  L.npad = (N + kTile - 1) / kTile * kTile;
+  const size_t vec = align256(bh * L.npad * sizeof(float));
+  L.dvec = 0;
+  L.lse2 = vec;
+  L.acc = 2 * vec;
+  L.total = L.acc + align256(bh * N * static_cast<size_t>(d + r) * sizeof(float));
+  return L;
+}
+
+template <int D, int RP>
+int launch_bwd_main(const Maps& m, const BwdArgs& a, cudaStream_t st) {
+  using C = BwdCfg<D, RP>;
+  static std::atomic<uint64_t> done{0};
+  if (int rc = ensure_smem(bwd_main_kernel<D, RP>, C::SMEM, done)) return rc;
+  const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
+  LaunchTimer timer(kIdBwdMain, st);
+  bwd_main_kernel<D, RP><<<grid, 192, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, m.g, a);
+  return launch_status();
+}
+
+int dispatch_bwd_main(int d, int rp, const Maps& m, const BwdArgs& a, cudaStream_t st) {
+#define RFB_BWD_CASE(DD, RR) \
+  if (d == DD && rp == RR) return launch_bwd_main<DD, RR>(m, a, st);
+  RFB_BWD_CASE(32, 0) RFB_BWD_CASE(32, 16) RFB_BWD_CASE(32, 32) RFB_BWD_CASE(32, 64)
+  RFB_BWD_CASE(64, 0) RFB_BWD_CASE(64, 16) RFB_BWD_CASE(64, 32) RFB_BWD_CASE(64, 64)
+#undef RFB_BWD_CASE
+  return RFB_ERR_UNSUPPORTED;
+}
+
+int grid_for(long long work, int per_block, int sms) {
+  long long g = (work + per_block - 1) / per_block;
+  const long long cap = static_cast<long long>(sms) * 8;
+  if (g > cap) g = cap;
+  return g < 1 ? 1 : static_cast<int>(g);
+}
+
+}  // namespace
+}  // namespace rfb
+
+using namespace rfb;
+
+extern "C" {
+
+int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, const void* w,
+                 void* o, float* lse, int B, int H, int N, int d, int r, float scale,
+                 void* stream) {
+  bool empty = false;
+  if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
+  if (empty) return RFB_OK;
+  if (!q || !k || !v || !o || !lse || (r > 0 && (!u || !w))) return RFB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (r > 0 && (!aligned16(u) || !aligned16(w))))
+    return RFB_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  const int BH = B * H;
+  const int rp = pad_rank(r);
+  Maps m;
+  std::memset(&m, 0, sizeof(m));
+  int rows = kTile, heads = 1;
+  if (N <= 64) {
+    rows = 64;
+    heads = 2;
+  }
+  int rc = encode_3d(&m.q, q, d, N, BH, d, rows, heads);
+  if (!rc) rc = encode_3d(&m.k, k, d, N, BH, d, rows, heads);
+  if (!rc) rc = encode_3d(&m.v, v, d, N, BH, d, rows, heads);
+  if (!rc && r > 0) rc = encode_3d(&m.u, u, r, N, BH, rp, rows, heads);
+  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, rows, heads);
+  if (rc) return rc;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.err = dev.err_word;
+  a.BH = BH;
+  a.N = N;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.inv_scale = 1.0f / scale;
+  a.timeout_ns = kWaitTimeoutNs;
+  return dispatch_fwd_rp(d, rp, m, a, dev.sms, static_cast<cudaStream_t>(stream));
+}
+
+size_t rfb_attn_bwd_workspace_size(int B, int H, int N, int d, int r) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, r, 1.0f, &empty) != RFB_OK || empty) return 0;
+  return ws_layout(B, H, N, d, r).total;
+}
+
+int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, const void* w,
+                 const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                 void* du, void* dw, void* workspace, size_t workspace_bytes, int B, int H,
+                 int N, int d, int r, float scale, void* stream) {
+  bool empty = false;
+  if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
+  if (empty) return RFB_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv ||
+      (r > 0 && (!u || !w || !du || !dw)))
+    return RFB_ERR_INVALID_ARG;
+  const void* all[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void* p : all)
+    if (!aligned16(p)) return RFB_ERR_ALIGNMENT;
+  if (r > 0 && (!aligned16(u) || !aligned16(w) || !aligned16(du) || !aligned16(dw)))
+    return RFB_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(B, H, N, d, r);
+  if (!workspace || workspace_bytes < L.total) return RFB_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return RFB_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  const int BH = B * H;
+  const int rp = pad_rank(r);
+  Maps m;
+  std::memset(&m, 0, sizeof(m));
+  int rc = encode_3d(&m.q, q, d, N, BH, d, kTile, 1);
+  if (!rc) rc = encode_3d(&m.k, k, d, N, BH, d, kTile, 1);
+  if (!rc) rc = encode_3d(&m.v, v, d, N, BH, d, kTile, 1);
+  if (!rc) rc = encode_3d(&m.g, dout, d, N, BH, d, kTile, 1);
+  if (!rc && r > 0) rc = encode_3d(&m.u, u, r, N, BH, rp, kTile, 1);
+  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, kTile, 1);
+  if (rc) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdArgs a;
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.lse = lse;
+  a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.dvec = reinterpret_cast<float*>(ws + L.dvec);
+  a.lse2 = reinterpret_cast<float*>(ws + L.lse2);
+  a.acc = reinterpret_cast<float*>(ws + L.acc);
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.du = static_cast<__nv_bfloat16*>(du);
+  a.dw = static_cast<__nv_bfloat16*>(dw);
+  a.err = dev.err_word;
+  a.BH = BH;
+  a.N = N;
+  a.Npad = L.npad;
+  a.D = d;
+  a.r = r;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.inv_scale = 1.0f / scale;
+  a.timeout_ns = kWaitTimeoutNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long rows = static_cast<long long>(BH) * L.npad;
+  {
+    LaunchTimer timer(kIdBwdPre, st);
+    bwd_pre_kernel<<<grid_for(rows, 256 / (d / 8), dev.sms), 256, 0, st>>>(a);
+  }
+  if ((rc = launch_status())) return rc;
+  if ((rc = dispatch_bwd_main(d, rp, m, a, st))) return rc;
+  const long long groups = static_cast<long long>(BH) * N * ((d + r) / 8);
+  {
+    LaunchTimer timer(kIdBwdPost, st);
+    bwd_post_kernel<<<grid_for(groups, 256, dev.sms), 256, 0, st>>>(a);
+  }
+  return launch_status();
+}
+
+const char* rfb_strerror(int status) {
+  switch (status) {
+    case RFB_OK: return "success";
+    case RFB_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or non-finite scale)";
+    case RFB_ERR_UNSUPPORTED: return "unsupported shape (d must be 32 or 64; r a multiple of 8 in [0, 64])";
+    case RFB_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case RFB_ERR_WORKSPACE: return "workspace missing or too small";
+    case RFB_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case RFB_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    default: return "unknown status";
+  }
+}
+
+int rfb_last_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -RFB_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(int)) != cudaSuccess) return -RFB_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return -RFB_ERR_CUDA;
+  return v;
+}
+
+int rfb_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      dev.err_word, static_cast<uint64_t>(timeout_us) * 1000ull);
+  return launch_status();
+}
+
+int rfb_profile_enable(int on) {
+  g_prof.on.store(on != 0, std::memory_order_relaxed);
+  return RFB_OK;
+}
+
+int rfb_profile_read(float* ms, int* launches) {
+  if (!ms || !launches) return RFB_ERR_INVALID_ARG;
+  for (int i = 0; i < RFB_PROFILE_KERNELS; ++i) {
+    ms[i] = 0.f;
+    launches[i] = 0;
+  }
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  int rc = RFB_OK;
+  for (int i = 0; i < g_prof.n; ++i) {
+    Profiler::Rec& r = g_prof.recs[i];
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      rc = RFB_ERR_CUDA;
+    if (r.id >= 0 && r.id < RFB_PROFILE_KERNELS) {
+      ms[r.id] += t;
+      launches[r.id] += 1;
+    }
+    g_prof.put(r.a);
+    g_prof.put(r.b);
+  }
+  g_prof.n = 0;
+  return rc;
+}
+
+const char* rfb_profile_kernel_name(int id) {
+  switch (id) {
+    case kIdFwd: return "fwd";
+    case kIdBwdPre: return "bwd_pre";
+    case kIdBwdMain: return "bwd_main";
+    case kIdBwdPost: return "bwd_post";
+    default: return "unknown";
+  }
+}
+
+int rfb_last_cuda_error(int* site) {
+  if (site) *site = g_last_cuda_site.load();
+  return g_last_cuda_err.load();
+}
+
+const char* rfb_version(void) { return "rfb_attn 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,83 @@
+"""The C-ABI library builds, loads and exports every symbol its header declares;
+host-side argument checks work without a GPU (no compute call is made: every
+case here is rejected before anything touches the device)."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                names += re.findall(r"RFB_API\s+[\w\s\*]+?\b(rfb_\w+)\s*\(", f.read())
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for want in ("rfb_attn_fwd", "rfb_attn_bwd", "rfb_attn_bwd_workspace_size", "rfb_strerror",
+                 "rfb_last_device_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(rfb_lib):
+    lib = rfb_lib.load_library()
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    from rank_biased_window_b200.binding import SIGNATURES
+    assert set(SIGNATURES) == set(_declared_symbols())
+
+
+def test_strerror_and_version(rfb_lib):
+    lib = rfb_lib.load_library()
+    assert lib.rfb_version().decode().startswith("rfb_attn")
+    assert "success" in lib.rfb_strerror(0).decode()
+    for code in range(1, 7):
+        assert lib.rfb_strerror(code).decode() != "unknown status"
+    assert lib.rfb_strerror(99).decode() == "unknown status"
+
+
+def test_host_side_argument_checks(rfb_lib):
+    lib = rfb_lib.load_library()
+    n = None
+    # empty problems are no-ops, whatever the pointers
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 0, 4, 64, 32, 8, 0.1, n) == 0
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 2, 4, 0, 32, 8, 0.1, n) == 0
+    # unsupported d / r
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 48, 8, 0.1, n) == 2
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 128, 8, 0.1, n) == 2
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 7, 0.1, n) == 2
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 72, 0.1, n) == 2
+    # null pointers, negative sizes, non-finite scale
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, 0.1, n) == 1
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, -1, 1, 64, 32, 8, 0.1, n) == 1
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, float("inf"), n) == 1
+    assert lib.rfb_attn_bwd(*([n] * 14), 0, 1, 1, 64, 32, 8, 0.1, n) == 1
+
+
+def test_workspace_size(rfb_lib):
+    lib = rfb_lib.load_library()
+    assert lib.rfb_attn_bwd_workspace_size(0, 1, 64, 32, 8) == 0
+    assert lib.rfb_attn_bwd_workspace_size(1, 1, 64, 48, 8) == 0
+    B, H, N, d, r = 2, 8, 16384, 64, 32
+    ws = lib.rfb_attn_bwd_workspace_size(B, H, N, d, r)
+    # two fp32 row vectors (padded to 128 rows) + the fp32 dQ|dU accumulator
+    assert ws >= B * H * N * (d + r) * 4 + 2 * B * H * N * 4
+    assert ws < B * H * N * (d + r) * 4 + 2 * B * H * (N + 128) * 4 + 1024
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from rank_biased_window_b200 import binding
+    # a fresh loader pointed at a missing file must raise, never fall back
+    saved = binding._lib
+    try:
+        binding._lib = None
+        with pytest.raises(RuntimeError, match="not built"):
+            binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        binding._lib = saved
