@@ -99,6 +99,42 @@ RFB_API int rfb_attn_bwd(const void* q, const void* k, const void* v, const void
                  void* du, void* dw, void* workspace, size_t workspace_bytes, int B, int H,
                  int N, int d, int r, float scale, void* stream);
 
+/*
+ * Backward that allocates nothing (the pages have no counterpart; this is an
+ * integration aid).  Same inputs, outputs and results as rfb_attn_bwd, but
+ * without the workspace argument: the scratch the backward needs (per-row
+ * statistics and the fp32 dQ|dU accumulator) lives in one fixed array of
+ * RFB_NOALLOC_SCRATCH_BYTES bytes compiled into the library.
+ *
+ * Who it is for: callers that may not allocate device memory while they run
+ * and have no workspace to lend -- for example a serving runtime that carves
+ * up all device memory when it starts and forbids cudaMalloc afterwards, or a
+ * plugin host that owns the allocator and hands its plugins nothing but their
+ * input and output buffers.
+ *
+ * Limit: a problem whose rfb_attn_bwd_workspace_size() exceeds
+ * RFB_NOALLOC_SCRATCH_BYTES (about B*H*N*(d+r) > 8 M elements) is rejected with
+ * RFB_ERR_WORKSPACE before anything is enqueued.  The call makes no cudaMalloc,
+ * cudaFree or other allocating call.
+ *
+ * Cost: every GPU on which this library's kernels are loaded keeps the array
+ * until the process exits.
+ *
+ * First call on a device: it looks up the array's device address with that
+ * device current (cudaGetSymbolAddress) and caches it; make that first call
+ * before any stream capture on the device.
+ *
+ * Sharing: all calls on one device use the same array, which keeps whatever
+ * the previous call left; each call clears the parts that must start at zero.
+ * Calls whose kernels overlap on the GPU (e.g. on two unordered streams) race
+ * on the array and produce wrong gradients -- order them, e.g. on one stream.
+ */
+#define RFB_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+RFB_API int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* u,
+                                 const void* w, const void* o, const float* lse, const void* dout,
+                                 void* dq, void* dk, void* dv, void* du, void* dw, int B, int H,
+                                 int N, int d, int r, float scale, void* stream);
+
 /* Human-readable text for a status code (static storage). */
 RFB_API const char* rfb_strerror(int status);
 

@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     LIB_PATH,
     RFBAttention,
     attn_bwd,
+    attn_bwd_noalloc,
     attn_fwd,
     bwd_workspace_size,
     last_device_error,
@@ -20,5 +21,5 @@ from .binding import (  # noqa: F401
     strerror,
 )
 
-__all__ = ["attn_fwd", "attn_bwd", "bwd_workspace_size", "rfb_attention", "RFBAttention",
+__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "bwd_workspace_size", "rfb_attention", "RFBAttention",
            "last_device_error", "selftest_wait_timeout", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]

@@ -32,6 +32,7 @@ SIGNATURES = {
     "rfb_attn_fwd": (_i, [_vp] * 6 + [_fp] + [_i] * 5 + [_f, _vp]),
     "rfb_attn_bwd_workspace_size": (_sz, [_i] * 5),
     "rfb_attn_bwd": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
+    "rfb_attn_bwd_noalloc": (_i, [_vp] * 6 + [_fp] + [_vp] * 6 + [_i] * 5 + [_f, _vp]),
     "rfb_strerror": (ctypes.c_char_p, [_i]),
     "rfb_last_device_error": (_i, []),
     "rfb_last_cuda_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
@@ -170,6 +171,45 @@ def attn_bwd(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=None, grads=N
             _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, H, N, d, r, s,
             _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_bwd")
+    return dq, dk, dv, du, dw
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def attn_bwd_noalloc(q, k, v, u, w, o, lse, dout, scale=None, *, grads=None, stream=None):
+    """Backward through rfb_attn_bwd_noalloc: the library uses its own fixed
+    32 MiB device scratch instead of a caller workspace (for callers that may
+    not allocate device memory while they run).  Problems needing more scratch
+    than that raise; concurrent calls on one device must be ordered."""
+    B, H, N, d, r = _dims(q, u)
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_operand(name, t, (B, H, N, d), dev)
+    if r > 0:
+        _check_operand("u", u, (B, H, N, r), dev)
+        _check_operand("w", w, (B, H, N, r), dev)
+    else:
+        u = w = None
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    if grads is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        du = torch.empty_like(u) if r else None
+        dw = torch.empty_like(w) if r else None
+    else:
+        dq, dk, dv, du, dw = grads
+    with torch.cuda.device(dev):
+        rc = load_library().rfb_attn_bwd_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(du), _ptr(dw), B, H, N, d, r, s, _stream_ptr(stream, dev))
+    if rc == RFB_ERR_WORKSPACE:
+        raise RuntimeError(
+            f"rfb_attn_bwd_noalloc: this problem needs {bwd_workspace_size(B, H, N, d, r)} bytes "
+            f"of scratch, more than the library's fixed {NOALLOC_SCRATCH_BYTES} bytes")
+    _check(rc, "rfb_attn_bwd_noalloc")
     return dq, dk, dv, du, dw
 
 

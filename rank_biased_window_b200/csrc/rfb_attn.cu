@@ -38,6 +38,11 @@ __global__ void selftest_wait_kernel(int* err, uint64_t timeout_ns) {
   __syncthreads();
 }
 
+// Scratch of rfb_attn_bwd_noalloc: a fixed module array, so that entry point
+// needs no allocation.  In host code this name is only a stand-in; its device
+// address comes from cudaGetSymbolAddress (noalloc_scratch below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RFB_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
@@ -316,6 +321,26 @@ int grid_for(long long work, int per_block, int sms) {
   return g < 1 ? 1 : static_cast<int>(g);
 }
 
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device with that device current.  Returns RFB_OK or RFB_ERR_CUDA.
+int noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail(e, kSiteGetDevice);
+  if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e, kSiteGetDevice);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess)
+      return cuda_fail(e, kSiteSymbol);
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return RFB_OK;
+}
+
 }  // namespace
 }  // namespace rfb
 
@@ -436,6 +461,22 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
     bwd_post_kernel<<<grid_for(groups, 256, dev.sms), 256, 0, st>>>(a);
   }
   return launch_status();
+}
+
+int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* u,
+                         const void* w, const void* o, const float* lse, const void* dout,
+                         void* dq, void* dk, void* dv, void* du, void* dw, int B, int H, int N,
+                         int d, int r, float scale, void* stream) {
+  bool empty = false;
+  if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
+  if (empty) return RFB_OK;
+  if (ws_layout(B, H, N, d, r).total > RFB_NOALLOC_SCRATCH_BYTES) return RFB_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  // The backward's first kernel zeroes the accumulator and rewrites the row
+  // statistics, so what an earlier call left in the array does not matter.
+  return rfb_attn_bwd(q, k, v, u, w, o, lse, dout, dq, dk, dv, du, dw, scratch,
+                      RFB_NOALLOC_SCRATCH_BYTES, B, H, N, d, r, scale, stream);
 }
 
 const char* rfb_strerror(int status) {
