@@ -54,7 +54,7 @@ extern "C" {
 
 typedef enum {
   RFB_OK = 0,
-  RFB_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, non-finite scale */
+  RFB_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, scale not finite and > 0 */
   RFB_ERR_UNSUPPORTED = 2,    /* d or r outside the supported set, sizes beyond int32 */
   RFB_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
   RFB_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
@@ -69,7 +69,8 @@ typedef enum {
  *   o       : [B, H, N, d] bf16 output.
  *   lse     : [B, H, N] fp32 output (natural-log log-sum-exp of each score row,
  *             consumed by rfb_attn_bwd).
- *   scale   : s, any finite value (usually 1/sqrt(d)).
+ *   scale   : s, finite and > 0 (usually 1/sqrt(d)); anything else is
+ *             RFB_ERR_INVALID_ARG.
  */
 RFB_API int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, const void* w,
                  void* o, float* lse, int B, int H, int N, int d, int r, float scale,

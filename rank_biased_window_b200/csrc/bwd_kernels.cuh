@@ -15,11 +15,13 @@
 //              LSE_i log2(e), and zeroes the fp32 dQ|dU accumulator.
 //   bwd_main : one CTA per (head, 128-key tile); K, W, V stay in shared memory,
 //              dV, dK, dW accumulate in TMEM across all 128-query tiles.  Per
-//              query tile: S^T and dP^T by tcgen05 into TMEM, P^T and dS^T
-//              formed by the compute warps into swizzled shared memory, then
-//              dV, dK, dW (+=) and the partial dQ|dU tile (into the S^T
-//              columns), which the compute warps add into the fp32
-//              accumulator with vector reductions.
+//              query tile: S^T and dP^T by tcgen05 into TMEM; two compute
+//              warpgroups (64 query columns each) form P^T and dS^T into
+//              swizzled shared memory; then dV, dK, dW (+=) and the partial
+//              dQ|dU tile into TMEM columns of its own (when they fit), which
+//              the compute warps stage in 128-byte-swizzled shared memory and
+//              add into the fp32 accumulator with TMA bulk tensor reductions,
+//              while the next tile's S^T / dP^T MMAs run.
 //   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]).
 #pragma once
 #include "fwd_kernels.cuh"
@@ -148,28 +150,37 @@ struct BwdCfg {
   static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UB, S_DV = S_L2 + 512;
   static constexpr int STAGE = 2 * QB + UB + 1024;
   static constexpr int PB = kTile * kTile * 2;
-  static constexpr int NS_FIT = (222 * 1024 - KVB - 2 * PB) / STAGE;
+  static constexpr int STG = kTile * 32 * 4;  // one 128 x 32 fp32 staging chunk per warpgroup
+  static constexpr int NS_FIT = (226 * 1024 - KVB - 2 * PB - 2 * STG) / STAGE;
   static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
   static constexpr int OFF_STAGE = KVB;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_DS = OFF_P + PB;
-  static constexpr int OFF_BAR = OFF_DS + PB;
-  // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain
-  static constexpr int NBAR = 2 * NS + 6;
+  static constexpr int OFF_STG = OFF_DS + PB;
+  static constexpr int OFF_BAR = OFF_STG + 2 * STG;
+  // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain wg_sync[2]
+  static constexpr int NBAR = 2 * NS + 8;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  // TMEM columns
+  // dQ | dU chunks of 32 columns
+  static constexpr int NCH = (D + RP + 31) / 32;
+  // TMEM columns.  dQ | dU get their own columns when they fit, so the next
+  // query tile's S^T / dP^T MMAs need not wait for the dQ reduction.
   static constexpr int T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D, T_DW = 256 + 2 * D;
-  static_assert(NS >= 2, "not enough shared memory for two query stages");
+  static constexpr bool SEP_DQ = (256 + 2 * D + RP + NCH * 32) <= 512;
+  static constexpr int T_DQ = SEP_DQ ? 256 + 2 * D + RP : 0;
+  static_assert(NS >= 1, "shared memory budget");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
-  static_assert(T_DW + RP <= 512 && D + RP <= 128, "TMEM budget");
+  static_assert(T_DW + RP <= 512 && NCH * 32 <= 128, "TMEM budget");
 };
 
+constexpr int kBwdThreads = 320;  // warps 0-7 compute (two warpgroups), 8 TMA, 9 MMA
+
 template <int D, int RP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
                     const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mDO,
-                    const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap mAcc, const BwdArgs args) {
   using C = BwdCfg<D, RP>;
   constexpr int NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -184,6 +195,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t dq_full = bar0 + 8u * (3 + 2 * NS);
   const uint32_t dq_free = bar0 + 8u * (4 + 2 * NS);
   const uint32_t drain_bar = bar0 + 8u * (5 + 2 * NS);
+  // Per-warpgroup barriers (128 arrivals) guarding the dQ staging buffers.
+  auto wg_bar = [&](int w) { return bar0 + 8u * (6 + 2 * NS + w); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -202,23 +215,26 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(q_empty(s), 1);
     }
     mbar_init(sdp_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(dq_free, 256);
     mbar_init(drain_bar, 1);
+    mbar_init(wg_bar(0), 128);
+    mbar_init(wg_bar(1), 128);
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch(&mQ);
     tma_prefetch(&mK);
     tma_prefetch(&mV);
     tma_prefetch(&mDO);
+    tma_prefetch(&mAcc);
     if constexpr (RP > 0) {
       tma_prefetch(&mU);
       tma_prefetch(&mW);
     }
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -228,7 +244,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_expect_tx(kv_full, C::KVB);
@@ -253,23 +269,22 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = (i > NS ? i - NS : 0); j < i; ++j)
         wait_drain(q_full(j % NS), (j / NS) & 1, args.timeout_ns);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ----------------------------------------------------------- MMA issue
     constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-    bool ok = wait_warp(kv_full, 0, g, 32);
-    for (int i = 0; ok && i < nq; ++i) {
+    // S^T / s = K Q^T + W U'^T and dP^T = V dO^T for query tile i.
+    auto issue_sdp = [&](int i) -> bool {
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-      if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) break;
+      if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) return false;
       if constexpr (RP > 0) {
         scale_tile_bf16(st + C::S_U, C::UB, args.inv_scale);
         fence_async_smem();
       }
       __syncwarp();
-      if (i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) break;
+      if (!C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
       tc_fence_after();
       if (lane == 0) {
-        // S^T / s = K Q^T + W U'^T ;  dP^T = V dO^T
         issue_scores<D, RP>(tmem + C::T_S, sb + C::OFF_K, st + C::S_Q, sb + C::OFF_W, st + C::S_U);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -278,19 +293,33 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit(sdp_full);
       }
       __syncwarp();
+      return true;
+    };
+    bool ok = wait_warp(kv_full, 0, g, 32);
+    if (ok && nq > 0) ok = issue_sdp(0);
+    for (int i = 0; ok && i < nq; ++i) {
+      const int s = i % NS;
+      const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(ds_full, i & 1, g, 35)) break;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t pb = sb + C::OFF_P, dsb = sb + C::OFF_DS;
-        issue_k128<D>(tmem + C::T_DV, pb, st + C::S_DO, i > 0);   // dV += P^T dO
-        issue_k128<D>(tmem + C::T_DK, dsb, st + C::S_Q, i > 0);   // dK += dS^T Q
+        issue_k128<D>(tmem + C::T_DV, pb, st + C::S_DO, i > 0);  // dV += P^T dO
+        issue_k128<D>(tmem + C::T_DK, dsb, st + C::S_Q, i > 0);  // dK += dS^T Q
         if constexpr (RP > 0) issue_k128<RP>(tmem + C::T_DW, dsb, st + C::S_U, i > 0);  // dW += dS^T U'
-        issue_k128_at<D>(tmem + C::T_S, dsb, sb + C::OFF_K);       // dQ = dS K
-        if constexpr (RP > 0) issue_k128_at<RP>(tmem + C::T_S + D, dsb, sb + C::OFF_W);  // dU = dS W
+      }
+      __syncwarp();
+      if (C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 36)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t dsb = sb + C::OFF_DS;
+        issue_k128_at<D>(tmem + C::T_DQ, dsb, sb + C::OFF_K);  // dQ = dS K
+        if constexpr (RP > 0) issue_k128_at<RP>(tmem + C::T_DQ + D, dsb, sb + C::OFF_W);  // dU = dS W
         umma_commit(dq_full);
         umma_commit(q_empty(s));
       }
       __syncwarp();
+      if (i + 1 < nq && !issue_sdp(i + 1)) break;
     }
     if (lane == 0) {
       umma_commit(drain_bar);
@@ -298,34 +327,50 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------ compute warps
-    const int row = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------- compute warps (two warpgroups)
+    const int wg = warp >> 2;                  // 0: queries 0-63, 1: queries 64-127
+    const int row = threadIdx.x & 127;         // TMEM lane == key row (S^T) == query row (dQ)
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const bool key_ok = (k0 + row) < N;
     const float sl2 = args.scale_log2;
-    const int DA = D + args.r;
+    const bool leader = (threadIdx.x & 127) == 0;  // issues this warpgroup's reductions
+    const uint32_t stg = sb + C::OFF_STG + wg * C::STG;
+    uint32_t wg_phase = 0;
+    // Bounded barrier over this warpgroup's 128 threads.
+    auto wg_sync = [&]() -> bool {
+      mbar_arrive(wg_bar(wg));
+      const bool r = wait_warp(wg_bar(wg), wg_phase & 1u, g, 40);
+      ++wg_phase;
+      return r;
+    };
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-      if (!wait_warp(q_full(s), (i / NS) & 1, g, 36)) { ok = false; break; }
-      if (!wait_warp(sdp_full, i & 1, g, 37)) { ok = false; break; }
+      if (!wait_warp(q_full(s), (i / NS) & 1, g, 37)) { ok = false; break; }
+      if (!wait_warp(sdp_full, i & 1, g, 38)) { ok = false; break; }
       tc_fence_after();
-      const float* l2 = reinterpret_cast<const float*>(smem + C::OFF_STAGE + s * C::STAGE + C::S_L2);
-      const float* dvv = reinterpret_cast<const float*>(smem + C::OFF_STAGE + s * C::STAGE + C::S_DV);
       const int qvalid = N - i * kTile;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = wg * 64; c < wg * 64 + 64; c += 32) {
         uint32_t x[32], y[32];
         tmem_ld32(tmem + lane_base + C::T_S + c, x);
         tmem_ld32(tmem + lane_base + C::T_DP + c, y);
         float p[32], ds[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = c + e;
-          const bool valid = key_ok && (q < qvalid);
-          p[e] = valid ? fast_exp2(fmaf(__uint_as_float(x[e]), sl2, -l2[q])) : 0.f;
-          ds[e] = p[e] * (__uint_as_float(y[e]) - dvv[q]);
+        for (int e = 0; e < 32; e += 4) {
+          const uint4 lv = ld_shared_v4(st + C::S_L2 + (c + e) * 4);
+          const uint4 dv = ld_shared_v4(st + C::S_DV + (c + e) * 4);
+          const float l4[4] = {__uint_as_float(lv.x), __uint_as_float(lv.y), __uint_as_float(lv.z),
+                               __uint_as_float(lv.w)};
+          const float d4[4] = {__uint_as_float(dv.x), __uint_as_float(dv.y), __uint_as_float(dv.z),
+                               __uint_as_float(dv.w)};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const bool valid = key_ok && (c + e + t < qvalid);
+            p[e + t] = valid ? fast_exp2(fmaf(__uint_as_float(x[e + t]), sl2, -l4[t])) : 0.f;
+            ds[e + t] = p[e + t] * (__uint_as_float(y[e + t]) - d4[t]);
+          }
         }
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
@@ -340,102 +385,84 @@ __global__ void __launch_bounds__(192, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
-      // Partial dQ | dU of this query tile (TMEM lane = query row).
-      if (!wait_warp(dq_full, i & 1, g, 38)) { ok = false; break; }
+      // Partial dQ | dU of this query tile (TMEM lane = query row): this
+      // warpgroup takes chunks wg, wg + 2, ... of 32 columns, reads them all,
+      // frees the TMEM columns, then reduces each through its staging buffer.
+      if (!wait_warp(dq_full, i & 1, g, 39)) { ok = false; break; }
       tc_fence_after();
-      const int q = i * kTile + row;
-      float* accrow = args.acc + (static_cast<size_t>(bh) * N + q) * DA;
-      if constexpr (D == 32) {
-        uint32_t z[32];
-        tmem_ld32(tmem + lane_base + C::T_S, z);
-        if constexpr (RP > 0) {
-          uint32_t zu[RP];
-          tmem_ld_cols<RP>(tmem + lane_base + C::T_S + D, zu);
-          tc_fence_before();
-          mbar_arrive(dq_free);
-          if (q < N) {
+      constexpr int MY_MAX = (C::NCH + 1) / 2;
+      uint32_t z[MY_MAX][32];
 #pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              red_add_v4(accrow + c, __uint_as_float(z[c]) * args.scale,
-                         __uint_as_float(z[c + 1]) * args.scale, __uint_as_float(z[c + 2]) * args.scale,
-                         __uint_as_float(z[c + 3]) * args.scale);
+      for (int m = 0; m < MY_MAX; ++m) {
+        const int ch = wg + 2 * m;
+        if (ch < C::NCH) tmem_ld32(tmem + lane_base + C::T_DQ + ch * 32, z[m]);
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
 #pragma unroll
-            for (int c = 0; c < RP; c += 4)
-              if (c < args.r)
-                red_add_v4(accrow + D + c, __uint_as_float(zu[c]), __uint_as_float(zu[c + 1]),
-                           __uint_as_float(zu[c + 2]), __uint_as_float(zu[c + 3]));
+      for (int m = 0; m < MY_MAX; ++m) {
+        const int ch = wg + 2 * m;
+        if (ch >= C::NCH) break;
+        if (leader) bulk_wait_read_all();  // previous reduction from this buffer has read it
+        if (!wg_sync()) { ok = false; break; }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v4[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int col = ch * 32 + j * 4 + t;
+            v4[t] = __uint_as_float(z[m][j * 4 + t]) * (col < D ? args.scale : 1.0f);
           }
-        } else {
-          tc_fence_before();
-          mbar_arrive(dq_free);
-          if (q < N) {
-#pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              red_add_v4(accrow + c, __uint_as_float(z[c]) * args.scale,
-                         __uint_as_float(z[c + 1]) * args.scale, __uint_as_float(z[c + 2]) * args.scale,
-                         __uint_as_float(z[c + 3]) * args.scale);
-          }
+          st_shared_v4(stg + row * 128 + ((j ^ (row & 7)) << 4), __float_as_uint(v4[0]),
+                       __float_as_uint(v4[1]), __float_as_uint(v4[2]), __float_as_uint(v4[3]));
         }
-      } else {
-        // D == 64: two 32-column halves of dQ, then dU.
-        uint32_t z[64];
-        tmem_ld64(tmem + lane_base + C::T_S, z);
-        uint32_t zu[RP > 0 ? RP : 1];
-        if constexpr (RP > 0) tmem_ld_cols<RP>(tmem + lane_base + C::T_S + D, zu);
-        tc_fence_before();
-        mbar_arrive(dq_free);
-        if (q < N) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 4)
-            red_add_v4(accrow + c, __uint_as_float(z[c]) * args.scale,
-                       __uint_as_float(z[c + 1]) * args.scale, __uint_as_float(z[c + 2]) * args.scale,
-                       __uint_as_float(z[c + 3]) * args.scale);
-          if constexpr (RP > 0) {
-#pragma unroll
-            for (int c = 0; c < RP; c += 4)
-              if (c < args.r)
-                red_add_v4(accrow + D + c, __uint_as_float(zu[c]), __uint_as_float(zu[c + 1]),
-                           __uint_as_float(zu[c + 2]), __uint_as_float(zu[c + 3]));
-          }
+        fence_async_smem();
+        if (!wg_sync()) { ok = false; break; }
+        if (leader) {
+          tma_reduce_add_3d(&mAcc, stg, ch * 32, i * kTile, bh);
+          bulk_commit();
         }
       }
+      if (!ok) break;
     }
     if (ok && nq > 0) {
       // dq_full of the last tile implies all dV, dK, dW MMAs have completed.
-      uint32_t gv[D], gk[D];
-      tmem_ld_cols<D>(tmem + lane_base + C::T_DV, gv);
-      tmem_ld_cols<D>(tmem + lane_base + C::T_DK, gk);
-      if (key_ok) {
-        const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
-        store_o_row<D>(args.dv + r0 * D, gv, 1.0f);
-        store_o_row<D>(args.dk + r0 * D, gk, args.scale);
-      }
-      if constexpr (RP > 0) {
-        uint32_t gw[RP];
-        tmem_ld_cols<RP>(tmem + lane_base + C::T_DW, gw);
-        if (key_ok) {
-          const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
-          uint4* dst = reinterpret_cast<uint4*>(args.dw + r0 * args.r);
+      const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
+      if (wg == 0) {
+        uint32_t gv[D];
+        tmem_ld_cols<D>(tmem + lane_base + C::T_DV, gv);
+        if (key_ok) store_o_row<D>(args.dv + r0 * D, gv, 1.0f);
+        if constexpr (RP > 0) {
+          uint32_t gw[RP];
+          tmem_ld_cols<RP>(tmem + lane_base + C::T_DW, gw);
+          if (key_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(args.dw + r0 * args.r);
+            const float f = args.scale;
 #pragma unroll
-          for (int c = 0; c < RP; c += 8) {
-            if (c < args.r) {
-              const float f = args.scale;
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(gw[c]) * f, __uint_as_float(gw[c + 1]) * f);
-              v.y = pack_bf16x2(__uint_as_float(gw[c + 2]) * f, __uint_as_float(gw[c + 3]) * f);
-              v.z = pack_bf16x2(__uint_as_float(gw[c + 4]) * f, __uint_as_float(gw[c + 5]) * f);
-              v.w = pack_bf16x2(__uint_as_float(gw[c + 6]) * f, __uint_as_float(gw[c + 7]) * f);
-              dst[c >> 3] = v;
+            for (int c = 0; c < RP; c += 8) {
+              if (c < args.r) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(gw[c]) * f, __uint_as_float(gw[c + 1]) * f);
+                v.y = pack_bf16x2(__uint_as_float(gw[c + 2]) * f, __uint_as_float(gw[c + 3]) * f);
+                v.z = pack_bf16x2(__uint_as_float(gw[c + 4]) * f, __uint_as_float(gw[c + 5]) * f);
+                v.w = pack_bf16x2(__uint_as_float(gw[c + 6]) * f, __uint_as_float(gw[c + 7]) * f);
+                dst[c >> 3] = v;
+              }
             }
           }
         }
+      } else {
+        uint32_t gk[D];
+        tmem_ld_cols<D>(tmem + lane_base + C::T_DK, gk);
+        if (key_ok) store_o_row<D>(args.dk + r0 * D, gk, args.scale);
       }
     }
+    if (leader) bulk_wait_all();  // reductions complete before the CTA exits
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

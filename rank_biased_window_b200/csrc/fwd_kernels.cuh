@@ -84,6 +84,51 @@ __device__ __forceinline__ void store_o_row(__nv_bfloat16* dst, const uint32_t (
   }
 }
 
+// Sets raw scores at positions >= valid to -inf (only the last key tile of a
+// row is ragged, so this runs at most once per row).
+template <int NC>
+__device__ __forceinline__ void mask_tail(uint32_t (&sv)[NC], int valid) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (c >= valid) sv[c] = 0xFF800000u;
+}
+
+// Row maximum with 8 independent partial maxima (short dependency chains).
+template <int NC>
+__device__ __forceinline__ float row_max(const uint32_t (&sv)[NC]) {
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = __uint_as_float(sv[e]);
+#pragma unroll
+  for (int c = 8; c < NC; c += 8)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], __uint_as_float(sv[c + e]));
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// p_j = 2^(s_j * sl2 - m) written as bf16 into the 128-byte-swizzled K-major P
+// tile (row `row`, columns col0..col0+NC); returns sum_j p_j (fp32, 8 partial
+// sums).  Masked scores are -inf and give p = 0.
+template <int NC>
+__device__ __forceinline__ float exp_row_to_smem(const uint32_t (&sv)[NC], float sl2, float m,
+                                                 uint32_t pbuf, int row, int col0) {
+  float l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) l[e] = 0.f;
+#pragma unroll
+  for (int c = 0; c < NC; c += 8) {
+    float p[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      p[e] = fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
+      l[e] += p[e];
+    }
+    st_shared_v4(pbuf + sw128_offset(row, col0 + c, 128), pack_bf16x2(p[0], p[1]),
+                 pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+  }
+  return ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
+}
+
 // Issue the score MMAs  S(tmem) = Q.K^T + U'.W^T  for one 128x128 tile.
 template <int D, int RP>
 __device__ __forceinline__ void issue_scores(uint32_t s_tmem, uint32_t q, uint32_t k, uint32_t u,
@@ -295,25 +340,9 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       uint32_t sv[NP];
       tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < N) mx = fmaxf(mx, __uint_as_float(sv[j]));
-      const float m = mx * sl2;
-      float l = 0.f;
-      const uint32_t pbuf = sb + C::OFF_P + a * C::PB;
-#pragma unroll
-      for (int c = 0; c < NP; c += 8) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = c + e;
-          p[e] = (j < N) ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -m)) : 0.f;
-          l += p[e];
-        }
-        st_shared_v4(pbuf + sw128_offset(row, wl * NP + c, 128), pack_bf16x2(p[0], p[1]),
-                     pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-      }
+      if (N < NP) mask_tail<NP>(sv, N);
+      const float m = row_max<NP>(sv) * sl2;
+      const float l = exp_row_to_smem<NP>(sv, sl2, m, sb + C::OFF_P + a * C::PB, row, wl * NP);
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(p_full(a));
@@ -497,11 +526,8 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(s_empty(b));
       const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c < kvalid) mx = fmaxf(mx, __uint_as_float(sv[c]));
-      const float m_new = fmaxf(m_run, mx * sl2);
+      if (kvalid < kTile) mask_tail<128>(sv, kvalid);
+      const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);
       // Lazy rescale: keep the running max unless it grew by more than 2^8.
       const bool need = m_new > m_run + 8.0f;
       float alpha = 1.f;
@@ -512,18 +538,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
       if (j >= 2 && !wait_warp(pv_done(b), ((j >> 1) + 1) & 1, g, 17)) { ok = false; break; }
-      const uint32_t pbuf = sb + C::OFF_P + b * C::PB;
-#pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = (c + e < kvalid) ? fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m_run)) : 0.f;
-          l += p[e];
-        }
-        st_shared_v4(pbuf + sw128_offset(row, c, 128), pack_bf16x2(p[0], p[1]),
-                     pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-      }
+      l += exp_row_to_smem<128>(sv, sl2, m_run, sb + C::OFF_P + b * C::PB, row, 0);
       if (fix_o) {
         // O holds the sum through tile j-1 at the old running max: wait for that
         // PV to land, then rescale this thread's row in place.

@@ -154,6 +154,23 @@ int encode_3d(CUtensorMap* m, const void* ptr, int cols, int N, int BH, int box_
   return rc == CUDA_SUCCESS ? RFB_OK : cuda_fail(static_cast<int>(rc), kSiteEncode);
 }
 
+// 3-D fp32 map over the [BH, N, cols] dQ|dU accumulator, box (32, 128, 1),
+// 128-byte swizzle (32 fp32 per row); used for bulk reductions.
+int encode_acc_3d(CUtensorMap* m, void* ptr, int cols, int N, int BH) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return cuda_fail(0, kSiteEncoder);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4,
+                                 static_cast<cuuint64_t>(cols) * 4 * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult rc = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? RFB_OK : cuda_fail(static_cast<int>(rc), kSiteEncode);
+}
+
 int pad_rank(int r) { return r == 0 ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -163,7 +180,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int check_shape(int B, int H, int N, int d, int r, float scale, bool* empty) {
   *empty = false;
   if (B < 0 || H < 0 || N < 0 || d < 0 || r < 0) return RFB_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return RFB_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return RFB_ERR_INVALID_ARG;
   if (d != 32 && d != 64) return RFB_ERR_UNSUPPORTED;
   if (r > 64 || (r % 8) != 0) return RFB_ERR_UNSUPPORTED;
   if (B == 0 || H == 0 || N == 0) {
@@ -231,7 +248,7 @@ struct LaunchTimer {
 };
 
 struct Maps {
-  CUtensorMap q, k, v, u, w, g;
+  CUtensorMap q, k, v, u, w, g, acc;
 };
 
 // ---------------------------------------------------------------- forward
@@ -301,7 +318,8 @@ int launch_bwd_main(const Maps& m, const BwdArgs& a, cudaStream_t st) {
   if (int rc = ensure_smem(bwd_main_kernel<D, RP>, C::SMEM, done)) return rc;
   const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
   LaunchTimer timer(kIdBwdMain, st);
-  bwd_main_kernel<D, RP><<<grid, 192, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, m.g, a);
+  bwd_main_kernel<D, RP><<<grid, kBwdThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, m.g, m.acc,
+                                                              a);
   return launch_status();
 }
 
@@ -423,8 +441,9 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   if (!rc) rc = encode_3d(&m.g, dout, d, N, BH, d, kTile, 1);
   if (!rc && r > 0) rc = encode_3d(&m.u, u, r, N, BH, rp, kTile, 1);
   if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, kTile, 1);
-  if (rc) return rc;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (!rc) rc = encode_acc_3d(&m.acc, ws + L.acc, d + r, N, BH);
+  if (rc) return rc;
   BwdArgs a;
   a.o = static_cast<const __nv_bfloat16*>(o);
   a.lse = lse;
@@ -482,7 +501,8 @@ int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
 const char* rfb_strerror(int status) {
   switch (status) {
     case RFB_OK: return "success";
-    case RFB_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or non-finite scale)";
+    case RFB_ERR_INVALID_ARG:
+      return "invalid argument (null pointer, negative size, or scale not finite and > 0)";
     case RFB_ERR_UNSUPPORTED: return "unsupported shape (d must be 32 or 64; r a multiple of 8 in [0, 64])";
     case RFB_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case RFB_ERR_WORKSPACE: return "workspace missing or too small";

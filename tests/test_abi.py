@@ -57,6 +57,8 @@ def test_host_side_argument_checks(rfb_lib):
     assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, 0.1, n) == 1
     assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, -1, 1, 64, 32, 8, 0.1, n) == 1
     assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, float("inf"), n) == 1
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, 0.0, n) == 1
+    assert lib.rfb_attn_fwd(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, -0.125, n) == 1
     assert lib.rfb_attn_bwd(*([n] * 14), 0, 1, 1, 64, 32, 8, 0.1, n) == 1
 
 

@@ -33,6 +33,9 @@ CASES = [
     (1, 1, 256, 64, 0),
     (1, 1, 384, 32, 64),
     (1, 1, 200, 64, 24),
+    (1, 1, 200, 64, 64),   # dQ|dU share the S^T columns (no room for their own)
+    (1, 2, 130, 64, 16),
+    (3, 1, 64, 32, 0),
 ]
 
 
