@@ -12,13 +12,16 @@
 //
 // Three kernels:
 //   bwd_pre  : D_i = rowsum(dO o O) (equal to sum_j P_ij dP_ij because O = P V),
-//              LSE_i log2(e), and zeroes the fp32 dQ|dU accumulator.
+//              LSE_i log2(e), U' = bf16(U / s), and zeroes the fp32 dQ|dU
+//              accumulator.
 //   bwd_main : one CTA per (head, 128-key tile); K, W, V stay in shared memory,
 //              dV, dK, dW accumulate in TMEM across all 128-query tiles.  Per
 //              query tile: S^T and dP^T by tcgen05 into TMEM; two compute
-//              warpgroups (64 query columns each) form P^T and dS^T into
-//              swizzled shared memory; then dV, dK, dW (+=) and the partial
-//              dQ|dU tile into TMEM columns of its own (when they fit), which
+//              warpgroups (64 query columns each) form P^T and dS^T and write
+//              them back into TMEM in place (bf16), dS^T also into swizzled
+//              shared memory; dV, dK, dW (+=) read their A operand from TMEM;
+//              the partial dQ|dU tile goes to TMEM columns of its own (when
+//              they fit), which
 //              the compute warps stage in 128-byte-swizzled shared memory and
 //              add into the fp32 accumulator with TMA bulk tensor reductions,
 //              while the next tile's S^T / dP^T MMAs run.
@@ -34,6 +37,8 @@ struct BwdArgs {
   const __nv_bfloat16* o;     // [BH, N, D]
   const float* lse;           // [BH, N]
   const __nv_bfloat16* dout;  // [BH, N, D]
+  const __nv_bfloat16* u;     // [BH, N, r]   bias factor U
+  __nv_bfloat16* uprime;      // [BH, N, r]   U' = bf16(U / s), written by bwd_pre
   float* dvec;                // [BH, Npad]   D_i
   float* lse2;                // [BH, Npad]   LSE_i * log2(e)
   float* acc;                 // [BH, N, D + r] fp32 dQ | dU accumulator
@@ -87,6 +92,19 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
   for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n4;
        t += static_cast<size_t>(gridDim.x) * blockDim.x)
     acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // U' = bf16(U / s), staged once here instead of once per (key tile, query tile).
+  const size_t n8 = static_cast<size_t>(a.BH) * a.N * a.r / 8;
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n8;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(a.u)[t];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      o[e] = pack_bf16x2(__uint_as_float(w[e] << 16) * a.inv_scale,
+                         __uint_as_float(w[e] & 0xFFFF0000u) * a.inv_scale);
+    reinterpret_cast<uint4*>(a.uprime)[t] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
 }
 
 // ----------------------------------------------------------------- bwd_post
@@ -125,6 +143,21 @@ __device__ __forceinline__ void issue_k128(uint32_t d_tmem, uint32_t a, uint32_t
     umma_bf16(d_tmem, ad, bd, id, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
+// Same contraction with A = a 128 x 128 bf16 tile held in TMEM (lane = row,
+// two elements per column), laid out as two 64-column halves of 32 columns
+// each at a_tmem and a_tmem + 64 (the in-place layout the compute warpgroups
+// write): K-step kk reads columns (kk / 4) * 64 + (kk % 4) * 8.
+template <int NN>
+__device__ __forceinline__ void issue_k128_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
+                                              bool accumulate) {
+  constexpr uint32_t id = idesc_bf16_f32(128, NN, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t bd = desc_mnmajor(b + kk * 16 * (NN * 2), NN * 2, 128 * NN * 2);
+    umma_bf16_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, bd, id,
+                 (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
 // Same contraction with A read transposed: the tile stored for dS^T (rows =
 // keys, queries contiguous) is used as MN-major A = dS (rows = queries).
 template <int NN>
@@ -149,20 +182,19 @@ struct BwdCfg {
   // stage: Q, dO, U, lse2[128], dvec[128]
   static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UB, S_DV = S_L2 + 512;
   static constexpr int STAGE = 2 * QB + UB + 1024;
-  static constexpr int PB = kTile * kTile * 2;
-  static constexpr int STG = kTile * 32 * 4;  // one 128 x 32 fp32 staging chunk per warpgroup
-  static constexpr int NS_FIT = (226 * 1024 - KVB - 2 * PB - 2 * STG) / STAGE;
+  static constexpr int PB = kTile * kTile * 2;  // dS tile (bf16)
+  static constexpr int STG = kTile * 32 * 4;    // one 128 x 32 fp32 staging buffer
+  // dQ | dU chunks of 32 columns, one staging buffer each
+  static constexpr int NCH = (D + RP + 31) / 32;
+  static constexpr int NS_FIT = (226 * 1024 - KVB - PB - NCH * STG) / STAGE;
   static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
   static constexpr int OFF_STAGE = KVB;
-  static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_DS = OFF_P + PB;
+  static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_STG = OFF_DS + PB;
-  static constexpr int OFF_BAR = OFF_STG + 2 * STG;
-  // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain wg_sync[2]
-  static constexpr int NBAR = 2 * NS + 8;
+  static constexpr int OFF_BAR = OFF_STG + NCH * STG;
+  // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain wg_sync[2] a_done
+  static constexpr int NBAR = 2 * NS + 9;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  // dQ | dU chunks of 32 columns
-  static constexpr int NCH = (D + RP + 31) / 32;
   // TMEM columns.  dQ | dU get their own columns when they fit, so the next
   // query tile's S^T / dP^T MMAs need not wait for the dQ reduction.
   static constexpr int T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D, T_DW = 256 + 2 * D;
@@ -197,6 +229,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (5 + 2 * NS);
   // Per-warpgroup barriers (128 arrivals) guarding the dQ staging buffers.
   auto wg_bar = [&](int w) { return bar0 + 8u * (6 + 2 * NS + w); };
+  // Completes when the MMAs reading P^T / dS^T from TMEM (dV, dK, dW) are done.
+  const uint32_t a_done = bar0 + 8u * (8 + 2 * NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -221,6 +255,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(drain_bar, 1);
     mbar_init(wg_bar(0), 128);
     mbar_init(wg_bar(1), 128);
+    mbar_init(a_done, 1);
     fence_mbar_init();
   }
   if (warp == 8 && lane == 0) {
@@ -277,12 +312,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) return false;
-      if constexpr (RP > 0) {
-        scale_tile_bf16(st + C::S_U, C::UB, args.inv_scale);
-        fence_async_smem();
-      }
-      __syncwarp();
       if (!C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
+      // P^T / dS^T of the previous tile live in the S^T / dP^T columns: the MMAs
+      // reading them must be done before this tile's S^T / dP^T overwrite them.
+      if (i > 0 && !wait_warp(a_done, (i - 1) & 1, g, 41)) return false;
       tc_fence_after();
       if (lane == 0) {
         issue_scores<D, RP>(tmem + C::T_S, sb + C::OFF_K, st + C::S_Q, sb + C::OFF_W, st + C::S_U);
@@ -303,10 +336,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!wait_warp(ds_full, i & 1, g, 35)) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t pb = sb + C::OFF_P, dsb = sb + C::OFF_DS;
-        issue_k128<D>(tmem + C::T_DV, pb, st + C::S_DO, i > 0);  // dV += P^T dO
-        issue_k128<D>(tmem + C::T_DK, dsb, st + C::S_Q, i > 0);  // dK += dS^T Q
-        if constexpr (RP > 0) issue_k128<RP>(tmem + C::T_DW, dsb, st + C::S_U, i > 0);  // dW += dS^T U'
+        // A operands from TMEM: P^T over the S^T columns, dS^T over the dP^T columns.
+        issue_k128_ts<D>(tmem + C::T_DV, tmem + C::T_S, st + C::S_DO, i > 0);   // dV += P^T dO
+        issue_k128_ts<D>(tmem + C::T_DK, tmem + C::T_DP, st + C::S_Q, i > 0);   // dK += dS^T Q
+        if constexpr (RP > 0)
+          issue_k128_ts<RP>(tmem + C::T_DW, tmem + C::T_DP, st + C::S_U, i > 0);  // dW += dS^T U'
+        umma_commit(a_done);
       }
       __syncwarp();
       if (C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 36)) break;
@@ -334,7 +369,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool key_ok = (k0 + row) < N;
     const float sl2 = args.scale_log2;
     const bool leader = (threadIdx.x & 127) == 0;  // issues this warpgroup's reductions
-    const uint32_t stg = sb + C::OFF_STG + wg * C::STG;
+    constexpr int MY_MAX = (C::NCH + 1) / 2;
+    const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
     uint32_t wg_phase = 0;
     // Bounded barrier over this warpgroup's 128 threads.
     auto wg_sync = [&]() -> bool {
@@ -353,9 +389,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int qvalid = N - i * kTile;
 #pragma unroll 1
       for (int c = wg * 64; c < wg * 64 + 64; c += 32) {
-        uint32_t x[32], y[32];
-        tmem_ld32(tmem + lane_base + C::T_S + c, x);
-        tmem_ld32(tmem + lane_base + C::T_DP + c, y);
+        uint32_t xy[64];
+        tmem_ld32x2(tmem + lane_base + C::T_S + c, tmem + lane_base + C::T_DP + c, xy);
+        const uint32_t* x = xy;
+        const uint32_t* y = xy + 32;
         float p[32], ds[32];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -372,15 +409,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ds[e + t] = p[e + t] * (__uint_as_float(y[e + t]) - d4[t]);
           }
         }
+        // P^T and dS^T as packed bf16 into TMEM, in place over the columns this
+        // warpgroup has already read (columns wg*64 + [0, 32)); dS^T also into
+        // shared memory, where the dQ MMA reads it transposed.
+        uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          const uint32_t off = sw128_offset(row, c + e, 128);
-          st_shared_v4(sb + C::OFF_P + off, pack_bf16x2(p[e], p[e + 1]), pack_bf16x2(p[e + 2], p[e + 3]),
-                       pack_bf16x2(p[e + 4], p[e + 5]), pack_bf16x2(p[e + 6], p[e + 7]));
-          st_shared_v4(sb + C::OFF_DS + off, pack_bf16x2(ds[e], ds[e + 1]),
-                       pack_bf16x2(ds[e + 2], ds[e + 3]), pack_bf16x2(ds[e + 4], ds[e + 5]),
-                       pack_bf16x2(ds[e + 6], ds[e + 7]));
+        for (int e = 0; e < 16; ++e) {
+          pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+          dk[e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
         }
+        const int pcol = wg * 64 + (c - wg * 64) / 2;
+        tmem_st16(tmem + lane_base + C::T_S + pcol, pk);
+        tmem_st16(tmem + lane_base + C::T_DP + pcol, dk);
+#pragma unroll
+        for (int e = 0; e < 32; e += 8)
+          st_shared_v4(sb + C::OFF_DS + sw128_offset(row, c + e, 128), dk[e / 2], dk[e / 2 + 1],
+                       dk[e / 2 + 2], dk[e / 2 + 3]);
       }
       fence_async_smem();
       tc_fence_before();
@@ -390,7 +434,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // frees the TMEM columns, then reduces each through its staging buffer.
       if (!wait_warp(dq_full, i & 1, g, 39)) { ok = false; break; }
       tc_fence_after();
-      constexpr int MY_MAX = (C::NCH + 1) / 2;
       uint32_t z[MY_MAX][32];
 #pragma unroll
       for (int m = 0; m < MY_MAX; ++m) {
@@ -403,7 +446,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int m = 0; m < MY_MAX; ++m) {
         const int ch = wg + 2 * m;
         if (ch >= C::NCH) break;
-        if (leader) bulk_wait_read_all();  // previous reduction from this buffer has read it
+        const uint32_t stg = sb + C::OFF_STG + ch * C::STG;
+        // This chunk's buffer was last read by the reduction issued one tile ago;
+        // at most my_chunks - 1 newer reductions of this thread may still read.
+        if (leader) {
+          if (my_chunks >= 2) bulk_wait_read<1>();
+          else bulk_wait_read<0>();
+        }
         if (!wg_sync()) { ok = false; break; }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {

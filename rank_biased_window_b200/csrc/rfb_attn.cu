@@ -293,7 +293,7 @@ int dispatch_fwd_rp(int d, int rp, const Maps& m, const FwdArgs& a, int sms, cud
 
 // --------------------------------------------------------------- backward
 struct WsLayout {
-  size_t dvec, lse2, acc, total;
+  size_t dvec, lse2, acc, uprime, total;
   int npad;
 };
 
@@ -307,7 +307,8 @@ WsLayout ws_layout(int B, int H, int N, int d, int r) {
   L.dvec = 0;
   L.lse2 = vec;
   L.acc = 2 * vec;
-  L.total = L.acc + align256(bh * N * static_cast<size_t>(d + r) * sizeof(float));
+  L.uprime = L.acc + align256(bh * N * static_cast<size_t>(d + r) * sizeof(float));
+  L.total = L.uprime + align256(bh * N * static_cast<size_t>(r) * 2);
   return L;
 }
 
@@ -439,15 +440,18 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   if (!rc) rc = encode_3d(&m.k, k, d, N, BH, d, kTile, 1);
   if (!rc) rc = encode_3d(&m.v, v, d, N, BH, d, kTile, 1);
   if (!rc) rc = encode_3d(&m.g, dout, d, N, BH, d, kTile, 1);
-  if (!rc && r > 0) rc = encode_3d(&m.u, u, r, N, BH, rp, kTile, 1);
-  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, kTile, 1);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // The backward stages U' = U / s once (bwd_pre) and tiles that copy.
+  if (!rc && r > 0) rc = encode_3d(&m.u, ws + L.uprime, r, N, BH, rp, kTile, 1);
+  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, kTile, 1);
   if (!rc) rc = encode_acc_3d(&m.acc, ws + L.acc, d + r, N, BH);
   if (rc) return rc;
   BwdArgs a;
   a.o = static_cast<const __nv_bfloat16*>(o);
   a.lse = lse;
   a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.u = static_cast<const __nv_bfloat16*>(u);
+  a.uprime = reinterpret_cast<__nv_bfloat16*>(ws + L.uprime);
   a.dvec = reinterpret_cast<float*>(ws + L.dvec);
   a.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   a.acc = reinterpret_cast<float*>(ws + L.acc);
