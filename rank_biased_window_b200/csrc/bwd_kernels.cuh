@@ -317,15 +317,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // reading them must be done before this tile's S^T / dP^T overwrite them.
       if (i > 0 && !wait_warp(a_done, (i - 1) & 1, g, 41)) return false;
       tc_fence_after();
-      if (lane == 0) {
-        issue_scores<D, RP>(tmem + C::T_S, sb + C::OFF_K, st + C::S_Q, sb + C::OFF_W, st + C::S_U);
+      {
+        // S^T and dP^T K-steps alternate: consecutive MMAs then target
+        // different accumulators and can overlap in the tensor pipe.
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk) {
+          umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2),
+                    desc_kmajor(st + C::S_Q + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
           umma_bf16(tmem + C::T_DP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2),
                     desc_kmajor(st + C::S_DO + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < RP / 16; ++kk)
+          umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_W + kk * 32, RP * 2),
+                    desc_kmajor(st + C::S_U + kk * 32, RP * 2), idS, 1u);
         umma_commit(sdp_full);
       }
-      __syncwarp();
       return true;
     };
     bool ok = wait_warp(kv_full, 0, g, 32);
@@ -335,31 +342,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(ds_full, i & 1, g, 35)) break;
       tc_fence_after();
-      if (lane == 0) {
-        // A operands from TMEM: P^T over the S^T columns, dS^T over the dP^T columns.
-        issue_k128_ts<D>(tmem + C::T_DV, tmem + C::T_S, st + C::S_DO, i > 0);   // dV += P^T dO
-        issue_k128_ts<D>(tmem + C::T_DK, tmem + C::T_DP, st + C::S_Q, i > 0);   // dK += dS^T Q
-        if constexpr (RP > 0)
-          issue_k128_ts<RP>(tmem + C::T_DW, tmem + C::T_DP, st + C::S_U, i > 0);  // dW += dS^T U'
+      {
+        // A operands from TMEM: P^T over the S^T columns, dS^T over the dP^T
+        // columns.  dV += P^T dO, dK += dS^T Q, dW += dS^T U', K-steps
+        // round-robin over the three accumulators.
+        constexpr uint32_t idD = idesc_bf16_f32(128, D, false, true);
+        constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t aoff = (kk >> 2) * 64 + (kk & 3) * 8;
+          umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + aoff,
+                       desc_mnmajor(st + C::S_DO + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+          umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
+                       desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+          if constexpr (RP > 0)
+            umma_bf16_ts(tmem + C::T_DW, tmem + C::T_DP + aoff,
+                         desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+                         acc);
+        }
         umma_commit(a_done);
       }
-      __syncwarp();
       if (C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 36)) break;
       tc_fence_after();
-      if (lane == 0) {
+      {
+        // dQ = dS K and dU = dS W (A = dS^T tile read transposed), interleaved.
         const uint32_t dsb = sb + C::OFF_DS;
-        issue_k128_at<D>(tmem + C::T_DQ, dsb, sb + C::OFF_K);  // dQ = dS K
-        if constexpr (RP > 0) issue_k128_at<RP>(tmem + C::T_DQ + D, dsb, sb + C::OFF_W);  // dU = dS W
+        constexpr uint32_t idD = idesc_bf16_f32(128, D, true, true);
+        constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = desc_mnmajor(dsb + kk * 16 * 128, 128, 128 * 128);
+          umma_bf16(tmem + C::T_DQ, ad,
+                    desc_mnmajor(sb + C::OFF_K + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD,
+                    kk > 0 ? 1u : 0u);
+          if constexpr (RP > 0)
+            umma_bf16(tmem + C::T_DQ + D, ad,
+                      desc_mnmajor(sb + C::OFF_W + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+                      kk > 0 ? 1u : 0u);
+        }
         umma_commit(dq_full);
         umma_commit(q_empty(s));
       }
-      __syncwarp();
       if (i + 1 < nq && !issue_sdp(i + 1)) break;
     }
-    if (lane == 0) {
-      umma_commit(drain_bar);
-      wait_drain(drain_bar, 0, args.timeout_ns);
-    }
+    umma_commit(drain_bar);
+    wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
   } else {
     // ------------------------------------- compute warps (two warpgroups)
@@ -391,8 +419,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int c = wg * 64; c < wg * 64 + 64; c += 32) {
         uint32_t xy[64];
         tmem_ld32x2(tmem + lane_base + C::T_S + c, tmem + lane_base + C::T_DP + c, xy);
-        const uint32_t* x = xy;
+        uint32_t* x = xy;
         const uint32_t* y = xy + 32;
+        // Padding keys / queries: a score of -inf gives P = 0 and dS = 0.
+        if (!key_ok || c + 32 > qvalid) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (!key_ok || c + e >= qvalid) x[e] = 0xFF800000u;
+        }
         float p[32], ds[32];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -404,8 +438,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                __uint_as_float(dv.w)};
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const bool valid = key_ok && (c + e + t < qvalid);
-            p[e + t] = valid ? fast_exp2(fmaf(__uint_as_float(x[e + t]), sl2, -l4[t])) : 0.f;
+            p[e + t] = fast_exp2(fmaf(__uint_as_float(x[e + t]), sl2, -l4[t]));
             ds[e + t] = p[e + t] * (__uint_as_float(y[e + t]) - d4[t]);
           }
         }
@@ -419,13 +452,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dk[e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
         }
         const int pcol = wg * 64 + (c - wg * 64) / 2;
-        tmem_st16(tmem + lane_base + C::T_S + pcol, pk);
-        tmem_st16(tmem + lane_base + C::T_DP + pcol, dk);
+        tmem_st16_nowait(tmem + lane_base + C::T_S + pcol, pk);
+        tmem_st16_nowait(tmem + lane_base + C::T_DP + pcol, dk);
 #pragma unroll
         for (int e = 0; e < 32; e += 8)
           st_shared_v4(sb + C::OFF_DS + sw128_offset(row, c + e, 128), dk[e / 2], dk[e / 2 + 1],
                        dk[e / 2 + 2], dk[e / 2 + 3]);
       }
+      tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);

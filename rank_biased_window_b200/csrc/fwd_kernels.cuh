@@ -271,13 +271,10 @@ __global__ void __launch_bounds__(192, 1)
       const int a = j & 1, s = j % NS;
       if (!wait_warp(p_full(a), (j >> 1) & 1, g, 3)) return false;
       tc_fence_after();
-      if (lane == 0) {
-        issue_pv<D>(tmem + 256 + a * D, sb + C::OFF_P + a * C::PB, sb + s * C::STAGE + 2 * C::QB,
-                    false);
-        umma_commit(o_full(a));
-        umma_commit(in_empty(s));
-      }
-      __syncwarp();
+      issue_pv<D>(tmem + 256 + a * D, sb + C::OFF_P + a * C::PB, sb + s * C::STAGE + 2 * C::QB,
+                  false);
+      umma_commit(o_full(a));
+      umma_commit(in_empty(s));
       return true;
     };
     int it = 0;
@@ -292,18 +289,13 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (it >= 2 && !wait_warp(acc_empty(a), ((it >> 1) + 1) & 1, g, 4)) { ok = false; break; }
       tc_fence_after();
-      if (lane == 0) {
-        issue_scores<D, RP>(tmem + a * 128, st, st + C::QB, st + 3 * C::QB, st + 3 * C::QB + C::UB);
-        umma_commit(s_full(a));
-      }
-      __syncwarp();
+      issue_scores<D, RP>(tmem + a * 128, st, st + C::QB, st + 3 * C::QB, st + 3 * C::QB + C::UB);
+      umma_commit(s_full(a));
       if (it > 0 && !do_pv(it - 1)) { ok = false; break; }
     }
     if (ok && it > 0) do_pv(it - 1);
-    if (lane == 0) {
-      umma_commit(drain_bar);
-      wait_drain(drain_bar, 0, args.timeout_ns);
-    }
+    umma_commit(drain_bar);
+    wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
   } else {
     // ------------------------------------------------- softmax + epilogue
@@ -480,25 +472,19 @@ __global__ void __launch_bounds__(192, 1)
       if (!wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
       if (j >= 2 && !wait_warp(s_empty(b), ((j >> 1) + 1) & 1, g, 14)) return false;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-        issue_scores<D, RP>(tmem + b * 128, sb + C::OFF_Q, st, sb + C::OFF_U, st + 2 * C::QB);
-        umma_commit(s_full(b));
-      }
-      __syncwarp();
+      const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+      issue_scores<D, RP>(tmem + b * 128, sb + C::OFF_Q, st, sb + C::OFF_U, st + 2 * C::QB);
+      umma_commit(s_full(b));
       return true;
     };
     auto do_pv = [&](int j) -> bool {
       const int s = j % NS, b = j & 1;
       if (!wait_warp(p_full(b), (j >> 1) & 1, g, 15)) return false;
       tc_fence_after();
-      if (lane == 0) {
-        issue_pv<D>(tmem + 256, sb + C::OFF_P + b * C::PB, sb + C::OFF_STAGE + s * C::STAGE + C::QB,
-                    j > 0);
-        umma_commit(kv_empty(s));
-        umma_commit(pv_done(b));
-      }
-      __syncwarp();
+      issue_pv<D>(tmem + 256, sb + C::OFF_P + b * C::PB, sb + C::OFF_STAGE + s * C::STAGE + C::QB,
+                  j > 0);
+      umma_commit(kv_empty(s));
+      umma_commit(pv_done(b));
       return true;
     };
     if (ok) ok = do_s(0);
@@ -506,10 +492,8 @@ __global__ void __launch_bounds__(192, 1)
       if (j + 1 < nkv && !do_s(j + 1)) break;
       if (!do_pv(j)) break;
     }
-    if (lane == 0) {
-      umma_commit(drain_bar);
-      wait_drain(drain_bar, 0, args.timeout_ns);
-    }
+    umma_commit(drain_bar);
+    wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
   } else {
     const int row = threadIdx.x;
