@@ -11,9 +11,9 @@
 //     [dQ | dU] = dS . [K | W] with per-column scales (s | 1).
 //
 // Three kernels:
-//   bwd_pre  : D_i = rowsum(dO o O) (equal to sum_j P_ij dP_ij because O = P V),
-//              LSE_i log2(e), U' = bf16(U / s), and zeroes the fp32 dQ|dU
-//              accumulator.
+//   bwd_pre  : D_i = rowsum(dO o O) (equal to sum_j P_ij dP_ij because O = P V)
+//              and LSE_i log2(e), both stored negated, U' = bf16(U / s), and
+//              zeroes the fp32 dQ|dU accumulator.
 //   bwd_main : one CTA per (head, 128-key tile); K, W, V stay in shared memory,
 //              dV, dK, dW accumulate in TMEM across all 128-query tiles.  Per
 //              query tile: S^T and dP^T by tcgen05 into TMEM; two compute
@@ -23,8 +23,10 @@
 //              the partial dQ|dU tile goes to TMEM columns of its own (when
 //              they fit), which
 //              the compute warps stage in 128-byte-swizzled shared memory and
-//              add into the fp32 accumulator with TMA bulk tensor reductions,
-//              while the next tile's S^T / dP^T MMAs run.
+//              add into the fp32 accumulator with TMA bulk tensor reductions.
+//              The reduction of tile i runs after the softmax of tile i + 1,
+//              overlapping tile i + 1's MMAs; all MMAs are issued by one
+//              converged warp.
 //   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]).
 #pragma once
 #include "fwd_kernels.cuh"
@@ -39,8 +41,8 @@ struct BwdArgs {
   const __nv_bfloat16* dout;  // [BH, N, D]
   const __nv_bfloat16* u;     // [BH, N, r]   bias factor U
   __nv_bfloat16* uprime;      // [BH, N, r]   U' = bf16(U / s), written by bwd_pre
-  float* dvec;                // [BH, Npad]   D_i
-  float* lse2;                // [BH, Npad]   LSE_i * log2(e)
+  float* dvec;                // [BH, Npad]   -D_i
+  float* lse2;                // [BH, Npad]   -LSE_i * log2(e)
   float* acc;                 // [BH, N, D + r] fp32 dQ | dU accumulator
   __nv_bfloat16* dq;          // [BH, N, D]
   __nv_bfloat16* dk;          // [BH, N, D]
@@ -66,7 +68,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
        row += static_cast<long>(gridDim.x) * rows_per_block) {
     const int bh = static_cast<int>(row / a.Npad);
     const int i = static_cast<int>(row % a.Npad);
-    float dsum = 0.f, l2 = 0.f;
+    float dsum = 0.f, l2 = 0.f;  // stored negated: -D_i and -LSE_i log2(e)
     if (i < a.N) {
       const size_t base = (static_cast<size_t>(bh) * a.N + i) * a.D + sub * 8;
       const uint4 ov = *reinterpret_cast<const uint4*>(a.o + base);
@@ -82,8 +84,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
     }
     for (int off = G / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off, G);
     if (sub == 0) {
-      a.dvec[row] = dsum;
-      a.lse2[row] = l2;
+      a.dvec[row] = -dsum;
+      a.lse2[row] = -l2;
     }
   }
   // Zero the dQ | dU accumulator.
@@ -130,47 +132,6 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdArgs a) {
   }
 }
 
-// Contraction over 128 rows of K-major A (two 64-column blocks, 128-byte
-// swizzle) with an MN-major B whose rows are NN elements wide:
-//     D[128 x NN] (+)= A[128 x 128] . B[128 x NN]
-template <int NN>
-__device__ __forceinline__ void issue_k128(uint32_t d_tmem, uint32_t a, uint32_t b, bool accumulate) {
-  constexpr uint32_t id = idesc_bf16_f32(128, NN, false, true);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint64_t ad = desc_kmajor(a + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 128);
-    const uint64_t bd = desc_mnmajor(b + kk * 16 * (NN * 2), NN * 2, 128 * NN * 2);
-    umma_bf16(d_tmem, ad, bd, id, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-// Same contraction with A = a 128 x 128 bf16 tile held in TMEM (lane = row,
-// two elements per column), laid out as two 64-column halves of 32 columns
-// each at a_tmem and a_tmem + 64 (the in-place layout the compute warpgroups
-// write): K-step kk reads columns (kk / 4) * 64 + (kk % 4) * 8.
-template <int NN>
-__device__ __forceinline__ void issue_k128_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
-                                              bool accumulate) {
-  constexpr uint32_t id = idesc_bf16_f32(128, NN, false, true);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint64_t bd = desc_mnmajor(b + kk * 16 * (NN * 2), NN * 2, 128 * NN * 2);
-    umma_bf16_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, bd, id,
-                 (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-// Same contraction with A read transposed: the tile stored for dS^T (rows =
-// keys, queries contiguous) is used as MN-major A = dS (rows = queries).
-template <int NN>
-__device__ __forceinline__ void issue_k128_at(uint32_t d_tmem, uint32_t a, uint32_t b) {
-  constexpr uint32_t id = idesc_bf16_f32(128, NN, true, true);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint64_t ad = desc_mnmajor(a + kk * 16 * 128, 128, 128 * 128);
-    const uint64_t bd = desc_mnmajor(b + kk * 16 * (NN * 2), NN * 2, 128 * NN * 2);
-    umma_bf16(d_tmem, ad, bd, id, kk > 0 ? 1u : 0u);
-  }
-}
-
 template <int D, int RP>
 struct BwdCfg {
   static constexpr int QB = kTile * D * 2;
@@ -179,27 +140,30 @@ struct BwdCfg {
   static constexpr int OFF_V = QB;
   static constexpr int OFF_W = 2 * QB;
   static constexpr int KVB = 2 * QB + UB;
-  // stage: Q, dO, U, lse2[128], dvec[128]
+  // stage: Q, dO, U', -LSE log2(e) [128], -D [128]
   static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UB, S_DV = S_L2 + 512;
   static constexpr int STAGE = 2 * QB + UB + 1024;
-  static constexpr int PB = kTile * kTile * 2;  // dS tile (bf16)
+  static constexpr int PB = kTile * kTile * 2;  // one dS tile (bf16)
   static constexpr int STG = kTile * 32 * 4;    // one 128 x 32 fp32 staging buffer
-  // dQ | dU chunks of 32 columns, one staging buffer each
-  static constexpr int NCH = (D + RP + 31) / 32;
-  static constexpr int NS_FIT = (226 * 1024 - KVB - PB - NCH * STG) / STAGE;
+  static constexpr int NCH = (D + RP + 31) / 32;  // dQ | dU chunks of 32 columns
+  // TMEM columns.  When dQ | dU fit in columns of their own, the dQ reduction
+  // of tile i is deferred until after the softmax of tile i + 1 (DEFER): the
+  // next tile's S^T / dP^T MMAs are issued before tile i's dQ | dU MMAs, so
+  // the dS tile in shared memory is double buffered.  Otherwise dQ | dU reuse
+  // the S^T columns and each tile runs its phases in order.
+  static constexpr int T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D, T_DW = 256 + 2 * D;
+  static constexpr bool DEFER = (256 + 2 * D + RP + NCH * 32) <= 512;
+  static constexpr int T_DQ = DEFER ? 256 + 2 * D + RP : 0;
+  static constexpr int NDS = DEFER ? 2 : 1;
+  static constexpr int NS_FIT = (226 * 1024 - KVB - NDS * PB - 2 * STG) / STAGE;
   static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
   static constexpr int OFF_STAGE = KVB;
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_STG = OFF_DS + PB;
-  static constexpr int OFF_BAR = OFF_STG + NCH * STG;
+  static constexpr int OFF_STG = OFF_DS + NDS * PB;
+  static constexpr int OFF_BAR = OFF_STG + 2 * STG;
   // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain wg_sync[2] a_done
   static constexpr int NBAR = 2 * NS + 9;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  // TMEM columns.  dQ | dU get their own columns when they fit, so the next
-  // query tile's S^T / dP^T MMAs need not wait for the dQ reduction.
-  static constexpr int T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D, T_DW = 256 + 2 * D;
-  static constexpr bool SEP_DQ = (256 + 2 * D + RP + NCH * 32) <= 512;
-  static constexpr int T_DQ = SEP_DQ ? 256 + 2 * D + RP : 0;
   static_assert(NS >= 1, "shared memory budget");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
   static_assert(T_DW + RP <= 512 && NCH * 32 <= 128, "TMEM budget");
@@ -231,6 +195,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto wg_bar = [&](int w) { return bar0 + 8u * (6 + 2 * NS + w); };
   // Completes when the MMAs reading P^T / dS^T from TMEM (dV, dK, dW) are done.
   const uint32_t a_done = bar0 + 8u * (8 + 2 * NS);
+  auto ds_buf = [&](int i) { return sb + C::OFF_DS + (C::NDS == 2 ? (i & 1) : 0) * C::PB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -305,86 +270,93 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         wait_drain(q_full(j % NS), (j / NS) & 1, args.timeout_ns);
     }
   } else if (warp == 9) {
-    // ----------------------------------------------------------- MMA issue
+    // ------------------------------------------------ MMA issue (whole warp)
     constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
     // S^T / s = K Q^T + W U'^T and dP^T = V dO^T for query tile i.
     auto issue_sdp = [&](int i) -> bool {
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) return false;
-      if (!C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
+      if (!C::DEFER && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
       // P^T / dS^T of the previous tile live in the S^T / dP^T columns: the MMAs
       // reading them must be done before this tile's S^T / dP^T overwrite them.
       if (i > 0 && !wait_warp(a_done, (i - 1) & 1, g, 41)) return false;
       tc_fence_after();
-      {
-        // S^T and dP^T K-steps alternate: consecutive MMAs then target
-        // different accumulators and can overlap in the tensor pipe.
+      // S^T and dP^T K-steps alternate between the two accumulators.
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2),
-                    desc_kmajor(st + C::S_Q + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
-          umma_bf16(tmem + C::T_DP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2),
-                    desc_kmajor(st + C::S_DO + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < RP / 16; ++kk)
-          umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_W + kk * 32, RP * 2),
-                    desc_kmajor(st + C::S_U + kk * 32, RP * 2), idS, 1u);
-        umma_commit(sdp_full);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2),
+                  desc_kmajor(st + C::S_Q + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
+        umma_bf16(tmem + C::T_DP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2),
+                  desc_kmajor(st + C::S_DO + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
       }
+#pragma unroll
+      for (int kk = 0; kk < RP / 16; ++kk)
+        umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_W + kk * 32, RP * 2),
+                  desc_kmajor(st + C::S_U + kk * 32, RP * 2), idS, 1u);
+      umma_commit(sdp_full);
       return true;
+    };
+    // dV += P^T dO, dK += dS^T Q, dW += dS^T U' with A read from TMEM (P^T over
+    // the S^T columns, dS^T over the dP^T columns), K-steps round-robin.
+    auto issue_grad_kv = [&](int i) {
+      const uint32_t st = sb + C::OFF_STAGE + (i % NS) * C::STAGE;
+      constexpr uint32_t idD = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        const uint32_t aoff = (kk >> 2) * 64 + (kk & 3) * 8;
+        umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + aoff,
+                     desc_mnmajor(st + C::S_DO + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+        umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
+                     desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+        if constexpr (RP > 0)
+          umma_bf16_ts(tmem + C::T_DW, tmem + C::T_DP + aoff,
+                       desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+                       acc);
+      }
+      umma_commit(a_done);
+      umma_commit(q_empty(i % NS));  // Q, dO, U' of this tile are no longer read
+    };
+    // dQ = dS K and dU = dS W (A = the dS^T tile read transposed), interleaved.
+    auto issue_grad_q = [&](int i) {
+      const uint32_t dsb = ds_buf(i);
+      constexpr uint32_t idD = idesc_bf16_f32(128, D, true, true);
+      constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, true, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t ad = desc_mnmajor(dsb + kk * 16 * 128, 128, 128 * 128);
+        umma_bf16(tmem + C::T_DQ, ad,
+                  desc_mnmajor(sb + C::OFF_K + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD,
+                  kk > 0 ? 1u : 0u);
+        if constexpr (RP > 0)
+          umma_bf16(tmem + C::T_DQ + D, ad,
+                    desc_mnmajor(sb + C::OFF_W + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+                    kk > 0 ? 1u : 0u);
+      }
+      umma_commit(dq_full);
     };
     bool ok = wait_warp(kv_full, 0, g, 32);
     if (ok && nq > 0) ok = issue_sdp(0);
     for (int i = 0; ok && i < nq; ++i) {
-      const int s = i % NS;
-      const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(ds_full, i & 1, g, 35)) break;
       tc_fence_after();
-      {
-        // A operands from TMEM: P^T over the S^T columns, dS^T over the dP^T
-        // columns.  dV += P^T dO, dK += dS^T Q, dW += dS^T U', K-steps
-        // round-robin over the three accumulators.
-        constexpr uint32_t idD = idesc_bf16_f32(128, D, false, true);
-        constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, false, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t aoff = (kk >> 2) * 64 + (kk & 3) * 8;
-          umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + aoff,
-                       desc_mnmajor(st + C::S_DO + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
-          umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
-                       desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
-          if constexpr (RP > 0)
-            umma_bf16_ts(tmem + C::T_DW, tmem + C::T_DP + aoff,
-                         desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
-                         acc);
-        }
-        umma_commit(a_done);
+      issue_grad_kv(i);
+      if constexpr (C::DEFER) {
+        // Next tile's scores first, then this tile's dQ | dU (its reduction
+        // happens after the next softmax).
+        if (i + 1 < nq && !issue_sdp(i + 1)) break;
+        if (i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 36)) break;
+        tc_fence_after();
+        issue_grad_q(i);
+      } else {
+        // dQ | dU overwrite the S^T columns that dV / dK / dW read P^T from.
+        if (!wait_warp(a_done, i & 1, g, 42)) break;
+        tc_fence_after();
+        issue_grad_q(i);
+        if (i + 1 < nq && !issue_sdp(i + 1)) break;
       }
-      if (C::SEP_DQ && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 36)) break;
-      tc_fence_after();
-      {
-        // dQ = dS K and dU = dS W (A = dS^T tile read transposed), interleaved.
-        const uint32_t dsb = sb + C::OFF_DS;
-        constexpr uint32_t idD = idesc_bf16_f32(128, D, true, true);
-        constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = desc_mnmajor(dsb + kk * 16 * 128, 128, 128 * 128);
-          umma_bf16(tmem + C::T_DQ, ad,
-                    desc_mnmajor(sb + C::OFF_K + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD,
-                    kk > 0 ? 1u : 0u);
-          if constexpr (RP > 0)
-            umma_bf16(tmem + C::T_DQ + D, ad,
-                      desc_mnmajor(sb + C::OFF_W + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
-                      kk > 0 ? 1u : 0u);
-        }
-        umma_commit(dq_full);
-        umma_commit(q_empty(s));
-      }
-      if (i + 1 < nq && !issue_sdp(i + 1)) break;
     }
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0, args.timeout_ns);
@@ -395,10 +367,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = threadIdx.x & 127;         // TMEM lane == key row (S^T) == query row (dQ)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const bool key_ok = (k0 + row) < N;
-    const float sl2 = args.scale_log2;
+    const uint64_t sl2x2 = f2_pack(args.scale_log2, args.scale_log2);
     const bool leader = (threadIdx.x & 127) == 0;  // issues this warpgroup's reductions
-    constexpr int MY_MAX = (C::NCH + 1) / 2;
-    const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
+    const uint32_t stg = sb + C::OFF_STG + wg * C::STG;
     uint32_t wg_phase = 0;
     // Bounded barrier over this warpgroup's 128 threads.
     auto wg_sync = [&]() -> bool {
@@ -407,67 +378,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ++wg_phase;
       return r;
     };
-    bool ok = true;
-    for (int i = 0; i < nq; ++i) {
+    // P^T = 2^(S^T s log2e - LSE log2e), dS^T = P^T o (dP^T - D) for this
+    // warpgroup's 64 query columns of tile i; P^T and dS^T go back into TMEM in
+    // place (packed bf16, columns wg*64 + [0, 32)), dS^T also into shared memory.
+    auto softmax = [&](int i) -> bool {
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-      if (!wait_warp(q_full(s), (i / NS) & 1, g, 37)) { ok = false; break; }
-      if (!wait_warp(sdp_full, i & 1, g, 38)) { ok = false; break; }
+      if (!wait_warp(q_full(s), (i / NS) & 1, g, 37)) return false;
+      if (!wait_warp(sdp_full, i & 1, g, 38)) return false;
       tc_fence_after();
       const int qvalid = N - i * kTile;
+      const uint32_t dsb = ds_buf(i);
 #pragma unroll 1
       for (int c = wg * 64; c < wg * 64 + 64; c += 32) {
         uint32_t xy[64];
         tmem_ld32x2(tmem + lane_base + C::T_S + c, tmem + lane_base + C::T_DP + c, xy);
-        uint32_t* x = xy;
-        const uint32_t* y = xy + 32;
         // Padding keys / queries: a score of -inf gives P = 0 and dS = 0.
         if (!key_ok || c + 32 > qvalid) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (!key_ok || c + e >= qvalid) x[e] = 0xFF800000u;
+            if (!key_ok || c + e >= qvalid) xy[e] = 0xFF800000u;
         }
-        float p[32], ds[32];
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const uint4 lv = ld_shared_v4(st + C::S_L2 + (c + e) * 4);
-          const uint4 dv = ld_shared_v4(st + C::S_DV + (c + e) * 4);
-          const float l4[4] = {__uint_as_float(lv.x), __uint_as_float(lv.y), __uint_as_float(lv.z),
-                               __uint_as_float(lv.w)};
-          const float d4[4] = {__uint_as_float(dv.x), __uint_as_float(dv.y), __uint_as_float(dv.z),
-                               __uint_as_float(dv.w)};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            p[e + t] = fast_exp2(fmaf(__uint_as_float(x[e + t]), sl2, -l4[t]));
-            ds[e + t] = p[e + t] * (__uint_as_float(y[e + t]) - d4[t]);
-          }
-        }
-        // P^T and dS^T as packed bf16 into TMEM, in place over the columns this
-        // warpgroup has already read (columns wg*64 + [0, 32)); dS^T also into
-        // shared memory, where the dQ MMA reads it transposed.
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          pk[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
-          dk[e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
+        for (int e = 0; e < 32; e += 4) {
+          const uint4 nl = ld_shared_v4(st + C::S_L2 + (c + e) * 4);  // -LSE log2e
+          const uint4 nd = ld_shared_v4(st + C::S_DV + (c + e) * 4);  // -D
+#pragma unroll
+          for (int t = 0; t < 4; t += 2) {
+            const uint64_t nl2 = (t == 0) ? (static_cast<uint64_t>(nl.y) << 32 | nl.x)
+                                          : (static_cast<uint64_t>(nl.w) << 32 | nl.z);
+            const uint64_t nd2 = (t == 0) ? (static_cast<uint64_t>(nd.y) << 32 | nd.x)
+                                          : (static_cast<uint64_t>(nd.w) << 32 | nd.z);
+            const uint64_t x2 = static_cast<uint64_t>(xy[e + t + 1]) << 32 | xy[e + t];
+            const uint64_t y2 = static_cast<uint64_t>(xy[32 + e + t + 1]) << 32 | xy[32 + e + t];
+            const float2 arg = f2_unpack(f2_fma(x2, sl2x2, nl2));
+            const float p0 = fast_exp2(arg.x), p1 = fast_exp2(arg.y);
+            const float2 ds = f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(y2, nd2)));
+            pk[(e + t) >> 1] = pack_bf16x2(p0, p1);
+            dk[(e + t) >> 1] = pack_bf16x2(ds.x, ds.y);
+          }
         }
         const int pcol = wg * 64 + (c - wg * 64) / 2;
         tmem_st16_nowait(tmem + lane_base + C::T_S + pcol, pk);
         tmem_st16_nowait(tmem + lane_base + C::T_DP + pcol, dk);
 #pragma unroll
         for (int e = 0; e < 32; e += 8)
-          st_shared_v4(sb + C::OFF_DS + sw128_offset(row, c + e, 128), dk[e / 2], dk[e / 2 + 1],
+          st_shared_v4(dsb + sw128_offset(row, c + e, 128), dk[e / 2], dk[e / 2 + 1],
                        dk[e / 2 + 2], dk[e / 2 + 3]);
       }
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
-      // Partial dQ | dU of this query tile (TMEM lane = query row): this
-      // warpgroup takes chunks wg, wg + 2, ... of 32 columns, reads them all,
-      // frees the TMEM columns, then reduces each through its staging buffer.
-      if (!wait_warp(dq_full, i & 1, g, 39)) { ok = false; break; }
+      return true;
+    };
+    // Partial dQ | dU of tile j (TMEM lane = query row): this warpgroup reads its
+    // chunks (wg, wg + 2, ... of 32 columns), frees the TMEM columns, then
+    // stages each chunk in its 128-byte-swizzled buffer and reduces it into the
+    // fp32 accumulator with one TMA bulk tensor reduction.
+    auto reduce_dq = [&](int j) -> bool {
+      if (!wait_warp(dq_full, j & 1, g, 39)) return false;
       tc_fence_after();
+      constexpr int MY_MAX = (C::NCH + 1) / 2;
       uint32_t z[MY_MAX][32];
 #pragma unroll
       for (int m = 0; m < MY_MAX; ++m) {
@@ -480,36 +453,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int m = 0; m < MY_MAX; ++m) {
         const int ch = wg + 2 * m;
         if (ch >= C::NCH) break;
-        const uint32_t stg = sb + C::OFF_STG + ch * C::STG;
-        // This chunk's buffer was last read by the reduction issued one tile ago;
-        // at most my_chunks - 1 newer reductions of this thread may still read.
-        if (leader) {
-          if (my_chunks >= 2) bulk_wait_read<1>();
-          else bulk_wait_read<0>();
-        }
-        if (!wg_sync()) { ok = false; break; }
+        if (leader) bulk_wait_read_all();  // the previous reduction has read the buffer
+        if (!wg_sync()) return false;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int q = 0; q < 8; ++q) {
           float v4[4];
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const int col = ch * 32 + j * 4 + t;
-            v4[t] = __uint_as_float(z[m][j * 4 + t]) * (col < D ? args.scale : 1.0f);
+            const int col = ch * 32 + q * 4 + t;
+            v4[t] = __uint_as_float(z[m][q * 4 + t]) * (col < D ? args.scale : 1.0f);
           }
-          st_shared_v4(stg + row * 128 + ((j ^ (row & 7)) << 4), __float_as_uint(v4[0]),
+          st_shared_v4(stg + row * 128 + ((q ^ (row & 7)) << 4), __float_as_uint(v4[0]),
                        __float_as_uint(v4[1]), __float_as_uint(v4[2]), __float_as_uint(v4[3]));
         }
         fence_async_smem();
-        if (!wg_sync()) { ok = false; break; }
+        if (!wg_sync()) return false;
         if (leader) {
-          tma_reduce_add_3d(&mAcc, stg, ch * 32, i * kTile, bh);
+          tma_reduce_add_3d(&mAcc, stg, ch * 32, j * kTile, bh);
           bulk_commit();
         }
       }
+      return true;
+    };
+    bool ok = true;
+    for (int i = 0; ok && i < nq; ++i) {
+      ok = softmax(i);
       if (!ok) break;
+      if constexpr (C::DEFER) {
+        if (i > 0) ok = reduce_dq(i - 1);
+      } else {
+        ok = reduce_dq(i);
+      }
     }
+    if (C::DEFER && ok && nq > 0) ok = reduce_dq(nq - 1);
     if (ok && nq > 0) {
-      // dq_full of the last tile implies all dV, dK, dW MMAs have completed.
+      // The last dq_full implies all dV, dK, dW MMAs have completed.
       const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
       if (wg == 0) {
         uint32_t gv[D];
