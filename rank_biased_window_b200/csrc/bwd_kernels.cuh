@@ -370,6 +370,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t sl2x2 = f2_pack(args.scale_log2, args.scale_log2);
     const bool leader = (threadIdx.x & 127) == 0;  // issues this warpgroup's reductions
     const uint32_t stg = sb + C::OFF_STG + wg * C::STG;
+    const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
     uint32_t wg_phase = 0;
     // Bounded barrier over this warpgroup's 128 threads.
     auto wg_sync = [&]() -> bool {
@@ -387,6 +388,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!wait_warp(q_full(s), (i / NS) & 1, g, 37)) return false;
       if (!wait_warp(sdp_full, i & 1, g, 38)) return false;
       tc_fence_after();
+      if constexpr (C::DEFER) {
+        // Block wg of this dS buffer staged dQ | dU chunk wg of tile i - 2; the
+        // reduction reading it is followed by (2 * my_chunks - 1) newer ones.
+        if (i >= 2) {
+          if (leader) {
+            if (my_chunks >= 2) bulk_wait_read<3>();
+            else bulk_wait_read<1>();
+          }
+          if (!wg_sync()) return false;
+        }
+      }
       const int qvalid = N - i * kTile;
       const uint32_t dsb = ds_buf(i);
 #pragma unroll 1
@@ -453,8 +465,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int m = 0; m < MY_MAX; ++m) {
         const int ch = wg + 2 * m;
         if (ch >= C::NCH) break;
-        if (leader) bulk_wait_read_all();  // the previous reduction has read the buffer
-        if (!wg_sync()) return false;
+        uint32_t buf = stg;
+        if (C::DEFER && m == 0) {
+          // This warpgroup's first chunk goes into its own 64-query block of the
+          // dS buffer of tile j, free now that dQ_j's MMAs have read it (dq_full)
+          // and the reduction staged there earlier was awaited by softmax(j).
+          buf = ds_buf(j) + wg * (kTile * 128);
+        } else {
+          if (leader) {
+            if (C::DEFER) bulk_wait_read<1>();  // only this tile's first chunk may still read
+            else bulk_wait_read_all();
+          }
+          if (!wg_sync()) return false;
+        }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           float v4[4];
@@ -463,13 +486,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int col = ch * 32 + q * 4 + t;
             v4[t] = __uint_as_float(z[m][q * 4 + t]) * (col < D ? args.scale : 1.0f);
           }
-          st_shared_v4(stg + row * 128 + ((q ^ (row & 7)) << 4), __float_as_uint(v4[0]),
+          st_shared_v4(buf + row * 128 + ((q ^ (row & 7)) << 4), __float_as_uint(v4[0]),
                        __float_as_uint(v4[1]), __float_as_uint(v4[2]), __float_as_uint(v4[3]));
         }
         fence_async_smem();
         if (!wg_sync()) return false;
         if (leader) {
-          tma_reduce_add_3d(&mAcc, stg, ch * 32, j * kTile, bh);
+          tma_reduce_add_3d(&mAcc, buf, ch * 32, j * kTile, bh);
           bulk_commit();
         }
       }
