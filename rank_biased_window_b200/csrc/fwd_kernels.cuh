@@ -16,11 +16,13 @@
 //     128/NP whole windows (NP = 64 or 128 rows per window).  One S tile per
 //     tile, single-pass softmax, block-diagonal P (off-window blocks stay 0).
 //   * fwd_long_kernel    (N > 128): one CTA per (head, 128-query tile); loops
-//     over 128-key tiles with an online softmax (lazy rescale of O in TMEM).
+//     over 128-key tiles with an online softmax (lazy rescale of O in TMEM);
+//     two softmax warpgroups split each score tile by key columns.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue (thread = row =
-// TMEM lane), warp 4 TMA producer, warp 5 U' scaling + MMA issue (lane 0) +
-// TMEM allocation.  Operands are staged by TMA with the swizzle that matches
+// Window kernel warp roles (192 threads): warps 0-3 softmax + epilogue (thread
+// = row = TMEM lane), warp 4 TMA producer, warp 5 U' scaling + MMA issue +
+// TMEM allocation.  The long kernel uses 320 threads: warps 0-7 softmax (two
+// warpgroups), warp 8 TMA, warp 9 MMA.  Operands are staged by TMA with the swizzle that matches
 // their row width; P is written by the softmax threads into a 128-byte
 // swizzled K-major tile.
 #pragma once
@@ -367,21 +369,33 @@ struct LongCfg {
   static constexpr int OFF_U = QB;
   static constexpr int OFF_STAGE = QB + UB;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_BAR = OFF_P + 2 * PB;
+  static constexpr int OFF_X = OFF_P + 2 * PB;     // row-statistics exchange, fp32
+  static constexpr int X_BYTES = (2 * 2 + 2) * kTile * 4;  // max[2 tiles][2 wg], sum[2 wg]
+  static constexpr int OFF_BAR = OFF_X + X_BYTES;
   // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
-  static constexpr int NBAR = 2 * NS + 10;
+  // mx_bar[2] end_bar
+  static constexpr int NBAR = 2 * NS + 13;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static constexpr int OC = D / 2;  // O columns each softmax warpgroup owns
   static_assert(NS >= 2, "not enough shared memory for two KV stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
 };
 
+constexpr int kLongThreads = 320;  // warps 0-7 softmax (two warpgroups), 8 TMA, 9 MMA
+
+// Long regime: one CTA per (head, 128-query tile), looping over 128-key tiles.
+// The two softmax warpgroups split each score tile by key columns (64 each):
+// they exchange per-row partial maxima through shared memory (bounded
+// barrier), keep partial row sums, and each owns half of O's columns for the
+// lazy rescale and the epilogue.
 template <int D, int RP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kLongThreads, 1)
     fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
                     const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
   using C = LongCfg<D, RP>;
   constexpr int NS = C::NS;
+  constexpr int OC = C::OC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   const uint32_t sb = smem_u32(smem);
@@ -394,6 +408,10 @@ __global__ void __launch_bounds__(192, 1)
   auto p_full = [&](int b) { return bar0 + 8u * (5 + 2 * NS + b); };
   auto pv_done = [&](int b) { return bar0 + 8u * (7 + 2 * NS + b); };
   const uint32_t drain_bar = bar0 + 8u * (9 + 2 * NS);
+  auto mx_bar = [&](int b) { return bar0 + 8u * (10 + 2 * NS + b); };
+  const uint32_t end_bar = bar0 + 8u * (12 + 2 * NS);
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_X);              // [2][2][128]
+  float* xsum = reinterpret_cast<float*>(smem + C::OFF_X + 4 * kTile * 4);  // [2][128]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -413,14 +431,16 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
-      mbar_init(s_empty(b), 128);
-      mbar_init(p_full(b), 128);
+      mbar_init(s_empty(b), 256);
+      mbar_init(p_full(b), 256);
       mbar_init(pv_done(b), 1);
+      mbar_init(mx_bar(b), 256);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(end_bar, 256);
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch(&mQ);
     tma_prefetch(&mK);
     tma_prefetch(&mV);
@@ -429,7 +449,7 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch(&mW);
     }
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -439,7 +459,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       mbar_expect_tx(q_full, C::QB + C::UB);
       tma_load_3d(sb + C::OFF_Q, &mQ, q_full, 0, q0, bh);
@@ -458,7 +478,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = (j > NS ? j - NS : 0); i < j; ++i)
         wait_drain(kv_full(i % NS), (i / NS) & 1, args.timeout_ns);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     bool ok = wait_warp(q_full, 0, g, 12);
     if (ok) {
       if constexpr (RP > 0) {
@@ -496,8 +516,9 @@ __global__ void __launch_bounds__(192, 1)
     wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
   } else {
-    const int row = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int wg = warp >> 2;            // key columns wg*64 .. wg*64+63
+    const int row = threadIdx.x & 127;   // TMEM lane == query row
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = args.scale_log2;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
@@ -505,13 +526,18 @@ __global__ void __launch_bounds__(192, 1)
       const int b = j & 1;
       if (!wait_warp(s_full(b), (j >> 1) & 1, g, 16)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[128];
-      tmem_ld_cols<128>(tmem + lane_base + b * 128, sv);
+      uint32_t sv[64];
+      tmem_ld64(tmem + lane_base + b * 128 + wg * 64, sv);
       tc_fence_before();
       mbar_arrive(s_empty(b));
-      const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
-      if (kvalid < kTile) mask_tail<128>(sv, kvalid);
-      const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);
+      const int kvalid = N - j * kTile - wg * 64;  // valid keys in this half (may be <= 0)
+      if (kvalid < 64) mask_tail<64>(sv, kvalid);
+      // Row maximum over the full 128 keys: exchange the two halves' maxima.
+      xmax[(b * 2 + wg) * kTile + row] = row_max<64>(sv);
+      mbar_arrive(mx_bar(b));
+      if (!wait_warp(mx_bar(b), (j >> 1) & 1, g, 20)) { ok = false; break; }
+      const float mx = fmaxf(xmax[(b * 2 + wg) * kTile + row], xmax[(b * 2 + (wg ^ 1)) * kTile + row]);
+      const float m_new = fmaxf(m_run, mx * sl2);
       // Lazy rescale: keep the running max unless it grew by more than 2^8.
       const bool need = m_new > m_run + 8.0f;
       float alpha = 1.f;
@@ -522,17 +548,17 @@ __global__ void __launch_bounds__(192, 1)
       }
       const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
       if (j >= 2 && !wait_warp(pv_done(b), ((j >> 1) + 1) & 1, g, 17)) { ok = false; break; }
-      l += exp_row_to_smem<128>(sv, sl2, m_run, sb + C::OFF_P + b * C::PB, row, 0);
+      l += exp_row_to_smem<64>(sv, sl2, m_run, sb + C::OFF_P + b * C::PB, row, wg * 64);
       if (fix_o) {
         // O holds the sum through tile j-1 at the old running max: wait for that
-        // PV to land, then rescale this thread's row in place.
+        // PV to land, then rescale this thread's half row in place.
         if (!wait_warp(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, g, 18)) { ok = false; break; }
         tc_fence_after();
-        uint32_t ov[D];
-        tmem_ld_cols<D>(tmem + lane_base + 256, ov);
+        uint32_t ov[OC];
+        tmem_ld_cols<OC>(tmem + lane_base + 256 + wg * OC, ov);
 #pragma unroll
-        for (int c = 0; c < D; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-        tmem_st_cols<D>(tmem + lane_base + 256, ov);
+        for (int c = 0; c < OC; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+        tmem_st_cols<OC>(tmem + lane_base + 256 + wg * OC, ov);
       }
       fence_async_smem();
       tc_fence_before();
@@ -541,14 +567,19 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) {
       const int jl = nkv - 1;
       if (wait_warp(pv_done(jl & 1), (jl >> 1) & 1, g, 19)) {
-        tc_fence_after();
-        uint32_t ov[D];
-        tmem_ld_cols<D>(tmem + lane_base + 256, ov);
-        const int q = q0 + row;
-        if (q < N) {
-          const size_t r = static_cast<size_t>(bh) * N + q;
-          store_o_row<D>(args.o + r * D, ov, 1.0f / l);
-          args.lse[r] = (m_run + __log2f(l)) * kLn2;
+        xsum[wg * kTile + row] = l;
+        mbar_arrive(end_bar);
+        if (wait_warp(end_bar, 0, g, 21)) {
+          const float lt = xsum[row] + xsum[kTile + row];
+          tc_fence_after();
+          uint32_t ov[OC];
+          tmem_ld_cols<OC>(tmem + lane_base + 256 + wg * OC, ov);
+          const int q = q0 + row;
+          if (q < N) {
+            const size_t r = static_cast<size_t>(bh) * N + q;
+            store_o_row<OC>(args.o + r * D + wg * OC, ov, 1.0f / lt);
+            if (wg == 0) args.lse[r] = (m_run + __log2f(lt)) * kLn2;
+          }
         }
       }
     }
@@ -556,7 +587,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
