@@ -15,14 +15,14 @@
 //   * fwd_window_kernel  (N <= 128): persistent CTAs; each 128-row tile packs
 //     128/NP whole windows (NP = 64 or 128 rows per window).  One S tile per
 //     tile, single-pass softmax, block-diagonal P (off-window blocks stay 0).
-//   * fwd_long_kernel    (N > 128): one CTA per (head, 128-query tile); loops
-//     over 128-key tiles with an online softmax (lazy rescale of O in TMEM);
-//     two softmax warpgroups split each score tile by key columns.
+//   * fwd_long_kernel    (N > 128): one CTA per (head, two 128-query tiles);
+//     loops over 128-key tiles with an online softmax (lazy rescale of O in
+//     TMEM); one softmax warpgroup per query tile, running out of phase.
 //
 // Window kernel warp roles (192 threads): warps 0-3 softmax + epilogue (thread
 // = row = TMEM lane), warp 4 TMA producer, warp 5 U' scaling + MMA issue +
-// TMEM allocation.  The long kernel uses 320 threads: warps 0-7 softmax (two
-// warpgroups), warp 8 TMA, warp 9 MMA.  Operands are staged by TMA with the swizzle that matches
+// TMEM allocation.  The long kernel uses 320 threads: warps 0-7 softmax (one
+// warpgroup per query tile), warp 8 TMA, warp 9 MMA.  Operands are staged by TMA with the swizzle that matches
 // their row width; P is written by the softmax threads into a 128-byte
 // swizzled K-major tile.
 #pragma once
@@ -363,31 +363,27 @@ struct LongCfg {
   static constexpr int UB = kTile * RP * 2;
   static constexpr int STAGE = 2 * QB + UB;  // K, V, W
   static constexpr int PB = kTile * kTile * 2;
-  static constexpr int NS_FIT = (200 * 1024 - 2 * PB - QB - UB) / STAGE;
+  // Two query tiles per CTA: Q0 U0 Q1 U1, KV stages, P0 P1.
+  static constexpr int OFF_Q = 0;            // Q tile t at OFF_Q + t * (QB + UB), U right after
+  static constexpr int OFF_STAGE = 2 * (QB + UB);
+  static constexpr int NS_FIT = (226 * 1024 - OFF_STAGE - 2 * PB) / STAGE;
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_U = QB;
-  static constexpr int OFF_STAGE = QB + UB;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_X = OFF_P + 2 * PB;     // row-statistics exchange, fp32
-  static constexpr int X_BYTES = (2 * 2 + 2) * kTile * 4;  // max[2 tiles][2 wg], sum[2 wg]
-  static constexpr int OFF_BAR = OFF_X + X_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * PB;
   // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
-  // mx_bar[2] end_bar
-  static constexpr int NBAR = 2 * NS + 13;
+  static constexpr int NBAR = 2 * NS + 10;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr int OC = D / 2;  // O columns each softmax warpgroup owns
   static_assert(NS >= 2, "not enough shared memory for two KV stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
 };
 
-constexpr int kLongThreads = 320;  // warps 0-7 softmax (two warpgroups), 8 TMA, 9 MMA
+constexpr int kLongThreads = 320;  // warps 0-3 softmax of query tile 0, 4-7 of tile 1, 8 TMA, 9 MMA
 
-// Long regime: one CTA per (head, 128-query tile), looping over 128-key tiles.
-// The two softmax warpgroups split each score tile by key columns (64 each):
-// they exchange per-row partial maxima through shared memory (bounded
-// barrier), keep partial row sums, and each owns half of O's columns for the
-// lazy rescale and the epilogue.
+// Long regime: one CTA per (head, pair of 128-query tiles), looping over
+// 128-key tiles.  Each query tile has its own softmax warpgroup, S buffer
+// (TMEM columns t*128), O accumulator (TMEM 256 + t*D) and P buffer; the two
+// warpgroups run out of phase, so one's exponentials overlap the other's
+// loads, maxima and waits, and each K/V tile serves 256 query rows.
 template <int D, int RP>
 __global__ void __launch_bounds__(kLongThreads, 1)
     fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
@@ -395,7 +391,6 @@ __global__ void __launch_bounds__(kLongThreads, 1)
                     const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
   using C = LongCfg<D, RP>;
   constexpr int NS = C::NS;
-  constexpr int OC = C::OC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   const uint32_t sb = smem_u32(smem);
@@ -403,15 +398,13 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   const uint32_t q_full = bar0;
   auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto kv_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (1 + 2 * NS + b); };
-  auto s_empty = [&](int b) { return bar0 + 8u * (3 + 2 * NS + b); };
-  auto p_full = [&](int b) { return bar0 + 8u * (5 + 2 * NS + b); };
-  auto pv_done = [&](int b) { return bar0 + 8u * (7 + 2 * NS + b); };
+  auto s_full = [&](int t) { return bar0 + 8u * (1 + 2 * NS + t); };
+  auto s_empty = [&](int t) { return bar0 + 8u * (3 + 2 * NS + t); };
+  auto p_full = [&](int t) { return bar0 + 8u * (5 + 2 * NS + t); };
+  auto pv_done = [&](int t) { return bar0 + 8u * (7 + 2 * NS + t); };
   const uint32_t drain_bar = bar0 + 8u * (9 + 2 * NS);
-  auto mx_bar = [&](int b) { return bar0 + 8u * (10 + 2 * NS + b); };
-  const uint32_t end_bar = bar0 + 8u * (12 + 2 * NS);
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_X);              // [2][2][128]
-  float* xsum = reinterpret_cast<float*>(smem + C::OFF_X + 4 * kTile * 4);  // [2][128]
+  auto q_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB); };
+  auto u_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB) + C::QB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -419,7 +412,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   const int lane = static_cast<int>(lane_id());
   const int N = args.N;
   const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * kTile;
+  const int q0 = blockIdx.x * 2 * kTile;
   const int nkv = (N + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
@@ -429,15 +422,13 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full(b), 1);
-      mbar_init(s_empty(b), 256);
-      mbar_init(p_full(b), 256);
-      mbar_init(pv_done(b), 1);
-      mbar_init(mx_bar(b), 256);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(s_empty(t), 128);
+      mbar_init(p_full(t), 128);
+      mbar_init(pv_done(t), 1);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(end_bar, 256);
     fence_mbar_init();
   }
   if (warp == 8 && lane == 0) {
@@ -461,9 +452,11 @@ __global__ void __launch_bounds__(kLongThreads, 1)
 
   if (warp == 8) {
     if (lane == 0) {
-      mbar_expect_tx(q_full, C::QB + C::UB);
-      tma_load_3d(sb + C::OFF_Q, &mQ, q_full, 0, q0, bh);
-      if constexpr (RP > 0) tma_load_3d(sb + C::OFF_U, &mU, q_full, 0, q0, bh);
+      mbar_expect_tx(q_full, 2 * (C::QB + C::UB));
+      for (int t = 0; t < 2; ++t) {
+        tma_load_3d(q_addr(t), &mQ, q_full, 0, q0 + t * kTile, bh);
+        if constexpr (RP > 0) tma_load_3d(u_addr(t), &mU, q_full, 0, q0 + t * kTile, bh);
+      }
       int j = 0;
       for (; j < nkv; ++j) {
         const int s = j % NS;
@@ -482,62 +475,64 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     bool ok = wait_warp(q_full, 0, g, 12);
     if (ok) {
       if constexpr (RP > 0) {
-        scale_tile_bf16(sb + C::OFF_U, C::UB, args.inv_scale);
+        scale_tile_bf16(u_addr(0), C::UB, args.inv_scale);
+        scale_tile_bf16(u_addr(1), C::UB, args.inv_scale);
         fence_async_smem();
       }
       __syncwarp();
     }
-    auto do_s = [&](int j) -> bool {
-      const int s = j % NS, b = j & 1;
-      if (!wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
-      if (j >= 2 && !wait_warp(s_empty(b), ((j >> 1) + 1) & 1, g, 14)) return false;
+    // S_t = Q_t K_j^T + U'_t W_j^T into query tile t's S columns; the previous
+    // scores of tile t must have been loaded by its warpgroup (s_empty).
+    auto do_s = [&](int j, int t) -> bool {
+      const int s = j % NS;
+      if (t == 0 && !wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
+      if (j >= 1 && !wait_warp(s_empty(t), (j - 1) & 1, g, 14)) return false;
       tc_fence_after();
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-      issue_scores<D, RP>(tmem + b * 128, sb + C::OFF_Q, st, sb + C::OFF_U, st + 2 * C::QB);
-      umma_commit(s_full(b));
+      issue_scores<D, RP>(tmem + t * 128, q_addr(t), st, u_addr(t), st + 2 * C::QB);
+      umma_commit(s_full(t));
       return true;
     };
-    auto do_pv = [&](int j) -> bool {
-      const int s = j % NS, b = j & 1;
-      if (!wait_warp(p_full(b), (j >> 1) & 1, g, 15)) return false;
+    auto do_pv = [&](int j, int t) -> bool {
+      const int s = j % NS;
+      if (!wait_warp(p_full(t), j & 1, g, 15)) return false;
       tc_fence_after();
-      issue_pv<D>(tmem + 256, sb + C::OFF_P + b * C::PB, sb + C::OFF_STAGE + s * C::STAGE + C::QB,
-                  j > 0);
-      umma_commit(kv_empty(s));
-      umma_commit(pv_done(b));
+      issue_pv<D>(tmem + 256 + t * D, sb + C::OFF_P + t * C::PB,
+                  sb + C::OFF_STAGE + s * C::STAGE + C::QB, j > 0);
+      umma_commit(pv_done(t));
+      if (t == 1) umma_commit(kv_empty(s));
       return true;
     };
-    if (ok) ok = do_s(0);
+    if (ok) ok = do_s(0, 0) && do_s(0, 1);
     for (int j = 0; ok && j < nkv; ++j) {
-      if (j + 1 < nkv && !do_s(j + 1)) break;
-      if (!do_pv(j)) break;
+      if (j + 1 < nkv && !do_s(j + 1, 0)) break;
+      if (!do_pv(j, 0)) break;
+      if (j + 1 < nkv && !do_s(j + 1, 1)) break;
+      if (!do_pv(j, 1)) break;
     }
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
   } else {
-    const int wg = warp >> 2;            // key columns wg*64 .. wg*64+63
-    const int row = threadIdx.x & 127;   // TMEM lane == query row
+    const int t = warp >> 2;             // query tile of this warpgroup
+    const int row = threadIdx.x & 127;   // TMEM lane == query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_tm = tmem + lane_base + t * 128;
+    const uint32_t o_tm = tmem + lane_base + 256 + t * D;
+    const uint32_t pbuf = sb + C::OFF_P + t * C::PB;
     const float sl2 = args.scale_log2;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      if (!wait_warp(s_full(b), (j >> 1) & 1, g, 16)) { ok = false; break; }
+      if (!wait_warp(s_full(t), j & 1, g, 16)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld64(tmem + lane_base + b * 128 + wg * 64, sv);
+      uint32_t sv[128];
+      tmem_ld_cols<128>(s_tm, sv);
       tc_fence_before();
-      mbar_arrive(s_empty(b));
-      const int kvalid = N - j * kTile - wg * 64;  // valid keys in this half (may be <= 0)
-      if (kvalid < 64) mask_tail<64>(sv, kvalid);
-      // Row maximum over the full 128 keys: exchange the two halves' maxima.
-      xmax[(b * 2 + wg) * kTile + row] = row_max<64>(sv);
-      mbar_arrive(mx_bar(b));
-      if (!wait_warp(mx_bar(b), (j >> 1) & 1, g, 20)) { ok = false; break; }
-      const float mx = fmaxf(xmax[(b * 2 + wg) * kTile + row], xmax[(b * 2 + (wg ^ 1)) * kTile + row]);
-      const float m_new = fmaxf(m_run, mx * sl2);
+      mbar_arrive(s_empty(t));
+      const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
+      if (kvalid < kTile) mask_tail<128>(sv, kvalid);
+      const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);
       // Lazy rescale: keep the running max unless it grew by more than 2^8.
       const bool need = m_new > m_run + 8.0f;
       float alpha = 1.f;
@@ -547,39 +542,31 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         m_run = m_new;
       }
       const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
-      if (j >= 2 && !wait_warp(pv_done(b), ((j >> 1) + 1) & 1, g, 17)) { ok = false; break; }
-      l += exp_row_to_smem<64>(sv, sl2, m_run, sb + C::OFF_P + b * C::PB, row, wg * 64);
+      // The single P buffer of this tile and O: PV_{j-1} must have finished.
+      if (j >= 1 && !wait_warp(pv_done(t), (j - 1) & 1, g, 17)) { ok = false; break; }
+      l += exp_row_to_smem<128>(sv, sl2, m_run, pbuf, row, 0);
       if (fix_o) {
-        // O holds the sum through tile j-1 at the old running max: wait for that
-        // PV to land, then rescale this thread's half row in place.
-        if (!wait_warp(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, g, 18)) { ok = false; break; }
         tc_fence_after();
-        uint32_t ov[OC];
-        tmem_ld_cols<OC>(tmem + lane_base + 256 + wg * OC, ov);
+        uint32_t ov[D];
+        tmem_ld_cols<D>(o_tm, ov);
 #pragma unroll
-        for (int c = 0; c < OC; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-        tmem_st_cols<OC>(tmem + lane_base + 256 + wg * OC, ov);
+        for (int c = 0; c < D; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+        tmem_st_cols<D>(o_tm, ov);
       }
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full(b));
+      mbar_arrive(p_full(t));
     }
-    if (ok) {
-      const int jl = nkv - 1;
-      if (wait_warp(pv_done(jl & 1), (jl >> 1) & 1, g, 19)) {
-        xsum[wg * kTile + row] = l;
-        mbar_arrive(end_bar);
-        if (wait_warp(end_bar, 0, g, 21)) {
-          const float lt = xsum[row] + xsum[kTile + row];
-          tc_fence_after();
-          uint32_t ov[OC];
-          tmem_ld_cols<OC>(tmem + lane_base + 256 + wg * OC, ov);
-          const int q = q0 + row;
-          if (q < N) {
-            const size_t r = static_cast<size_t>(bh) * N + q;
-            store_o_row<OC>(args.o + r * D + wg * OC, ov, 1.0f / lt);
-            if (wg == 0) args.lse[r] = (m_run + __log2f(lt)) * kLn2;
-          }
+    if (ok && nkv > 0) {
+      if (wait_warp(pv_done(t), (nkv - 1) & 1, g, 19)) {
+        tc_fence_after();
+        uint32_t ov[D];
+        tmem_ld_cols<D>(o_tm, ov);
+        const int q = q0 + t * kTile + row;
+        if (q < N) {
+          const size_t r = static_cast<size_t>(bh) * N + q;
+          store_o_row<D>(args.o + r * D, ov, 1.0f / l);
+          args.lse[r] = (m_run + __log2f(l)) * kLn2;
         }
       }
     }

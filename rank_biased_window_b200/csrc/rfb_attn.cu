@@ -269,7 +269,7 @@ int launch_long(const Maps& m, const FwdArgs& a, cudaStream_t st) {
   using C = LongCfg<D, RP>;
   static std::atomic<uint64_t> done{0};
   if (int rc = ensure_smem(fwd_long_kernel<D, RP>, C::SMEM, done)) return rc;
-  const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
+  const dim3 grid((a.N + 2 * kTile - 1) / (2 * kTile), a.BH);
   LaunchTimer timer(kIdFwd, st);
   fwd_long_kernel<D, RP><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
