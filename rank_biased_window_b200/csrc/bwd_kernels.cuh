@@ -136,13 +136,19 @@ template <int D, int RP>
 struct BwdCfg {
   static constexpr int QB = kTile * D * 2;
   static constexpr int UB = kTile * RP * 2;
+  // With d = 64, U' is staged 64 columns wide (128-byte rows, zero padded
+  // beyond r) so that [Q | U'] forms one MN-major B operand of two 128-byte
+  // swizzle atoms and dK | dW come from a single MMA chain (N = d + r_pad).
+  static constexpr bool MERGE_KW = (D == 64) && (RP > 0);
+  static constexpr int UW = MERGE_KW ? 64 : RP;     // staged width of U'
+  static constexpr int UQB = kTile * UW * 2;        // bytes of the staged U' tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = QB;
   static constexpr int OFF_W = 2 * QB;
   static constexpr int KVB = 2 * QB + UB;
   // stage: Q, dO, U', -LSE log2(e) [128], -D [128]
-  static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UB, S_DV = S_L2 + 512;
-  static constexpr int STAGE = 2 * QB + UB + 1024;
+  static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UQB, S_DV = S_L2 + 512;
+  static constexpr int STAGE = 2 * QB + UQB + 1024;
   static constexpr int PB = kTile * kTile * 2;  // one dS tile (bf16)
   static constexpr int STG = kTile * 32 * 4;    // one 128 x 32 fp32 staging buffer
   static constexpr int NCH = (D + RP + 31) / 32;  // dQ | dU chunks of 32 columns
@@ -155,12 +161,15 @@ struct BwdCfg {
   static constexpr bool DEFER = (256 + 2 * D + RP + NCH * 32) <= 512;
   static constexpr int T_DQ = DEFER ? 256 + 2 * D + RP : 0;
   static constexpr int NDS = DEFER ? 2 : 1;
-  static constexpr int NS_FIT = (226 * 1024 - KVB - NDS * PB - 2 * STG) / STAGE;
+  // Staging buffers: with DEFER each warpgroup's first chunk is staged in its
+  // block of the dS buffer, so only warpgroup 0's further chunks need one.
+  static constexpr int NSTG = DEFER ? 1 : 2;
+  static constexpr int NS_FIT = (226 * 1024 - KVB - NDS * PB - NSTG * STG) / STAGE;
   static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
   static constexpr int OFF_STAGE = KVB;
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_STG = OFF_DS + NDS * PB;
-  static constexpr int OFF_BAR = OFF_STG + 2 * STG;
+  static constexpr int OFF_BAR = OFF_STG + NSTG * STG;
   // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain wg_sync[2] a_done
   static constexpr int NBAR = 2 * NS + 9;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
@@ -293,7 +302,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < RP / 16; ++kk)
         umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_W + kk * 32, RP * 2),
-                  desc_kmajor(st + C::S_U + kk * 32, RP * 2), idS, 1u);
+                  desc_kmajor(st + C::S_U + kk * 32, C::UW * 2), idS, 1u);
       umma_commit(sdp_full);
       return true;
     };
@@ -309,12 +318,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t aoff = (kk >> 2) * 64 + (kk & 3) * 8;
         umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + aoff,
                      desc_mnmajor(st + C::S_DO + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
-        umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
-                     desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
-        if constexpr (RP > 0)
-          umma_bf16_ts(tmem + C::T_DW, tmem + C::T_DP + aoff,
-                       desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
-                       acc);
+        if constexpr (C::MERGE_KW) {
+          // [dK | dW] += dS^T [Q | U']: one B operand, atoms Q (64 cols) and U'
+          // (C::S_U - C::S_Q bytes further), N = D + RP.
+          constexpr uint32_t idKW = idesc_bf16_f32(128, D + RP, false, true);
+          umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
+                       desc_mnmajor(st + C::S_Q + kk * 16 * 128, 128, C::S_U - C::S_Q), idKW, acc);
+        } else {
+          umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
+                       desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+          if constexpr (RP > 0)
+            umma_bf16_ts(tmem + C::T_DW, tmem + C::T_DP + aoff,
+                         desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+                         acc);
+        }
       }
       umma_commit(a_done);
       umma_commit(q_empty(i % NS));  // Q, dO, U' of this tile are no longer read
@@ -369,7 +386,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool key_ok = (k0 + row) < N;
     const uint64_t sl2x2 = f2_pack(args.scale_log2, args.scale_log2);
     const bool leader = (threadIdx.x & 127) == 0;  // issues this warpgroup's reductions
-    const uint32_t stg = sb + C::OFF_STG + wg * C::STG;
+    const uint32_t stg = sb + C::OFF_STG + (C::NSTG == 2 ? wg : 0) * C::STG;
     const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
     uint32_t wg_phase = 0;
     // Bounded barrier over this warpgroup's 128 threads.

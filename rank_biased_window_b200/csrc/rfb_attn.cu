@@ -442,7 +442,9 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   if (!rc) rc = encode_3d(&m.g, dout, d, N, BH, d, kTile, 1);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   // The backward stages U' = U / s once (bwd_pre) and tiles that copy.
-  if (!rc && r > 0) rc = encode_3d(&m.u, ws + L.uprime, r, N, BH, rp, kTile, 1);
+  // With d = 64 the U' tile is staged 64 columns wide (zero padded), so it can
+  // sit beside Q as one MMA operand.
+  if (!rc && r > 0) rc = encode_3d(&m.u, ws + L.uprime, r, N, BH, d == 64 ? 64 : rp, kTile, 1);
   if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, kTile, 1);
   if (!rc) rc = encode_acc_3d(&m.acc, ws + L.acc, d + r, N, BH);
   if (rc) return rc;
