@@ -377,13 +377,15 @@ struct LongCfg {
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
 };
 
-constexpr int kLongThreads = 320;  // warps 0-3 softmax of query tile 0, 4-7 of tile 1, 8 TMA, 9 MMA
+// warps 0-3 softmax of query tile 0, 4-7 of tile 1, 8 TMA, 9 / 10 MMA issue for tile 0 / 1
+constexpr int kLongThreads = 352;
 
 // Long regime: one CTA per (head, pair of 128-query tiles), looping over
-// 128-key tiles.  Each query tile has its own softmax warpgroup, S buffer
-// (TMEM columns t*128), O accumulator (TMEM 256 + t*D) and P buffer; the two
-// warpgroups run out of phase, so one's exponentials overlap the other's
-// loads, maxima and waits, and each K/V tile serves 256 query rows.
+// 128-key tiles.  Each query tile has its own softmax warpgroup, MMA-issuing
+// warp, S buffer (TMEM columns t*128), O accumulator (TMEM 256 + t*D) and P
+// buffer; the two pipelines run independently and out of phase, so one's
+// exponentials overlap the other's loads, maxima and waits, and each K/V tile
+// serves 256 query rows.
 template <int D, int RP>
 __global__ void __launch_bounds__(kLongThreads, 1)
     fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
@@ -420,7 +422,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(kv_empty(s), 2);  // one arrival per query tile's MMA warp
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full(t), 1);
@@ -428,7 +430,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_bar, 2);
     fence_mbar_init();
   }
   if (warp == 8 && lane == 0) {
@@ -471,21 +473,22 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       for (int i = (j > NS ? j - NS : 0); i < j; ++i)
         wait_drain(kv_full(i % NS), (i / NS) & 1, args.timeout_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp >= 9) {
+    // MMA issue for query tile t = warp - 9 (one converged warp each).
+    const int t = warp - 9;
     bool ok = wait_warp(q_full, 0, g, 12);
     if (ok) {
       if constexpr (RP > 0) {
-        scale_tile_bf16(u_addr(0), C::UB, args.inv_scale);
-        scale_tile_bf16(u_addr(1), C::UB, args.inv_scale);
+        scale_tile_bf16(u_addr(t), C::UB, args.inv_scale);
         fence_async_smem();
       }
       __syncwarp();
     }
-    // S_t = Q_t K_j^T + U'_t W_j^T into query tile t's S columns; the previous
-    // scores of tile t must have been loaded by its warpgroup (s_empty).
-    auto do_s = [&](int j, int t) -> bool {
+    // S_t = Q_t K_j^T + U'_t W_j^T into tile t's S columns, once its warpgroup
+    // has loaded the previous scores (s_empty).
+    auto do_s = [&](int j) -> bool {
       const int s = j % NS;
-      if (t == 0 && !wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
+      if (!wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
       if (j >= 1 && !wait_warp(s_empty(t), (j - 1) & 1, g, 14)) return false;
       tc_fence_after();
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
@@ -493,22 +496,20 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       umma_commit(s_full(t));
       return true;
     };
-    auto do_pv = [&](int j, int t) -> bool {
+    auto do_pv = [&](int j) -> bool {
       const int s = j % NS;
       if (!wait_warp(p_full(t), j & 1, g, 15)) return false;
       tc_fence_after();
       issue_pv<D>(tmem + 256 + t * D, sb + C::OFF_P + t * C::PB,
                   sb + C::OFF_STAGE + s * C::STAGE + C::QB, j > 0);
       umma_commit(pv_done(t));
-      if (t == 1) umma_commit(kv_empty(s));
+      umma_commit(kv_empty(s));
       return true;
     };
-    if (ok) ok = do_s(0, 0) && do_s(0, 1);
+    if (ok) ok = do_s(0);
     for (int j = 0; ok && j < nkv; ++j) {
-      if (j + 1 < nkv && !do_s(j + 1, 0)) break;
-      if (!do_pv(j, 0)) break;
-      if (j + 1 < nkv && !do_s(j + 1, 1)) break;
-      if (!do_pv(j, 1)) break;
+      if (j + 1 < nkv && !do_s(j + 1)) break;
+      if (!do_pv(j)) break;
     }
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0, args.timeout_ns);
