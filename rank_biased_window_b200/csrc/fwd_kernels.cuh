@@ -19,9 +19,9 @@
 //     loops over 128-key tiles with an online softmax (lazy rescale of O in
 //     TMEM); one softmax warpgroup per query tile, running out of phase.
 //
-// Window kernel warp roles (192 threads): warps 0-3 softmax + epilogue (thread
-// = row = TMEM lane), warp 4 TMA producer, warp 5 U' scaling + MMA issue +
-// TMEM allocation.  The long kernel uses 320 threads: warps 0-7 softmax (one
+// Window kernel warp roles (320 threads): warps 0-3 and 4-7 softmax + epilogue
+// of even and odd tiles (thread = row = TMEM lane), warp 8 TMA producer, warp 9
+// U' scaling + MMA issue + TMEM allocation.  The long kernel uses 320 threads: warps 0-7 softmax (one
 // warpgroup per query tile), warp 8 TMA, warp 9 MMA.  Operands are staged by TMA with the swizzle that matches
 // their row width; P is written by the softmax threads into a 128-byte
 // swizzled K-major tile.
@@ -178,8 +178,10 @@ struct WinCfg {
   static_assert(QB % 1024 == 0 && UB % 1024 == 0, "tile alignment");
 };
 
+constexpr int kWinThreads = 320;  // warps 0-3 / 4-7 softmax of even / odd tiles, 8 TMA, 9 MMA
+
 template <int D, int RP, int NP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kWinThreads, 1)
     fwd_window_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                       const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
                       const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(drain_bar, 1);
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch(&mQ);
     tma_prefetch(&mK);
     tma_prefetch(&mV);
@@ -227,14 +229,14 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch(&mW);
     }
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp < 4) {
+  if (warp < 8) {
     // P buffers start at zero: with NP = 64 each row only ever writes its own
     // window's 64-key block, so the other block stays zero (block-diagonal P).
-    for (int off = threadIdx.x * 16; off < 2 * C::PB; off += 128 * 16)
+    for (int off = threadIdx.x * 16; off < 2 * C::PB; off += 256 * 16)
       st_shared_v4(sb + C::OFF_P + off, 0u, 0u, 0u, 0u);
     fence_async_smem();
   }
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int it = 0;
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = (it > NS ? it - NS : 0); j < it; ++j)
         wait_drain(in_full(j % NS), (j / NS) & 1, args.timeout_ns);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------- U' scaling + MMA issue
     bool ok = true;
     auto do_pv = [&](int j) -> bool {
@@ -301,16 +303,30 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------- softmax + epilogue
-    const int row = threadIdx.x;  // TMEM lane == tile row
-    const int wl = row / NP;      // window inside the tile
-    const int n = row % NP;       // token inside the window
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // Warpgroup a (= warp / 4) takes the tiles with it % 2 == a, i.e. exactly
+    // the tiles that use S, O and P buffer a, so the two warpgroups work on
+    // consecutive tiles at the same time.
+    const int a = warp >> 2;
+    const int row = threadIdx.x & 127;  // TMEM lane == tile row
+    const int wl = row / NP;            // window inside the tile
+    const int n = row % NP;             // token inside the window
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int N = args.N;
     const float sl2 = args.scale_log2;
-
-    auto epilogue = [&](int j, int t, float m, float l) -> bool {
-      const int a = j & 1;
-      if (!wait_warp(o_full(a), (j >> 1) & 1, g, 6)) return false;
+    int it = a;
+    for (int t = blockIdx.x + a * gridDim.x; t < num_tiles; t += 2 * gridDim.x, it += 2) {
+      if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) break;
+      tc_fence_after();
+      uint32_t sv[NP];
+      tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
+      if (N < NP) mask_tail<NP>(sv, N);
+      const float m = row_max<NP>(sv) * sl2;
+      const float l = exp_row_to_smem<NP>(sv, sl2, m, sb + C::OFF_P + a * C::PB, row, wl * NP);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full(a));
+      // Epilogue of this tile once its PV has landed.
+      if (!wait_warp(o_full(a), (it >> 1) & 1, g, 6)) break;
       tc_fence_after();
       uint32_t ov[D];
       tmem_ld_cols<D>(tmem + lane_base + 256 + a * D, ov);
@@ -322,35 +338,12 @@ __global__ void __launch_bounds__(192, 1)
         store_o_row<D>(args.o + r * D, ov, 1.0f / l);
         args.lse[r] = (m + __log2f(l)) * kLn2;
       }
-      return true;
-    };
-
-    bool ok = true;
-    int it = 0, t_prev = 0;
-    float m_prev = 0.f, l_prev = 1.f;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int a = it & 1;
-      if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[NP];
-      tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
-      if (N < NP) mask_tail<NP>(sv, N);
-      const float m = row_max<NP>(sv) * sl2;
-      const float l = exp_row_to_smem<NP>(sv, sl2, m, sb + C::OFF_P + a * C::PB, row, wl * NP);
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full(a));
-      if (it > 0 && !epilogue(it - 1, t_prev, m_prev, l_prev)) { ok = false; break; }
-      m_prev = m;
-      l_prev = l;
-      t_prev = t;
     }
-    if (ok && it > 0) epilogue(it - 1, t_prev, m_prev, l_prev);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

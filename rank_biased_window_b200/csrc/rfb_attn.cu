@@ -260,7 +260,7 @@ int launch_window(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   const int tiles = (a.BH + C::NW - 1) / C::NW;
   const int grid = tiles < sms ? tiles : sms;
   LaunchTimer timer(kIdFwd, st);
-  fwd_window_kernel<D, RP, NP><<<grid, 192, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  fwd_window_kernel<D, RP, NP><<<grid, kWinThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
 }
 
