@@ -181,6 +181,13 @@ RFB_API int rfb_profile_enable(int on);
 RFB_API int rfb_profile_read(float* ms, int* launches);
 RFB_API const char* rfb_profile_kernel_name(int id);
 
+/*
+ * Self test of the software exp2 that the kernels use for part of the softmax
+ * exponentials: y[i] = 2^x[i] for i < n, computed on the device by that code
+ * path (x, y device pointers, fp32).  Inputs below -125 return about 2^-125.
+ */
+RFB_API int rfb_selftest_soft_exp2(const float* x, float* y, int n, void* stream);
+
 /* Library version string. */
 RFB_API const char* rfb_version(void);
 

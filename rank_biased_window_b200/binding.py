@@ -37,6 +37,7 @@ SIGNATURES = {
     "rfb_last_device_error": (_i, []),
     "rfb_last_cuda_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
     "rfb_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
+    "rfb_selftest_soft_exp2": (_i, [_vp, _vp, _i, _vp]),
     "rfb_profile_enable": (_i, [_i]),
     "rfb_profile_read": (_i, [_fp, ctypes.POINTER(ctypes.c_int)]),
     "rfb_profile_kernel_name": (ctypes.c_char_p, [_i]),
@@ -223,6 +224,18 @@ def selftest_wait_timeout(timeout_us: int = 1000, stream=None, device=None):
     with torch.cuda.device(dev):
         rc = load_library().rfb_selftest_wait_timeout(int(timeout_us), _stream_ptr(stream, dev))
     _check(rc, "rfb_selftest_wait_timeout")
+
+
+def selftest_soft_exp2(x):
+    """2^x through the kernels' software exp2 (device fp32 tensor in, out)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        rc = load_library().rfb_selftest_soft_exp2(_ptr(x), _ptr(y), x.numel(),
+                                                    _stream_ptr(None, x.device))
+    _check(rc, "rfb_selftest_soft_exp2")
+    return y
 
 
 def profile_enable(on: bool = True):

@@ -111,9 +111,12 @@ __device__ __forceinline__ float row_max(const uint32_t (&sv)[NC]) {
 // p_j = 2^(s_j * sl2 - m) written as bf16 into the 128-byte-swizzled K-major P
 // tile (row `row`, columns col0..col0+NC); returns sum_j p_j (fp32, 8 partial
 // sums).  Masked scores are -inf and give p = 0.
-template <int NC>
+// SOFT_PAIRS of every 8 exponentials use the software exp2 (FMA / integer
+// pipes) instead of the MUFU unit.
+template <int NC, int SOFT_PAIRS = 0>
 __device__ __forceinline__ float exp_row_to_smem(const uint32_t (&sv)[NC], float sl2, float m,
                                                  uint32_t pbuf, int row, int col0) {
+  constexpr int HW = 8 - 2 * SOFT_PAIRS;  // exponentials per 8 on the MUFU unit
   float l[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) l[e] = 0.f;
@@ -121,10 +124,13 @@ __device__ __forceinline__ float exp_row_to_smem(const uint32_t (&sv)[NC], float
   for (int c = 0; c < NC; c += 8) {
     float p[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      p[e] = fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
-      l[e] += p[e];
-    }
+    for (int e = 0; e < HW; ++e) p[e] = fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
+#pragma unroll
+    for (int e = HW; e < 8; e += 2)
+      soft_exp2_x2(fmaf(__uint_as_float(sv[c + e]), sl2, -m),
+                   fmaf(__uint_as_float(sv[c + e + 1]), sl2, -m), p[e], p[e + 1]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) l[e] += p[e];
     st_shared_v4(pbuf + sw128_offset(row, col0 + c, 128), pack_bf16x2(p[0], p[1]),
                  pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
   }
@@ -372,6 +378,9 @@ struct LongCfg {
 
 // warps 0-3 softmax of query tile 0, 4-7 of tile 1, 8 TMA, 9 / 10 MMA issue for tile 0 / 1
 constexpr int kLongThreads = 352;
+// Pairs of every 8 softmax exponentials computed in software in the long
+// forward (the MUFU unit is its limit; 1 pair = 25 %).
+constexpr int kLongSoftPairs = 1;
 
 // Long regime: one CTA per (head, pair of 128-query tiles), looping over
 // 128-key tiles.  Each query tile has its own softmax warpgroup, MMA-issuing
@@ -538,7 +547,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
       // The single P buffer of this tile and O: PV_{j-1} must have finished.
       if (j >= 1 && !wait_warp(pv_done(t), (j - 1) & 1, g, 17)) { ok = false; break; }
-      l += exp_row_to_smem<128>(sv, sl2, m_run, pbuf, row, 0);
+      l += exp_row_to_smem<128, kLongSoftPairs>(sv, sl2, m_run, pbuf, row, 0);
       if (fix_o) {
         tc_fence_after();
         uint32_t ov[D];

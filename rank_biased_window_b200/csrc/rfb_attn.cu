@@ -43,6 +43,16 @@ __global__ void selftest_wait_kernel(int* err, uint64_t timeout_ns) {
 // address comes from cudaGetSymbolAddress (noalloc_scratch below).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RFB_NOALLOC_SCRATCH_BYTES];
 
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    soft_exp2_x2(x[i], x[i + 1], y[i], y[i + 1]);
+  } else if (i < n) {
+    float dummy;
+    soft_exp2_x2(x[i], 0.f, y[i], dummy);
+  }
+}
+
 namespace {
 
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
@@ -525,6 +535,16 @@ int rfb_last_device_error(void) {
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return -RFB_ERR_CUDA;
   return v;
+}
+
+int rfb_selftest_soft_exp2(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return RFB_ERR_INVALID_ARG;
+  if (n == 0) return RFB_OK;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
 }
 
 int rfb_selftest_wait_timeout(unsigned int timeout_us, void* stream) {

@@ -305,6 +305,38 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Software 2^x for a pair of inputs on the FMA and integer pipes (relieves the
+// MUFU unit, which is the limit of the softmax).  x = n + f with n = round(x)
+// obtained by adding 1.5 * 2^23 (Cody and Waite's additive range reduction,
+// base 2) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with minimum
+// relative error (coefficients from gen_exp2_poly.py: max relative error
+// 7.6e-5, far below bf16's 2^-9 rounding of P); 2^n added to the exponent
+// field.  Inputs are clamped at -125 (results below 2^-125 are not needed by
+// the softmax: they are masked or negligible).  x <= 126 is assumed.
+__device__ __forceinline__ void soft_exp2_x2(float a, float b, float& ra, float& rb) {
+  constexpr float kC0 = 0.9999275803565979f, kC1 = 0.6932516098022461f;
+  constexpr float kC2 = 0.24261537194252014f, kC3 = 0.05522261559963226f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x2 = f2_pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+  const uint64_t r2 = f2_pack(kRound, kRound);
+  const uint64_t t2 = f2_add(x2, r2);
+  const uint64_t fr = f2_sub(x2, f2_sub(t2, r2));
+  uint64_t p = f2_fma(f2_pack(kC3, kC3), fr, f2_pack(kC2, kC2));
+  p = f2_fma(p, fr, f2_pack(kC1, kC1));
+  p = f2_fma(p, fr, f2_pack(kC0, kC0));
+  const float2 pf = f2_unpack(p), tf = f2_unpack(t2);
+  // t's low mantissa bits hold n (two's complement); shifting them into the
+  // exponent field adds n to p's exponent.
+  ra = __uint_as_float(__float_as_uint(pf.x) + (__float_as_uint(tf.x) << 23));
+  rb = __uint_as_float(__float_as_uint(pf.y) + (__float_as_uint(tf.y) << 23));
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),

@@ -134,3 +134,17 @@ def test_call_from_another_thread(rfb_lib, oracle_mod, cuda_dev):
     ref = oracle_mod.bwd(f["q"], f["k"], f["v"], f["u"], f["w"], f["dout"], 0.25)
     for name, got, want in zip(("dQ", "dK", "dV", "dU", "dW"), out["grads"], ref):
         assert_close(name, got, want)
+
+
+def test_software_exp2_accuracy(rfb_lib, cuda_dev):
+    """The software 2^x used for part of the softmax exponentials: relative
+    error against the exact value below 1e-4 on [-125, 10], and about 2^-125
+    for inputs below -125 (negligible against any row sum of the softmax)."""
+    x = torch.cat([torch.linspace(-125.0, 10.0, 200001), torch.tensor([-0.5, 0.0, 0.5, 1.0, -124.9])])
+    y = rfb_lib.binding.selftest_soft_exp2(x.to(cuda_dev)).cpu().double()
+    exact = torch.exp2(x.double())
+    rel = ((y - exact).abs() / exact).max().item()
+    assert rel < 1e-4, rel
+    low = rfb_lib.binding.selftest_soft_exp2(torch.tensor([-200.0, -1e30, float("-inf")],
+                                                          device=cuda_dev)).cpu().double()
+    assert torch.all((low / 2.0 ** -125 - 1).abs() < 1e-4)
