@@ -21,12 +21,15 @@
 //              them back into TMEM in place (bf16), dS^T also into swizzled
 //              shared memory; dV, dK, dW (+=) read their A operand from TMEM;
 //              the partial dQ|dU tile goes to TMEM columns of its own (when
-//              they fit), which
-//              the compute warps stage in 128-byte-swizzled shared memory and
-//              add into the fp32 accumulator with TMA bulk tensor reductions.
-//              The reduction of tile i runs after the softmax of tile i + 1,
-//              overlapping tile i + 1's MMAs; all MMAs are issued by one
-//              converged warp.
+//              they fit), which the compute warps stage in 128-byte-swizzled
+//              shared memory and add into the fp32 accumulator with TMA bulk
+//              tensor reductions.  The reduction of tile i runs after the
+//              softmax of tile i + 1, overlapping tile i + 1's MMAs.  Each
+//              query half (one warpgroup's 64 columns) has barriers of its
+//              own: S^T / dP^T of a half (N = 64 MMAs) and its dV / dK / dW
+//              MMAs are issued as soon as that half is ready, so one half's
+//              MMAs overlap the other half's softmax.  All MMAs are issued by
+//              one converged warp.
 //   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]).
 #pragma once
 #include "fwd_kernels.cuh"
@@ -136,16 +139,17 @@ template <int D, int RP>
 struct BwdCfg {
   static constexpr int QB = kTile * D * 2;
   static constexpr int UB = kTile * RP * 2;
-  // With d = 64, U' is staged 64 columns wide (128-byte rows, zero padded
-  // beyond r) so that [Q | U'] forms one MN-major B operand of two 128-byte
-  // swizzle atoms and dK | dW come from a single MMA chain (N = d + r_pad).
+  // With d = 64, U' and W are staged 64 columns wide (128-byte rows, zero
+  // padded beyond r) so that [Q | U'] and [K | W] each form one MN-major B
+  // operand of two 128-byte swizzle atoms: dK | dW and dQ | dU each come from a
+  // single MMA chain (N = d + r_pad).
   static constexpr bool MERGE_KW = (D == 64) && (RP > 0);
-  static constexpr int UW = MERGE_KW ? 64 : RP;     // staged width of U'
-  static constexpr int UQB = kTile * UW * 2;        // bytes of the staged U' tile
+  static constexpr int UW = MERGE_KW ? 64 : RP;     // staged width of U' and W
+  static constexpr int UQB = kTile * UW * 2;        // bytes of a staged U' or W tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = QB;
   static constexpr int OFF_W = 2 * QB;
-  static constexpr int KVB = 2 * QB + UB;
+  static constexpr int KVB = 2 * QB + UQB;
   // stage: Q, dO, U', -LSE log2(e) [128], -D [128]
   static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UQB, S_DV = S_L2 + 512;
   static constexpr int STAGE = 2 * QB + UQB + 1024;
@@ -164,15 +168,18 @@ struct BwdCfg {
   // Staging buffers: with DEFER each warpgroup's first chunk is staged in its
   // block of the dS buffer, so only warpgroup 0's further chunks need one.
   static constexpr int NSTG = DEFER ? 1 : 2;
-  static constexpr int NS_FIT = (226 * 1024 - KVB - NDS * PB - NSTG * STG) / STAGE;
+  // The dynamic shared memory is declared 1024-byte aligned (no slack); 256
+  // bytes are kept for the barriers.
+  static constexpr int NS_FIT = (232448 - 256 - KVB - NDS * PB - NSTG * STG) / STAGE;
   static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
   static constexpr int OFF_STAGE = KVB;
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_STG = OFF_DS + NDS * PB;
   static constexpr int OFF_BAR = OFF_STG + NSTG * STG;
-  // kv_full q_full[NS] q_empty[NS] sdp_full ds_full dq_full dq_free drain wg_sync[2] a_done
-  static constexpr int NBAR = 2 * NS + 9;
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  // kv_full q_full[NS] q_empty[NS] sdp_full[2] ds_full[2] dq_full dq_free drain wg_sync[2]
+  // a_done[2]
+  static constexpr int NBAR = 2 * NS + 12;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(NS >= 1, "shared memory budget");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
   static_assert(T_DW + RP <= 512 && NCH * 32 <= 128, "TMEM budget");
@@ -188,22 +195,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap mAcc, const BwdArgs args) {
   using C = BwdCfg<D, RP>;
   constexpr int NS = C::NS;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align_1024(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sb = smem_u32(smem);
+  if (sb & 1023u) {  // the swizzled operand tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(args.err, 0, kErrAlignment | (98 << 8));
+    return;
+  }
   const uint32_t bar0 = sb + C::OFF_BAR;
   const uint32_t kv_full = bar0;
   auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto q_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
-  const uint32_t sdp_full = bar0 + 8u * (1 + 2 * NS);
-  const uint32_t ds_full = bar0 + 8u * (2 + 2 * NS);
-  const uint32_t dq_full = bar0 + 8u * (3 + 2 * NS);
-  const uint32_t dq_free = bar0 + 8u * (4 + 2 * NS);
-  const uint32_t drain_bar = bar0 + 8u * (5 + 2 * NS);
+  // Query half h (columns 64h .. 64h + 63 of a tile, warpgroup h): its S^T and
+  // dP^T are in TMEM, its P^T / dS^T are written, its dV / dK / dW MMAs (which
+  // read P^T / dS^T from TMEM) are done.
+  auto sdp_full = [&](int h) { return bar0 + 8u * (1 + 2 * NS + h); };
+  auto ds_full = [&](int h) { return bar0 + 8u * (3 + 2 * NS + h); };
+  const uint32_t dq_full = bar0 + 8u * (5 + 2 * NS);
+  const uint32_t dq_free = bar0 + 8u * (6 + 2 * NS);
+  const uint32_t drain_bar = bar0 + 8u * (7 + 2 * NS);
   // Per-warpgroup barriers (128 arrivals) guarding the dQ staging buffers.
-  auto wg_bar = [&](int w) { return bar0 + 8u * (6 + 2 * NS + w); };
-  // Completes when the MMAs reading P^T / dS^T from TMEM (dV, dK, dW) are done.
-  const uint32_t a_done = bar0 + 8u * (8 + 2 * NS);
+  auto wg_bar = [&](int w) { return bar0 + 8u * (8 + 2 * NS + w); };
+  auto a_done = [&](int h) { return bar0 + 8u * (10 + 2 * NS + h); };
   auto ds_buf = [&](int i) { return sb + C::OFF_DS + (C::NDS == 2 ? (i & 1) : 0) * C::PB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -222,14 +235,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), 1);
     }
-    mbar_init(sdp_full, 1);
-    mbar_init(ds_full, 256);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(sdp_full(h), 1);
+      mbar_init(ds_full(h), 128);
+      mbar_init(wg_bar(h), 128);
+      mbar_init(a_done(h), 1);
+    }
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 256);
     mbar_init(drain_bar, 1);
-    mbar_init(wg_bar(0), 128);
-    mbar_init(wg_bar(1), 128);
-    mbar_init(a_done, 1);
     fence_mbar_init();
   }
   if (warp == 8 && lane == 0) {
@@ -280,40 +294,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------ MMA issue (whole warp)
-    constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-    // S^T / s = K Q^T + W U'^T and dP^T = V dO^T for query tile i.
-    auto issue_sdp = [&](int i) -> bool {
+    constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+    // Query half h of tile i:  S^T / s = K Q_h^T + W U'_h^T  and  dP^T = V dO_h^T
+    // into TMEM columns 64h .. 64h + 63 of the S^T / dP^T accumulators.
+    auto issue_sdp = [&](int i, int h) -> bool {
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) return false;
       if (!C::DEFER && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
-      // P^T / dS^T of the previous tile live in the S^T / dP^T columns: the MMAs
-      // reading them must be done before this tile's S^T / dP^T overwrite them.
-      if (i > 0 && !wait_warp(a_done, (i - 1) & 1, g, 41)) return false;
+      // P^T / dS^T of the previous tile live in these columns: the MMAs reading
+      // them must be done before this tile's S^T / dP^T overwrite them.
+      if (i > 0 && !wait_warp(a_done(h), (i - 1) & 1, g, 41)) return false;
       tc_fence_after();
+      const uint32_t tS = tmem + C::T_S + h * 64, tP = tmem + C::T_DP + h * 64;
+      const uint32_t q = st + C::S_Q + h * 64 * (D * 2), o = st + C::S_DO + h * 64 * (D * 2);
       // S^T and dP^T K-steps alternate between the two accumulators.
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2),
-                  desc_kmajor(st + C::S_Q + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
-        umma_bf16(tmem + C::T_DP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2),
-                  desc_kmajor(st + C::S_DO + kk * 32, D * 2), idS, kk > 0 ? 1u : 0u);
+        umma_bf16(tS, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2), desc_kmajor(q + kk * 32, D * 2),
+                  idS, kk > 0 ? 1u : 0u);
+        umma_bf16(tP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2), desc_kmajor(o + kk * 32, D * 2),
+                  idS, kk > 0 ? 1u : 0u);
       }
+      const uint32_t u = st + C::S_U + h * 64 * (C::UW * 2);
 #pragma unroll
       for (int kk = 0; kk < RP / 16; ++kk)
-        umma_bf16(tmem + C::T_S, desc_kmajor(sb + C::OFF_W + kk * 32, RP * 2),
-                  desc_kmajor(st + C::S_U + kk * 32, C::UW * 2), idS, 1u);
-      umma_commit(sdp_full);
+        umma_bf16(tS, desc_kmajor(sb + C::OFF_W + kk * 32, C::UW * 2),
+                  desc_kmajor(u + kk * 32, C::UW * 2), idS, 1u);
+      umma_commit(sdp_full(h));
       return true;
     };
-    // dV += P^T dO, dK += dS^T Q, dW += dS^T U' with A read from TMEM (P^T over
-    // the S^T columns, dS^T over the dP^T columns), K-steps round-robin.
-    auto issue_grad_kv = [&](int i) {
+    // dV += P^T dO, dK += dS^T Q, dW += dS^T U' over the 64 queries of half h,
+    // with A read from TMEM (P^T over the S^T columns, dS^T over the dP^T
+    // columns, packed bf16 in columns 64h .. 64h + 31), K-steps round-robin.
+    auto issue_grad_kv = [&](int i, int h) {
       const uint32_t st = sb + C::OFF_STAGE + (i % NS) * C::STAGE;
       constexpr uint32_t idD = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, false, true);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+      for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
         const uint32_t aoff = (kk >> 2) * 64 + (kk & 3) * 8;
         umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + aoff,
@@ -333,10 +352,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          acc);
         }
       }
-      umma_commit(a_done);
-      umma_commit(q_empty(i % NS));  // Q, dO, U' of this tile are no longer read
+      umma_commit(a_done(h));
     };
-    // dQ = dS K and dU = dS W (A = the dS^T tile read transposed), interleaved.
+    // dQ = dS K and dU = dS W (A = the dS^T tile read transposed): one chain
+    // over [K | W] (N = D + RP) when W is staged beside K, else interleaved.
     auto issue_grad_q = [&](int i) {
       const uint32_t dsb = ds_buf(i);
       constexpr uint32_t idD = idesc_bf16_f32(128, D, true, true);
@@ -344,35 +363,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint64_t ad = desc_mnmajor(dsb + kk * 16 * 128, 128, 128 * 128);
-        umma_bf16(tmem + C::T_DQ, ad,
-                  desc_mnmajor(sb + C::OFF_K + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD,
-                  kk > 0 ? 1u : 0u);
-        if constexpr (RP > 0)
-          umma_bf16(tmem + C::T_DQ + D, ad,
-                    desc_mnmajor(sb + C::OFF_W + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+        if constexpr (C::MERGE_KW) {
+          constexpr uint32_t idQU = idesc_bf16_f32(128, D + RP, true, true);
+          umma_bf16(tmem + C::T_DQ, ad,
+                    desc_mnmajor(sb + C::OFF_K + kk * 16 * 128, 128, C::OFF_W - C::OFF_K), idQU,
                     kk > 0 ? 1u : 0u);
+        } else {
+          umma_bf16(tmem + C::T_DQ, ad,
+                    desc_mnmajor(sb + C::OFF_K + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD,
+                    kk > 0 ? 1u : 0u);
+          if constexpr (RP > 0)
+            umma_bf16(tmem + C::T_DQ + D, ad,
+                      desc_mnmajor(sb + C::OFF_W + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+                      kk > 0 ? 1u : 0u);
+        }
       }
       umma_commit(dq_full);
     };
     bool ok = wait_warp(kv_full, 0, g, 32);
-    if (ok && nq > 0) ok = issue_sdp(0);
+    if (ok && nq > 0) ok = issue_sdp(0, 0) && issue_sdp(0, 1);
     for (int i = 0; ok && i < nq; ++i) {
-      if (!wait_warp(ds_full, i & 1, g, 35)) break;
-      tc_fence_after();
-      issue_grad_kv(i);
       if constexpr (C::DEFER) {
-        // Next tile's scores first, then this tile's dQ | dU (its reduction
-        // happens after the next softmax).
-        if (i + 1 < nq && !issue_sdp(i + 1)) break;
+        // Half by half: its dV / dK / dW MMAs, then its scores of the next tile,
+        // so that one warpgroup's softmax overlaps the other half's MMAs; this
+        // tile's dQ | dU last (their reduction happens after the next softmax).
+        for (int h = 0; ok && h < 2; ++h) {
+          if (!wait_warp(ds_full(h), i & 1, g, 35)) { ok = false; break; }
+          tc_fence_after();
+          issue_grad_kv(i, h);
+          if (h == 1) umma_commit(q_empty(i % NS));  // Q, dO, U' of this tile are read
+          if (i + 1 < nq && !issue_sdp(i + 1, h)) ok = false;
+        }
+        if (!ok) break;
         if (i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 36)) break;
         tc_fence_after();
         issue_grad_q(i);
       } else {
+        if (!wait_warp(ds_full(0), i & 1, g, 35) || !wait_warp(ds_full(1), i & 1, g, 35)) break;
+        tc_fence_after();
+        issue_grad_kv(i, 0);
+        issue_grad_kv(i, 1);
+        umma_commit(q_empty(i % NS));
         // dQ | dU overwrite the S^T columns that dV / dK / dW read P^T from.
-        if (!wait_warp(a_done, i & 1, g, 42)) break;
+        if (!wait_warp(a_done(1), i & 1, g, 42)) break;
         tc_fence_after();
         issue_grad_q(i);
-        if (i + 1 < nq && !issue_sdp(i + 1)) break;
+        if (i + 1 < nq && !(issue_sdp(i + 1, 0) && issue_sdp(i + 1, 1))) break;
       }
     }
     umma_commit(drain_bar);
@@ -403,15 +439,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int s = i % NS;
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(q_full(s), (i / NS) & 1, g, 37)) return false;
-      if (!wait_warp(sdp_full, i & 1, g, 38)) return false;
+      if (!wait_warp(sdp_full(wg), i & 1, g, 38)) return false;
       tc_fence_after();
       if constexpr (C::DEFER) {
-        // Block wg of this dS buffer staged dQ | dU chunk wg of tile i - 2; the
-        // reduction reading it is followed by (2 * my_chunks - 1) newer ones.
+        // Block wg of this dS buffer staged this warpgroup's first dQ | dU chunk
+        // of tile i - 2; the last reductions issued are reduce_dq(i - 2)'s, so
+        // only its later chunks (from the staging buffer) may still be read.
         if (i >= 2) {
           if (leader) {
-            if (my_chunks >= 2) bulk_wait_read<3>();
-            else bulk_wait_read<1>();
+            if (my_chunks >= 2) bulk_wait_read<1>();
+            else bulk_wait_read<0>();
           }
           if (!wg_sync()) return false;
         }
@@ -459,7 +496,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(ds_full(wg));
       return true;
     };
     // Partial dQ | dU of tile j (TMEM lane = query row): this warpgroup reads its

@@ -15,16 +15,17 @@
 //   * fwd_window_kernel  (N <= 128): persistent CTAs; each 128-row tile packs
 //     128/NP whole windows (NP = 64 or 128 rows per window).  One S tile per
 //     tile, single-pass softmax, block-diagonal P (off-window blocks stay 0).
-//   * fwd_long_kernel    (N > 128): one CTA per (head, two 128-query tiles);
-//     loops over 128-key tiles with an online softmax (lazy rescale of O in
-//     TMEM); one softmax warpgroup per query tile, running out of phase.
-//
-// Window kernel warp roles (320 threads): warps 0-3 and 4-7 softmax + epilogue
-// of even and odd tiles (thread = row = TMEM lane), warp 8 TMA producer, warp 9
-// U' scaling + MMA issue + TMEM allocation.  The long kernel uses 320 threads: warps 0-7 softmax (one
-// warpgroup per query tile), warp 8 TMA, warp 9 MMA.  Operands are staged by TMA with the swizzle that matches
-// their row width; P is written by the softmax threads into a 128-byte
-// swizzled K-major tile.
+//     Warps 0-3 and 4-7 softmax + epilogue of even and odd tiles (thread = row
+//     = TMEM lane), warp 8 TMA producer, warp 9 U' scaling + MMA issue; P is
+//     written into a 128-byte-swizzled K-major shared-memory tile.
+//   * fwd_long_kernel    (N > 128): persistent CTAs over units (head, two
+//     128-query tiles); each unit loops over 128-key tiles with an online
+//     softmax (lazy rescale of O in TMEM).  Warpgroups 0 / 1 softmax of query
+//     tile 0 / 1 (running out of phase), warp 8 TMA, warps 9 / 10 MMA issue
+//     for tile 0 / 1; P goes back into TMEM as packed bf16 and the PV MMA
+//     reads it from there.  The softmax warpgroups take registers from the
+//     control warpgroup (setmaxnreg).
+// Operands are staged by TMA with the swizzle that matches their row width.
 #pragma once
 #include "sm100.cuh"
 
@@ -95,24 +96,31 @@ __device__ __forceinline__ void mask_tail(uint32_t (&sv)[NC], int valid) {
     if (c >= valid) sv[c] = 0xFF800000u;
 }
 
-// Row maximum with 8 independent partial maxima (short dependency chains).
+// Row maximum with 8 independent partial maxima (short dependency chains),
+// two new values per three-input max.
 template <int NC>
 __device__ __forceinline__ float row_max(const uint32_t (&sv)[NC]) {
   float m[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) m[e] = __uint_as_float(sv[e]);
+  int c = 8;
 #pragma unroll
-  for (int c = 8; c < NC; c += 8)
+  for (; c + 16 <= NC; c += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      m[e] = fmax3(m[e], __uint_as_float(sv[c + e]), __uint_as_float(sv[c + 8 + e]));
+  if (c < NC) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], __uint_as_float(sv[c + e]));
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+  }
+  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // p_j = 2^(s_j * sl2 - m) written as bf16 into the 128-byte-swizzled K-major P
 // tile (row `row`, columns col0..col0+NC); returns sum_j p_j (fp32, 8 partial
 // sums).  Masked scores are -inf and give p = 0.
-// SOFT_PAIRS of every 8 exponentials use the software exp2 (FMA / integer
-// pipes) instead of the MUFU unit.
+// SOFT_PAIRS of every 4 pairs of exponentials use the software exp2 (FMA /
+// integer pipes) instead of the MUFU unit.
 template <int NC, int SOFT_PAIRS = 0>
 __device__ __forceinline__ float exp_row_to_smem(const uint32_t (&sv)[NC], float sl2, float m,
                                                  uint32_t pbuf, int row, int col0) {
@@ -137,6 +145,38 @@ __device__ __forceinline__ float exp_row_to_smem(const uint32_t (&sv)[NC], float
   return ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
 }
 
+// As exp_row_to_smem, but the bf16 pairs go to this thread's TMEM lane (column
+// p_tm + c / 2 holds keys c and c + 1), where the PV MMA reads them as its A
+// operand.  The stores are issued without waiting (tmem_st_wait() follows).
+template <int NC, int SOFT_PAIRS = 0>
+__device__ __forceinline__ float exp_row_to_tmem(const uint32_t (&sv)[NC], float sl2, float m,
+                                                 uint32_t p_tm) {
+  constexpr int HW = 8 - 2 * SOFT_PAIRS;
+  float l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) l[e] = 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < NC; c0 += 32) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = c0; c < c0 + 32; c += 8) {
+      float p[8];
+#pragma unroll
+      for (int e = 0; e < HW; ++e) p[e] = fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
+#pragma unroll
+      for (int e = HW; e < 8; e += 2)
+        soft_exp2_x2(fmaf(__uint_as_float(sv[c + e]), sl2, -m),
+                     fmaf(__uint_as_float(sv[c + e + 1]), sl2, -m), p[e], p[e + 1]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) l[e & 3] += p[e];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) pk[(c - c0 + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+    }
+    tmem_st16_nowait(p_tm + (c0 >> 1), pk);
+  }
+  return (l[0] + l[1]) + (l[2] + l[3]);
+}
+
 // Issue the score MMAs  S(tmem) = Q.K^T + U'.W^T  for one 128x128 tile.
 template <int D, int RP>
 __device__ __forceinline__ void issue_scores(uint32_t s_tmem, uint32_t q, uint32_t k, uint32_t u,
@@ -149,6 +189,18 @@ __device__ __forceinline__ void issue_scores(uint32_t s_tmem, uint32_t q, uint32
 #pragma unroll
   for (int kk = 0; kk < RP / 16; ++kk)
     umma_bf16(s_tmem, desc_kmajor(u + kk * 32, RP * 2), desc_kmajor(w + kk * 32, RP * 2), id, 1u);
+}
+
+// Issue O(tmem) (+)= P . V for a 128-key tile with P read from TMEM (packed
+// bf16, 8 columns per 16 keys), V MN-major in shared memory.
+template <int D>
+__device__ __forceinline__ void issue_pv_ts(uint32_t o_tmem, uint32_t p_tmem, uint32_t v,
+                                            bool accumulate) {
+  constexpr uint32_t id = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_mnmajor(v + kk * 16 * (D * 2), D * 2, 128 * D * 2),
+                 id, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Issue O(tmem) (+)= P . V for a 128-key tile; P is K-major in two 64-key
@@ -361,33 +413,42 @@ struct LongCfg {
   static constexpr int QB = kTile * D * 2;
   static constexpr int UB = kTile * RP * 2;
   static constexpr int STAGE = 2 * QB + UB;  // K, V, W
-  static constexpr int PB = kTile * kTile * 2;
-  // Two query tiles per CTA: Q0 U0 Q1 U1, KV stages, P0 P1.
+  // Two query tiles per CTA: Q0 U0 Q1 U1, then the KV stages.  P lives in TMEM.
   static constexpr int OFF_Q = 0;            // Q tile t at OFF_Q + t * (QB + UB), U right after
   static constexpr int OFF_STAGE = 2 * (QB + UB);
-  static constexpr int NS_FIT = (226 * 1024 - OFF_STAGE - 2 * PB) / STAGE;
-  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
-  static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_BAR = OFF_P + 2 * PB;
+  static constexpr int NS_FIT = (226 * 1024 - OFF_STAGE) / STAGE;
+  static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
+  static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
+  // TMEM columns: S_t at 128 t, O_t at 256 + D t, P_t (packed bf16) at 384 + 64 t.
+  static constexpr int T_O = 256, T_P = 384;
   // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
-  static constexpr int NBAR = 2 * NS + 10;
+  // q_empty o_empty[2]
+  static constexpr int NBAR = 2 * NS + 13;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static_assert(NS >= 2, "not enough shared memory for two KV stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
 };
 
-// warps 0-3 softmax of query tile 0, 4-7 of tile 1, 8 TMA, 9 / 10 MMA issue for tile 0 / 1
-constexpr int kLongThreads = 352;
-// Pairs of every 8 softmax exponentials computed in software in the long
-// forward (the MUFU unit is its limit; 1 pair = 25 %).
+// Warpgroups 0 / 1: softmax of query tile 0 / 1; warpgroup 2: warp 8 TMA, warps
+// 9 / 10 MMA issue for tile 0 / 1, warp 11 idle.  Registers: launched with 168
+// per thread (384 x 168 = 64512); warpgroup 2 gives its share down to 56 and
+// the softmax warpgroups take 208 (2 x 128 x 208 + 128 x 56 = 60416 <= 64512).
+constexpr int kLongThreads = 384;
+constexpr uint32_t kLongSoftmaxRegs = 208, kLongControlRegs = 56;
+static_assert(2 * 128 * kLongSoftmaxRegs + 128 * kLongControlRegs <= kLongThreads * 168,
+              "register split exceeds the launch budget");
+// Pairs of every 4 softmax exponentials computed in software in the long
+// forward (the MUFU unit is its limit): one, measured best for d = 32 and 64.
 constexpr int kLongSoftPairs = 1;
 
-// Long regime: one CTA per (head, pair of 128-query tiles), looping over
-// 128-key tiles.  Each query tile has its own softmax warpgroup, MMA-issuing
-// warp, S buffer (TMEM columns t*128), O accumulator (TMEM 256 + t*D) and P
-// buffer; the two pipelines run independently and out of phase, so one's
-// exponentials overlap the other's loads, maxima and waits, and each K/V tile
-// serves 256 query rows.
+// Long regime: a persistent CTA per SM works through units (head, pair of
+// 128-query tiles), each a loop over 128-key tiles.  Each query tile of a unit
+// has its own softmax warpgroup, MMA-issuing warp, S buffer (TMEM columns
+// t*128), O accumulator (TMEM 256 + t*D) and P buffer (TMEM 384 + 64 t); the two
+// pipelines run independently and out of phase, so one's exponentials overlap
+// the other's loads, maxima and waits, and each K/V tile serves 256 query rows.
+// Barrier phases run on across units, so the K/V loads and the scores of the
+// next unit start while the current unit's last tiles and epilogue finish.
 template <int D, int RP>
 __global__ void __launch_bounds__(kLongThreads, 1)
     fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
@@ -407,6 +468,10 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   auto p_full = [&](int t) { return bar0 + 8u * (5 + 2 * NS + t); };
   auto pv_done = [&](int t) { return bar0 + 8u * (7 + 2 * NS + t); };
   const uint32_t drain_bar = bar0 + 8u * (9 + 2 * NS);
+  // The unit's last score MMAs are done (Q / U' may be replaced), and tile t's
+  // epilogue has read O (the next unit's first PV may overwrite it).
+  const uint32_t q_empty = bar0 + 8u * (10 + 2 * NS);
+  auto o_empty = [&](int t) { return bar0 + 8u * (11 + 2 * NS + t); };
   auto q_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB); };
   auto u_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB) + C::QB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
@@ -415,13 +480,17 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   const int warp = static_cast<int>(warp_id());
   const int lane = static_cast<int>(lane_id());
   const int N = args.N;
-  const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * 2 * kTile;
   const int nkv = (N + kTile - 1) / kTile;
+  const int npairs = (N + 2 * kTile - 1) / (2 * kTile);
+  const int nunits = npairs * args.BH;
+  // Units of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...  (consecutive
+  // units share a head, so concurrent CTAs read the same K / V from L2).
+  const int first = blockIdx.x, stride = gridDim.x;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 2);  // one commit per query tile's MMA warp
     for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 2);  // one arrival per query tile's MMA warp
@@ -431,6 +500,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       mbar_init(s_empty(t), 128);
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
+      mbar_init(o_empty(t), 128);
     }
     mbar_init(drain_bar, 2);
     fence_mbar_init();
@@ -454,123 +524,151 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns};
 
-  if (warp == 8) {
+  if (warp >= 8) {
+   // Control warpgroup: all four warps shrink their budget at this point.
+   warpgroup_reg_dealloc<kLongControlRegs>();
+   if (warp == 8) {
     if (lane == 0) {
-      mbar_expect_tx(q_full, 2 * (C::QB + C::UB));
-      for (int t = 0; t < 2; ++t) {
-        tma_load_3d(q_addr(t), &mQ, q_full, 0, q0 + t * kTile, bh);
-        if constexpr (RP > 0) tma_load_3d(u_addr(t), &mU, q_full, 0, q0 + t * kTile, bh);
+      int it = 0, uc = 0;  // K/V tiles and units loaded so far
+      bool ok = true;
+      for (int u = first; ok && u < nunits; u += stride, ++uc) {
+        const int bh = u / npairs, q0 = (u % npairs) * 2 * kTile;
+        if (uc > 0 && !wait_bounded(q_empty, (uc - 1) & 1, g, 10)) break;
+        mbar_expect_tx(q_full, 2 * (C::QB + C::UB));
+        for (int t = 0; t < 2; ++t) {
+          tma_load_3d(q_addr(t), &mQ, q_full, 0, q0 + t * kTile, bh);
+          if constexpr (RP > 0) tma_load_3d(u_addr(t), &mU, q_full, 0, q0 + t * kTile, bh);
+        }
+        for (int j = 0; j < nkv; ++j, ++it) {
+          const int s = it % NS;
+          if (it >= NS && !wait_bounded(kv_empty(s), ((it / NS) + 1) & 1, g, 11)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
+          mbar_expect_tx(kv_full(s), C::STAGE);
+          tma_load_3d(st, &mK, kv_full(s), 0, j * kTile, bh);
+          tma_load_3d(st + C::QB, &mV, kv_full(s), 0, j * kTile, bh);
+          if constexpr (RP > 0) tma_load_3d(st + 2 * C::QB, &mW, kv_full(s), 0, j * kTile, bh);
+        }
       }
-      int j = 0;
-      for (; j < nkv; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !wait_bounded(kv_empty(s), ((j / NS) + 1) & 1, g, 11)) break;
-        const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-        mbar_expect_tx(kv_full(s), C::STAGE);
-        tma_load_3d(st, &mK, kv_full(s), 0, j * kTile, bh);
-        tma_load_3d(st + C::QB, &mV, kv_full(s), 0, j * kTile, bh);
-        if constexpr (RP > 0) tma_load_3d(st + 2 * C::QB, &mW, kv_full(s), 0, j * kTile, bh);
-      }
-      wait_drain(q_full, 0, args.timeout_ns);
-      for (int i = (j > NS ? j - NS : 0); i < j; ++i)
+      // No copy may still be in flight when the CTA exits.
+      if (uc > 0) wait_drain(q_full, (uc - 1) & 1, args.timeout_ns);
+      for (int i = (it > NS ? it - NS : 0); i < it; ++i)
         wait_drain(kv_full(i % NS), (i / NS) & 1, args.timeout_ns);
     }
-  } else if (warp >= 9) {
+   } else if (warp == 9 || warp == 10) {
     // MMA issue for query tile t = warp - 9 (one converged warp each).
     const int t = warp - 9;
-    bool ok = wait_warp(q_full, 0, g, 12);
-    if (ok) {
-      if constexpr (RP > 0) {
-        scale_tile_bf16(u_addr(t), C::UB, args.inv_scale);
-        fence_async_smem();
-      }
-      __syncwarp();
-    }
-    // S_t = Q_t K_j^T + U'_t W_j^T into tile t's S columns, once its warpgroup
-    // has loaded the previous scores (s_empty).
-    auto do_s = [&](int j) -> bool {
-      const int s = j % NS;
-      if (!wait_warp(kv_full(s), (j / NS) & 1, g, 13)) return false;
-      if (j >= 1 && !wait_warp(s_empty(t), (j - 1) & 1, g, 14)) return false;
+    int it = 0, jt = 0, uc = 0;  // K/V tiles, S tiles of this query tile, units
+    bool ok = true;
+    // S_t = Q_t K^T + U'_t W^T for K/V tile `it` into tile t's S columns, once
+    // its warpgroup has loaded the previous scores (s_empty).
+    auto do_s = [&](int itj, int jtj) -> bool {
+      const int s = itj % NS;
+      if (!wait_warp(kv_full(s), (itj / NS) & 1, g, 13)) return false;
+      if (jtj >= 1 && !wait_warp(s_empty(t), (jtj - 1) & 1, g, 14)) return false;
       tc_fence_after();
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       issue_scores<D, RP>(tmem + t * 128, q_addr(t), st, u_addr(t), st + 2 * C::QB);
       umma_commit(s_full(t));
       return true;
     };
-    auto do_pv = [&](int j) -> bool {
-      const int s = j % NS;
-      if (!wait_warp(p_full(t), j & 1, g, 15)) return false;
+    auto do_pv = [&](int itj, int jtj, bool first_of_unit) -> bool {
+      const int s = itj % NS;
+      if (!wait_warp(p_full(t), jtj & 1, g, 15)) return false;
       tc_fence_after();
-      issue_pv<D>(tmem + 256 + t * D, sb + C::OFF_P + t * C::PB,
-                  sb + C::OFF_STAGE + s * C::STAGE + C::QB, j > 0);
+      issue_pv_ts<D>(tmem + C::T_O + t * D, tmem + C::T_P + t * 64,
+                     sb + C::OFF_STAGE + s * C::STAGE + C::QB, !first_of_unit);
       umma_commit(pv_done(t));
       umma_commit(kv_empty(s));
       return true;
     };
-    if (ok) ok = do_s(0);
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (j + 1 < nkv && !do_s(j + 1)) break;
-      if (!do_pv(j)) break;
+    for (int u = first; ok && u < nunits; u += stride, ++uc) {
+      if (!wait_warp(q_full, uc & 1, g, 12)) break;
+      if constexpr (RP > 0) {
+        scale_tile_bf16(u_addr(t), C::UB, args.inv_scale);
+        fence_async_smem();
+      }
+      __syncwarp();
+      ok = do_s(it, jt);
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv) {
+          if (!do_s(it + 1, jt + 1)) { ok = false; break; }
+        } else {
+          umma_commit(q_empty);  // the unit's last scores read Q_t / U'_t
+        }
+        // The previous unit's epilogue must have read O before it is overwritten.
+        if (j == 0 && uc > 0 && !wait_warp(o_empty(t), (uc - 1) & 1, g, 18)) { ok = false; break; }
+        if (!do_pv(it, jt, j == 0)) { ok = false; break; }
+        ++it;
+        ++jt;
+      }
     }
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
+   }
   } else {
+    warpgroup_reg_alloc<kLongSoftmaxRegs>();
     const int t = warp >> 2;             // query tile of this warpgroup
     const int row = threadIdx.x & 127;   // TMEM lane == query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_tm = tmem + lane_base + t * 128;
-    const uint32_t o_tm = tmem + lane_base + 256 + t * D;
-    const uint32_t pbuf = sb + C::OFF_P + t * C::PB;
+    const uint32_t o_tm = tmem + lane_base + C::T_O + t * D;
+    const uint32_t p_tm = tmem + lane_base + C::T_P + t * 64;
     const float sl2 = args.scale_log2;
-    float m_run = -INFINITY, l = 0.f;
+    int jt = 0;  // S tiles of this query tile so far
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!wait_warp(s_full(t), j & 1, g, 16)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[128];
-      tmem_ld_cols<128>(s_tm, sv);
-      tc_fence_before();
-      mbar_arrive(s_empty(t));
-      const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
-      if (kvalid < kTile) mask_tail<128>(sv, kvalid);
-      const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);
-      // Lazy rescale: keep the running max unless it grew by more than 2^8.
-      const bool need = m_new > m_run + 8.0f;
-      float alpha = 1.f;
-      if (need) {
-        alpha = fast_exp2(m_run - m_new);
-        l *= alpha;
-        m_run = m_new;
-      }
-      const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
-      // The single P buffer of this tile and O: PV_{j-1} must have finished.
-      if (j >= 1 && !wait_warp(pv_done(t), (j - 1) & 1, g, 17)) { ok = false; break; }
-      l += exp_row_to_smem<128, kLongSoftPairs>(sv, sl2, m_run, pbuf, row, 0);
-      if (fix_o) {
+    for (int u = first; ok && u < nunits; u += stride) {
+      const int bh = u / npairs, q0 = (u % npairs) * 2 * kTile;
+      float m_run = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j, ++jt) {
+        if (!wait_warp(s_full(t), jt & 1, g, 16)) { ok = false; break; }
         tc_fence_after();
-        uint32_t ov[D];
-        tmem_ld_cols<D>(o_tm, ov);
-#pragma unroll
-        for (int c = 0; c < D; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-        tmem_st_cols<D>(o_tm, ov);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full(t));
-    }
-    if (ok && nkv > 0) {
-      if (wait_warp(pv_done(t), (nkv - 1) & 1, g, 19)) {
-        tc_fence_after();
-        uint32_t ov[D];
-        tmem_ld_cols<D>(o_tm, ov);
-        const int q = q0 + t * kTile + row;
-        if (q < N) {
-          const size_t r = static_cast<size_t>(bh) * N + q;
-          store_o_row<D>(args.o + r * D, ov, 1.0f / l);
-          args.lse[r] = (m_run + __log2f(l)) * kLn2;
+        uint32_t sv[128];
+        tmem_ld_cols<128>(s_tm, sv);
+        tc_fence_before();
+        mbar_arrive(s_empty(t));
+        const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
+        if (kvalid < kTile) mask_tail<128>(sv, kvalid);
+        const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);
+        // Lazy rescale: keep the running max unless it grew by more than 2^8.
+        const bool need = m_new > m_run + 8.0f;
+        float alpha = 1.f;
+        if (need) {
+          alpha = fast_exp2(m_run - m_new);
+          l *= alpha;
+          m_run = m_new;
         }
+        const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
+        // The P buffer of this tile and O: the previous PV must have finished.
+        if (jt >= 1 && !wait_warp(pv_done(t), (jt - 1) & 1, g, 17)) { ok = false; break; }
+        tc_fence_after();
+        l += exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
+        if (fix_o) {
+          uint32_t ov[D];
+          tmem_ld_cols<D>(o_tm, ov);
+#pragma unroll
+          for (int c = 0; c < D; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st_cols<D>(o_tm, ov);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full(t));
+      }
+      if (!ok || nkv == 0) break;
+      if (!wait_warp(pv_done(t), (jt - 1) & 1, g, 19)) break;
+      tc_fence_after();
+      uint32_t ov[D];
+      tmem_ld_cols<D>(o_tm, ov);
+      tc_fence_before();
+      mbar_arrive(o_empty(t));
+      const int q = q0 + t * kTile + row;
+      if (q < N) {
+        const size_t r = static_cast<size_t>(bh) * N + q;
+        store_o_row<D>(args.o + r * D, ov, 1.0f / l);
+        args.lse[r] = (m_run + __log2f(l)) * kLn2;
       }
     }
   }

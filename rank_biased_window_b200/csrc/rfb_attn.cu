@@ -275,11 +275,13 @@ int launch_window(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
 }
 
 template <int D, int RP>
-int launch_long(const Maps& m, const FwdArgs& a, cudaStream_t st) {
+int launch_long(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   using C = LongCfg<D, RP>;
   static std::atomic<uint64_t> done{0};
   if (int rc = ensure_smem(fwd_long_kernel<D, RP>, C::SMEM, done)) return rc;
-  const dim3 grid((a.N + 2 * kTile - 1) / (2 * kTile), a.BH);
+  // Persistent: one CTA per SM (at most one per unit).
+  const long long units = static_cast<long long>((a.N + 2 * kTile - 1) / (2 * kTile)) * a.BH;
+  const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
   LaunchTimer timer(kIdFwd, st);
   fwd_long_kernel<D, RP><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
@@ -289,7 +291,7 @@ template <int D, int RP>
 int dispatch_fwd(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   if (a.N <= 64) return launch_window<D, RP, 64>(m, a, sms, st);
   if (a.N <= 128) return launch_window<D, RP, 128>(m, a, sms, st);
-  return launch_long<D, RP>(m, a, st);
+  return launch_long<D, RP>(m, a, sms, st);
 }
 
 int dispatch_fwd_rp(int d, int rp, const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
@@ -452,10 +454,10 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   if (!rc) rc = encode_3d(&m.g, dout, d, N, BH, d, kTile, 1);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   // The backward stages U' = U / s once (bwd_pre) and tiles that copy.
-  // With d = 64 the U' tile is staged 64 columns wide (zero padded), so it can
-  // sit beside Q as one MMA operand.
+  // With d = 64 the U' and W tiles are staged 64 columns wide (zero padded), so
+  // they sit beside Q and K as one MMA operand each.
   if (!rc && r > 0) rc = encode_3d(&m.u, ws + L.uprime, r, N, BH, d == 64 ? 64 : rp, kTile, 1);
-  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, kTile, 1);
+  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, d == 64 ? 64 : rp, kTile, 1);
   if (!rc) rc = encode_acc_3d(&m.acc, ws + L.acc, d + r, N, BH);
   if (rc) return rc;
   BwdArgs a;

@@ -15,6 +15,7 @@
 namespace rfb {
 
 // Status codes written into the device error word (kept equal to the C-ABI codes).
+constexpr int kErrAlignment = 3;
 constexpr int kErrDeviceTimeout = 6;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -276,6 +277,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Per-warpgroup register budget changes (all four warps of a warpgroup execute
+// the same one).  The budgets of all warpgroups must add up to no more than the
+// registers the CTA was launched with.
+template <uint32_t R>
+__device__ __forceinline__ void warpgroup_reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void warpgroup_reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+
+// max(a, b, c) in one instruction (three-input max.f32 of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Packed fp32 pairs (Blackwell f32x2 arithmetic): lo in the low 32 bits.
