@@ -52,6 +52,8 @@ _lib = None
 def load_library(path: str = LIB_PATH):
     """Load (once) and return the ctypes handle; raises if the .so is absent."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lock:
         if _lib is None:
             if not os.path.exists(path):
@@ -90,7 +92,27 @@ def _stream_ptr(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+class _on_device:
+    """Makes `device` current for the call; a no-op when it already is."""
+
+    def __init__(self, device):
+        self.ctx = (None if device.index == torch.cuda.current_device()
+                    else torch.cuda.device(device))
+
+    def __enter__(self):
+        if self.ctx is not None:
+            self.ctx.__enter__()
+
+    def __exit__(self, *exc):
+        if self.ctx is not None:
+            self.ctx.__exit__(*exc)
+
+
 def _check_operand(name, t, shape, device):
+    # Fast path: one combined test; the detailed messages only on failure.
+    if (isinstance(t, torch.Tensor) and t.dtype is torch.bfloat16 and t.device == device
+            and t.shape == shape and t.is_contiguous()):
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != torch.bfloat16:
@@ -128,7 +150,7 @@ def attn_fwd(q, k, v, u=None, w=None, scale=None, *, out=None, lse=None, stream=
     _check_operand("out", o, (B, H, N, d), dev)
     if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
         raise ValueError("lse must be contiguous fp32 [B, H, N]")
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = load_library().rfb_attn_fwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
             ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, H, N, d, r, s,
@@ -165,7 +187,7 @@ def attn_bwd(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=None, grads=N
     nbytes = bwd_workspace_size(B, H, N, d, r)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = load_library().rfb_attn_bwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
             ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
@@ -201,7 +223,7 @@ def attn_bwd_noalloc(q, k, v, u, w, o, lse, dout, scale=None, *, grads=None, str
         dw = torch.empty_like(w) if r else None
     else:
         dq, dk, dv, du, dw = grads
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = load_library().rfb_attn_bwd_noalloc(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
             ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),

@@ -16,8 +16,8 @@
 //     128/NP whole windows (NP = 64 or 128 rows per window).  One S tile per
 //     tile, single-pass softmax, block-diagonal P (off-window blocks stay 0).
 //     Warps 0-3 and 4-7 softmax + epilogue of even and odd tiles (thread = row
-//     = TMEM lane), warp 8 TMA producer, warp 9 U' scaling + MMA issue; P is
-//     written into a 128-byte-swizzled K-major shared-memory tile.
+//     = TMEM lane), warp 8 TMA producer, warp 9 score MMAs, warp 10 PV MMAs,
+//     warp 11 U' scaling; P goes back into TMEM (packed bf16) for the PV MMA.
 //   * fwd_long_kernel    (N > 128): persistent CTAs over units (head, two
 //     128-query tiles); each unit loops over 128-key tiles with an online
 //     softmax (lazy rescale of O in TMEM).  Warpgroups 0 / 1 softmax of query
@@ -116,38 +116,12 @@ __device__ __forceinline__ float row_max(const uint32_t (&sv)[NC]) {
   return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// p_j = 2^(s_j * sl2 - m) written as bf16 into the 128-byte-swizzled K-major P
-// tile (row `row`, columns col0..col0+NC); returns sum_j p_j (fp32, 8 partial
-// sums).  Masked scores are -inf and give p = 0.
-// SOFT_PAIRS of every 4 pairs of exponentials use the software exp2 (FMA /
-// integer pipes) instead of the MUFU unit.
-template <int NC, int SOFT_PAIRS = 0>
-__device__ __forceinline__ float exp_row_to_smem(const uint32_t (&sv)[NC], float sl2, float m,
-                                                 uint32_t pbuf, int row, int col0) {
-  constexpr int HW = 8 - 2 * SOFT_PAIRS;  // exponentials per 8 on the MUFU unit
-  float l[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) l[e] = 0.f;
-#pragma unroll
-  for (int c = 0; c < NC; c += 8) {
-    float p[8];
-#pragma unroll
-    for (int e = 0; e < HW; ++e) p[e] = fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
-#pragma unroll
-    for (int e = HW; e < 8; e += 2)
-      soft_exp2_x2(fmaf(__uint_as_float(sv[c + e]), sl2, -m),
-                   fmaf(__uint_as_float(sv[c + e + 1]), sl2, -m), p[e], p[e + 1]);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) l[e] += p[e];
-    st_shared_v4(pbuf + sw128_offset(row, col0 + c, 128), pack_bf16x2(p[0], p[1]),
-                 pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-  }
-  return ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
-}
-
-// As exp_row_to_smem, but the bf16 pairs go to this thread's TMEM lane (column
-// p_tm + c / 2 holds keys c and c + 1), where the PV MMA reads them as its A
-// operand.  The stores are issued without waiting (tmem_st_wait() follows).
+// p_j = 2^(s_j * sl2 - m) for the NC scores of this thread's row, written as
+// packed bf16 pairs into its TMEM lane (column p_tm + c / 2 holds keys c and
+// c + 1), where the PV MMA reads them as its A operand; returns sum_j p_j
+// (fp32, 4 partial sums).  Masked scores are -inf and give p = 0.  SOFT_PAIRS
+// of every 4 pairs of exponentials use the software exp2 (FMA / integer pipes)
+// instead of the MUFU unit.  The stores are not awaited (tmem_st_wait()).
 template <int NC, int SOFT_PAIRS = 0>
 __device__ __forceinline__ float exp_row_to_tmem(const uint32_t (&sv)[NC], float sl2, float m,
                                                  uint32_t p_tm) {
@@ -203,19 +177,6 @@ __device__ __forceinline__ void issue_pv_ts(uint32_t o_tmem, uint32_t p_tmem, ui
                  id, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// Issue O(tmem) (+)= P . V for a 128-key tile; P is K-major in two 64-key
-// column blocks of 128 rows, V is MN-major (rows = keys, D contiguous).
-template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p, uint32_t v, bool accumulate) {
-  constexpr uint32_t id = idesc_bf16_f32(128, D, false, true);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint64_t ad = desc_kmajor(p + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 128);
-    const uint64_t bd = desc_mnmajor(v + kk * 16 * (D * 2), D * 2, 128 * D * 2);
-    umma_bf16(o_tmem, ad, bd, id, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-
 // ============================================================ window regime
 template <int D, int RP, int NP>
 struct WinCfg {
@@ -223,20 +184,27 @@ struct WinCfg {
   static constexpr int QB = kTile * D * 2;    // bytes of a Q / K / V tile
   static constexpr int UB = kTile * RP * 2;   // bytes of a U / W tile
   static constexpr int STAGE = 3 * QB + 2 * UB;
-  static constexpr int PB = kTile * kTile * 2;
-  static constexpr int NS_FIT = (224 * 1024 - 2 * PB) / STAGE;
-  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
-  static constexpr int OFF_P = NS * STAGE;
-  static constexpr int OFF_BAR = OFF_P + 2 * PB;
-  // in_full[NS] in_empty[NS] s_full[2] p_full[2] o_full[2] acc_empty[2] drain
-  static constexpr int NBAR = 2 * NS + 9;
+  static constexpr int NS_FIT = (224 * 1024) / STAGE;
+  static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
+  static constexpr int OFF_BAR = NS * STAGE;
+  // TMEM columns: S_a at 128 a, O_a at 256 + D a, P_a (packed bf16) at 384 + 64 a.
+  static constexpr int T_O = 256, T_P = 384;
+  // in_full[NS] u_ready[NS] in_empty[NS] s_full[2] s_empty[2] p_full[2] o_full[2]
+  // acc_empty[2] drain
+  static constexpr int NBAR = 3 * NS + 11;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static_assert(NS >= 2, "not enough shared memory for two input stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
   static_assert(QB % 1024 == 0 && UB % 1024 == 0, "tile alignment");
 };
 
-constexpr int kWinThreads = 320;  // warps 0-3 / 4-7 softmax of even / odd tiles, 8 TMA, 9 MMA
+// Warps 0-3 / 4-7 softmax + epilogue of even / odd tiles, 8 TMA, 9 score MMAs,
+// 10 PV MMAs, 11 U' scaling.  Registers as in the long kernel: launched with 168
+// per thread, control warpgroup down to 56, softmax warpgroups up to 208.
+constexpr int kWinThreads = 384;
+constexpr uint32_t kWinSoftmaxRegs = 208, kWinControlRegs = 56;
+static_assert(2 * 128 * kWinSoftmaxRegs + 128 * kWinControlRegs <= kWinThreads * 168,
+              "register split exceeds the launch budget");
 
 template <int D, int RP, int NP>
 __global__ void __launch_bounds__(kWinThreads, 1)
@@ -250,12 +218,14 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar0 = sb + C::OFF_BAR;
   auto in_full = [&](int s) { return bar0 + 8u * s; };
-  auto in_empty = [&](int s) { return bar0 + 8u * (NS + s); };
-  auto s_full = [&](int a) { return bar0 + 8u * (2 * NS + a); };
-  auto p_full = [&](int a) { return bar0 + 8u * (2 * NS + 2 + a); };
-  auto o_full = [&](int a) { return bar0 + 8u * (2 * NS + 4 + a); };
-  auto acc_empty = [&](int a) { return bar0 + 8u * (2 * NS + 6 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * NS + 8);
+  auto u_ready = [&](int s) { return bar0 + 8u * (NS + s); };  // U' scaled in stage s
+  auto in_empty = [&](int s) { return bar0 + 8u * (2 * NS + s); };
+  auto s_full = [&](int a) { return bar0 + 8u * (3 * NS + a); };
+  auto s_empty = [&](int a) { return bar0 + 8u * (3 * NS + 2 + a); };
+  auto p_full = [&](int a) { return bar0 + 8u * (3 * NS + 4 + a); };
+  auto o_full = [&](int a) { return bar0 + 8u * (3 * NS + 6 + a); };
+  auto acc_empty = [&](int a) { return bar0 + 8u * (3 * NS + 8 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (3 * NS + 10);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -267,15 +237,17 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     *abort_flag = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(in_full(s), 1);
+      mbar_init(u_ready(s), 1);
       mbar_init(in_empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full(a), 1);
+      mbar_init(s_empty(a), 128);
       mbar_init(p_full(a), 128);
       mbar_init(o_full(a), 1);
       mbar_init(acc_empty(a), 128);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_bar, 2);
     fence_mbar_init();
   }
   if (warp == 8 && lane == 0) {
@@ -291,20 +263,16 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp < 8) {
-    // P buffers start at zero: with NP = 64 each row only ever writes its own
-    // window's 64-key block, so the other block stays zero (block-diagonal P).
-    for (int off = threadIdx.x * 16; off < 2 * C::PB; off += 256 * 16)
-      st_shared_v4(sb + C::OFF_P + off, 0u, 0u, 0u, 0u);
-    fence_async_smem();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns};
 
-  if (warp == 8) {
+  if (warp >= 8) {
+   // Control warpgroup: all four warps shrink their budget at this point.
+   warpgroup_reg_dealloc<kWinControlRegs>();
+   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int it = 0;
@@ -326,41 +294,59 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       for (int j = (it > NS ? it - NS : 0); j < it; ++j)
         wait_drain(in_full(j % NS), (j / NS) & 1, args.timeout_ns);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------- U' scaling + MMA issue
+   } else if (warp == 9) {
+    // --------------------------------------------------- score MMA issue
     bool ok = true;
-    auto do_pv = [&](int j) -> bool {
-      const int a = j & 1, s = j % NS;
-      if (!wait_warp(p_full(a), (j >> 1) & 1, g, 3)) return false;
-      tc_fence_after();
-      issue_pv<D>(tmem + 256 + a * D, sb + C::OFF_P + a * C::PB, sb + s * C::STAGE + 2 * C::QB,
-                  false);
-      umma_commit(o_full(a));
-      umma_commit(in_empty(s));
-      return true;
-    };
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int s = it % NS, a = it & 1;
-      if (!wait_warp(in_full(s), (it / NS) & 1, g, 2)) { ok = false; break; }
-      const uint32_t st = sb + s * C::STAGE;
-      if constexpr (RP > 0) {
-        scale_tile_bf16(st + 3 * C::QB, C::UB, args.inv_scale);
-        fence_async_smem();
-      }
-      __syncwarp();
-      if (it >= 2 && !wait_warp(acc_empty(a), ((it >> 1) + 1) & 1, g, 4)) { ok = false; break; }
+      // Inputs landed (and, with a bias, U' scaled in place).
+      if (!wait_warp(RP > 0 ? u_ready(s) : in_full(s), (it / NS) & 1, g, 2)) { ok = false; break; }
+      // S_a is free once the softmax of tile it - 2 has loaded it.
+      if (it >= 2 && !wait_warp(s_empty(a), ((it >> 1) + 1) & 1, g, 4)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t st = sb + s * C::STAGE;
       issue_scores<D, RP>(tmem + a * 128, st, st + C::QB, st + 3 * C::QB, st + 3 * C::QB + C::UB);
       umma_commit(s_full(a));
-      if (it > 0 && !do_pv(it - 1)) { ok = false; break; }
     }
-    if (ok && it > 0) do_pv(it - 1);
+    (void)ok;
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0, args.timeout_ns);
     __syncwarp();
+   } else if (warp == 10) {
+    // ------------------------------------------------------ PV MMA issue
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int s = it % NS, a = it & 1;
+      if (!wait_warp(p_full(a), (it >> 1) & 1, g, 3)) break;
+      // O_a is free once the epilogue of tile it - 2 has read it.
+      if (it >= 2 && !wait_warp(acc_empty(a), ((it >> 1) + 1) & 1, g, 7)) break;
+      tc_fence_after();
+      issue_pv_ts<D>(tmem + C::T_O + a * D, tmem + C::T_P + a * 64, sb + s * C::STAGE + 2 * C::QB,
+                     false);
+      umma_commit(o_full(a));
+      umma_commit(in_empty(s));
+    }
+    umma_commit(drain_bar);
+    wait_drain(drain_bar, 0, args.timeout_ns);
+    __syncwarp();
+   } else {
+    // ------------------------------------------------- U' = U / s in place
+    if constexpr (RP > 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        const int s = it % NS;
+        if (!wait_warp(in_full(s), (it / NS) & 1, g, 8)) break;
+        scale_tile_bf16(sb + s * C::STAGE + 3 * C::QB, C::UB, args.inv_scale);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(u_ready(s));
+      }
+    }
+   }
   } else {
     // ------------------------------------------------- softmax + epilogue
+    warpgroup_reg_alloc<kWinSoftmaxRegs>();
     // Warpgroup a (= warp / 4) takes the tiles with it % 2 == a, i.e. exactly
     // the tiles that use S, O and P buffer a, so the two warpgroups work on
     // consecutive tiles at the same time.
@@ -369,25 +355,40 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     const int wl = row / NP;            // window inside the tile
     const int n = row % NP;             // token inside the window
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t p_tm = tmem + lane_base + C::T_P + a * 64;
     const int N = args.N;
     const float sl2 = args.scale_log2;
+    // P_a starts at zero: each row only ever writes its own window's block of
+    // NP / 2 columns, so the other blocks stay zero (block-diagonal P).
+    {
+      uint32_t zero[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll
+      for (int c = 0; c < 64; c += 16) tmem_st16_nowait(p_tm + c, zero);
+      tmem_st_wait();
+    }
     int it = a;
     for (int t = blockIdx.x + a * gridDim.x; t < num_tiles; t += 2 * gridDim.x, it += 2) {
       if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) break;
       tc_fence_after();
       uint32_t sv[NP];
       tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
+      tc_fence_before();
+      mbar_arrive(s_empty(a));
       if (N < NP) mask_tail<NP>(sv, N);
       const float m = row_max<NP>(sv) * sl2;
-      const float l = exp_row_to_smem<NP>(sv, sl2, m, sb + C::OFF_P + a * C::PB, row, wl * NP);
-      fence_async_smem();
+      // P_a was last read by PV(it - 2), complete since this warpgroup saw
+      // o_full for that tile.
+      const float l = exp_row_to_tmem<NP>(sv, sl2, m, p_tm + wl * (NP / 2));
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full(a));
       // Epilogue of this tile once its PV has landed.
       if (!wait_warp(o_full(a), (it >> 1) & 1, g, 6)) break;
       tc_fence_after();
       uint32_t ov[D];
-      tmem_ld_cols<D>(tmem + lane_base + 256 + a * D, ov);
+      tmem_ld_cols<D>(tmem + lane_base + C::T_O + a * D, ov);
       tc_fence_before();
       mbar_arrive(acc_empty(a));
       const int win = t * C::NW + wl;

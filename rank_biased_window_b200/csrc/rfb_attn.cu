@@ -146,8 +146,61 @@ CUtensorMapSwizzle swizzle_for(int row_bytes) {
 
 // 3-D bf16 map over a contiguous [BH, N, cols] tensor.  The box is
 // (box_cols, box_rows, box_heads); box_cols may exceed cols (zero fill).
+// Host cache of encoded tensor maps.  A map depends only on the address, the
+// tensor extents and the box, so a hit returns exactly what encoding would;
+// entries are replaced round-robin.
+struct MapCache {
+  struct Entry {
+    const void* ptr;
+    int kind, cols, N, BH, bc, br, bh;
+    CUtensorMap map;
+  };
+  static constexpr int kSize = 64;
+  std::mutex mu;
+  Entry e[kSize];
+  int used = 0, next = 0;
+
+  bool find(const Entry& k, CUtensorMap* out) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const Entry& x = e[i];
+      if (x.ptr == k.ptr && x.kind == k.kind && x.cols == k.cols && x.N == k.N && x.BH == k.BH &&
+          x.bc == k.bc && x.br == k.br && x.bh == k.bh) {
+        *out = x.map;
+        return true;
+      }
+    }
+    return false;
+  }
+  void put(const Entry& k) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < kSize) {
+      e[used++] = k;
+    } else {
+      e[next] = k;
+      next = (next + 1) % kSize;
+    }
+  }
+};
+MapCache g_maps;
+
+int encode_3d_uncached(CUtensorMap* m, const void* ptr, int cols, int N, int BH, int box_cols,
+                       int box_rows, int box_heads);
+
 int encode_3d(CUtensorMap* m, const void* ptr, int cols, int N, int BH, int box_cols, int box_rows,
               int box_heads) {
+  MapCache::Entry k{ptr, 0, cols, N, BH, box_cols, box_rows, box_heads, {}};
+  if (g_maps.find(k, m)) return RFB_OK;
+  const int rc = encode_3d_uncached(m, ptr, cols, N, BH, box_cols, box_rows, box_heads);
+  if (rc == RFB_OK) {
+    k.map = *m;
+    g_maps.put(k);
+  }
+  return rc;
+}
+
+int encode_3d_uncached(CUtensorMap* m, const void* ptr, int cols, int N, int BH, int box_cols,
+                       int box_rows, int box_heads) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return cuda_fail(0, kSiteEncoder);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
@@ -166,7 +219,20 @@ int encode_3d(CUtensorMap* m, const void* ptr, int cols, int N, int BH, int box_
 
 // 3-D fp32 map over the [BH, N, cols] dQ|dU accumulator, box (32, 128, 1),
 // 128-byte swizzle (32 fp32 per row); used for bulk reductions.
+int encode_acc_3d_uncached(CUtensorMap* m, void* ptr, int cols, int N, int BH);
+
 int encode_acc_3d(CUtensorMap* m, void* ptr, int cols, int N, int BH) {
+  MapCache::Entry k{ptr, 1, cols, N, BH, 0, 0, 0, {}};
+  if (g_maps.find(k, m)) return RFB_OK;
+  const int rc = encode_acc_3d_uncached(m, ptr, cols, N, BH);
+  if (rc == RFB_OK) {
+    k.map = *m;
+    g_maps.put(k);
+  }
+  return rc;
+}
+
+int encode_acc_3d_uncached(CUtensorMap* m, void* ptr, int cols, int N, int BH) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return cuda_fail(0, kSiteEncoder);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
