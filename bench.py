@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", choices=("rfb", "reference"), default="rfb")
     ap.add_argument("--workload", default="train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shared-bias", action="store_true",
+                    help="one U, W pair per head shared by all windows; with several "
+                         "ranks dU, dW are all-reduced (NCCL) inside the step")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall seconds of the CPU-baseline sample")
     return ap.parse_args()
@@ -286,6 +289,9 @@ def main():
     rfb.load_library()
 
     x = workload_inputs(wl, with_dout=True)
+    shared = args.shared_bias and wl.r > 0
+    if shared:  # one factor pair per head: the first window's
+        x["u"], x["w"] = x["u"][0].contiguous(), x["w"][0].contiguous()
     g = {k: v.to(dev) for k, v in x.items()}
     B, H, N, d, r = wl.B, wl.H, wl.N, wl.d, wl.r
     s = wl.scale
@@ -293,14 +299,22 @@ def main():
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     grads = (torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"]),
              torch.empty_like(g["u"]), torch.empty_like(g["w"]))
-    ws = torch.empty(rfb.bwd_workspace_size(B, H, N, d, r), dtype=torch.uint8, device=dev)
+    ws_bytes = (rfb.bwd_shared_bias_workspace_size if shared else rfb.bwd_workspace_size)(
+        B, H, N, d, r)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    fwd_fn = rfb.attn_fwd_shared_bias if shared else rfb.attn_fwd
+    bwd_fn = rfb.attn_bwd_shared_bias if shared else rfb.attn_bwd
 
     def step():
-        rfb.attn_fwd(g["q"], g["k"], g["v"], g["u"], g["w"], s, out=o, lse=lse, stream=stream)
+        fwd_fn(g["q"], g["k"], g["v"], g["u"], g["w"], s, out=o, lse=lse, stream=stream)
         if wl.backward:
-            rfb.attn_bwd(g["q"], g["k"], g["v"], g["u"], g["w"], o, lse, g["dout"], s,
-                         workspace=ws, grads=grads, stream=stream)
+            bwd_fn(g["q"], g["k"], g["v"], g["u"], g["w"], o, lse, g["dout"], s,
+                   workspace=ws, grads=grads, stream=stream)
+            if shared and dist is not None:
+                # data-parallel windows: the shared factors' gradients are summed
+                # over the ranks (the method's one exchange step)
+                rfb.allreduce_bias_grads(grads[3], grads[4])
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -434,7 +448,11 @@ def main():
         "data": "synthetic (seeded N(0,1) Q,K,V,dO; N(0,1/r) U,W; bf16)",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r,
                    "global_batch": wl.B * world, "seq_len": wl.N,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "parallelism": (f"data parallel over windows x{world}, dU/dW all-reduced "
+                                   f"(NCCL)" if shared and world > 1 else
+                                   f"replicas x{world}" if world > 1 else "single GPU"),
+                   "bias": ("U, W [H, N, r] shared by all windows" if shared else
+                            "U, W [B, H, N, r] per window and head"),
                    "l2": (f"inputs exceed L2 ({in_bytes / 2**20:.0f} MiB > 126 MiB), no flush"
                           if flush is None else
                           f"inputs {in_bytes / 2**20:.0f} MiB fit in L2: before each step a "

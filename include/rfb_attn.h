@@ -136,6 +136,36 @@ RFB_API int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  void* dq, void* dk, void* dv, void* du, void* dw, int B, int H,
                                  int N, int d, int r, float scale, void* stream);
 
+/*
+ * Shared bias factors: one pair U, W per head, used by every window.
+ * "Rank-Factorized Implicit Neural Bias" (Abstract) produces the bias of a
+ * head from an implicit neural representation of relative positions, the same
+ * for all windows of an image; these entry points take that form.  Window-head
+ * (b, h) uses U[h], W[h]:
+ *     O[b, h] = softmax(s Q[b, h] K[b, h]^T + U[h] W[h]^T) V[b, h].
+ * Arguments, layouts, ownership and errors as in rfb_attn_fwd / rfb_attn_bwd,
+ * except:
+ *   u, w   : [H, N, r] bf16 (NULL allowed iff r == 0).
+ *   du, dw : [H, N, r] bf16 outputs, the sums over the B windows of the
+ *            per-window gradients (dU[h] = sum_b dS[b, h] W[h],
+ *            dW[h] = sum_b dS[b, h]^T U[h]), accumulated in fp32.
+ *   workspace : at least rfb_attn_bwd_shared_bias_workspace_size() bytes
+ *            (adds fp32 [B, H, N, r] for the per-window dW).
+ * With data-parallel windows on several GPUs, each rank passes its own windows
+ * and sums du, dw over the ranks afterwards (an all-reduce); the library
+ * itself makes no collective call.
+ */
+RFB_API int rfb_attn_fwd_shared_bias(const void* q, const void* k, const void* v, const void* u,
+                                     const void* w, void* o, float* lse, int B, int H, int N,
+                                     int d, int r, float scale, void* stream);
+RFB_API size_t rfb_attn_bwd_shared_bias_workspace_size(int B, int H, int N, int d, int r);
+RFB_API int rfb_attn_bwd_shared_bias(const void* q, const void* k, const void* v,
+                                     const void* u, const void* w, const void* o,
+                                     const float* lse, const void* dout, void* dq, void* dk,
+                                     void* dv, void* du, void* dw, void* workspace,
+                                     size_t workspace_bytes, int B, int H, int N, int d, int r,
+                                     float scale, void* stream);
+
 /* Human-readable text for a status code (static storage). */
 RFB_API const char* rfb_strerror(int status);
 

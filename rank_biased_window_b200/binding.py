@@ -33,6 +33,9 @@ SIGNATURES = {
     "rfb_attn_bwd_workspace_size": (_sz, [_i] * 5),
     "rfb_attn_bwd": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
     "rfb_attn_bwd_noalloc": (_i, [_vp] * 6 + [_fp] + [_vp] * 6 + [_i] * 5 + [_f, _vp]),
+    "rfb_attn_fwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_i] * 5 + [_f, _vp]),
+    "rfb_attn_bwd_shared_bias_workspace_size": (_sz, [_i] * 5),
+    "rfb_attn_bwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
     "rfb_strerror": (ctypes.c_char_p, [_i]),
     "rfb_last_device_error": (_i, []),
     "rfb_last_cuda_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
@@ -197,6 +200,93 @@ def attn_bwd(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=None, grads=N
     return dq, dk, dv, du, dw
 
 
+def attn_fwd_shared_bias(q, k, v, u=None, w=None, scale=None, *, out=None, lse=None,
+                         stream=None):
+    """Forward with one bias-factor pair per head shared by all windows:
+    u, w are [H, N, r]; window-head (b, h) uses u[h], w[h]."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = (int(x) for x in q.shape)
+    r = 0 if u is None else int(u.shape[-1])
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_operand(name, t, (B, H, N, d), dev)
+    if r > 0:
+        _check_operand("u", u, (H, N, r), dev)
+        _check_operand("w", w, (H, N, r), dev)
+    else:
+        u = w = None
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_operand("out", o, (B, H, N, d), dev)
+    if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    with _on_device(dev):
+        rc = load_library().rfb_attn_fwd_shared_bias(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, H, N, d, r, s,
+            _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_fwd_shared_bias")
+    return o, l
+
+
+def bwd_shared_bias_workspace_size(B, H, N, d, r) -> int:
+    return int(load_library().rfb_attn_bwd_shared_bias_workspace_size(B, H, N, d, r))
+
+
+def attn_bwd_shared_bias(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=None, grads=None,
+                         stream=None):
+    """dQ, dK, dV ([B, H, N, d]) and dU, dW ([H, N, r], summed over the B
+    windows) for shared bias factors u, w [H, N, r]."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = (int(x) for x in q.shape)
+    r = 0 if u is None else int(u.shape[-1])
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_operand(name, t, (B, H, N, d), dev)
+    if r > 0:
+        _check_operand("u", u, (H, N, r), dev)
+        _check_operand("w", w, (H, N, r), dev)
+    else:
+        u = w = None
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    if grads is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        du = torch.empty_like(u) if r else None
+        dw = torch.empty_like(w) if r else None
+    else:
+        dq, dk, dv, du, dw = grads
+    nbytes = bwd_shared_bias_workspace_size(B, H, N, d, r)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    with _on_device(dev):
+        rc = load_library().rfb_attn_bwd_shared_bias(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, H, N, d, r, s,
+            _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_bwd_shared_bias")
+    return dq, dk, dv, du, dw
+
+
+def allreduce_bias_grads(du, dw, group=None):
+    """Data-parallel windows with shared bias factors: sum each rank's dU, dW
+    (already summed over its own windows) over the ranks of `group`, in fp32,
+    in place.  Every rank must call it, with tensors of the same shapes."""
+    import torch.distributed as dist
+    for t in (du, dw):
+        if t is None:
+            continue
+        acc = t.float()
+        dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
+        t.copy_(acc)
+    return du, dw
+
+
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -291,6 +381,30 @@ class RFBAttention(torch.autograd.Function):
         return dq, dk, dv, du, dw, None
 
 
+class RFBAttentionSharedBias(torch.autograd.Function):
+    """Autograd wrapper for shared factors u, w [H, N, r]."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, u, w, scale):
+        o, lse = attn_fwd_shared_bias(q, k, v, u, w, scale)
+        ctx.save_for_backward(q, k, v, u, w, o, lse)
+        ctx.scale = scale
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, u, w, o, lse = ctx.saved_tensors
+        dq, dk, dv, du, dw = attn_bwd_shared_bias(q, k, v, u, w, o, lse, dout.contiguous(),
+                                                  ctx.scale)
+        return dq, dk, dv, du, dw, None
+
+
 def rfb_attention(q, k, v, u, w, scale=None):
     s = (1.0 / math.sqrt(q.shape[-1])) if scale is None else float(scale)
     return RFBAttention.apply(q, k, v, u, w, s)
+
+
+def rfb_attention_shared_bias(q, k, v, u, w, scale=None):
+    """As rfb_attention with u, w [H, N, r] shared by all windows."""
+    s = (1.0 / math.sqrt(q.shape[-1])) if scale is None else float(scale)
+    return RFBAttentionSharedBias.apply(q, k, v, u, w, s)

@@ -51,9 +51,11 @@ struct BwdArgs {
   __nv_bfloat16* dk;          // [BH, N, D]
   __nv_bfloat16* dv;          // [BH, N, D]
   __nv_bfloat16* du;          // [BH, N, r]
-  __nv_bfloat16* dw;          // [BH, N, r]
+  __nv_bfloat16* dw;          // [BH, N, r]  (per-window factors)
+  float* dw_part;             // [BH, N, r]  fp32 dW of each window-head (shared factors)
   int* err;
   int BH, N, Npad, D, r;
+  int bias_heads;             // BH (per-window factors) or H (shared; bias head = bh % H)
   float scale;       // s
   float scale_log2;  // s log2(e)
   float inv_scale;   // 1/s
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
        t += static_cast<size_t>(gridDim.x) * blockDim.x)
     acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
   // U' = bf16(U / s), staged once here instead of once per (key tile, query tile).
-  const size_t n8 = static_cast<size_t>(a.BH) * a.N * a.r / 8;
+  const size_t n8 = static_cast<size_t>(a.bias_heads) * a.N * a.r / 8;
   for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n8;
        t += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const uint4 v = reinterpret_cast<const uint4*>(a.u)[t];
@@ -130,8 +132,42 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdArgs a) {
     v.w = pack_bf16x2(y.z, y.w);
     if (c < a.D)
       *reinterpret_cast<uint4*>(a.dq + row * a.D + c) = v;
-    else
+    else if (a.bias_heads == a.BH)
       *reinterpret_cast<uint4*>(a.du + row * a.r + (c - a.D)) = v;
+  }
+}
+
+// Shared factors: dU[h] = sum_b dU[b H + h] (from the accumulator's dU columns)
+// and dW[h] = sum_b dW[b H + h] (from the fp32 per-window partials), summed in
+// fp32 over b in order, then rounded to bf16.  One thread per 8 values.
+__global__ void __launch_bounds__(256) bwd_post_shared_kernel(const BwdArgs a) {
+  const int H = a.bias_heads, B = a.BH / a.bias_heads;
+  const int DA = a.D + a.r;
+  const int groups = a.r / 8;
+  const long per_mat = static_cast<long>(H) * a.N * groups;
+  for (long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; t < 2 * per_mat;
+       t += static_cast<long>(gridDim.x) * blockDim.x) {
+    const bool is_w = t >= per_mat;
+    const long tt = is_w ? t - per_mat : t;
+    const long hrow = tt / groups;  // h * N + n
+    const int c = static_cast<int>(tt % groups) * 8;
+    float s[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[e] = 0.f;
+    for (int b = 0; b < B; ++b) {
+      const long row = static_cast<long>(b) * H * a.N + hrow;  // (b H + h) N + n
+      const float* src = is_w ? a.dw_part + row * a.r + c : a.acc + row * DA + a.D + c;
+      const float4 x = reinterpret_cast<const float4*>(src)[0];
+      const float4 y = reinterpret_cast<const float4*>(src)[1];
+      s[0] += x.x; s[1] += x.y; s[2] += x.z; s[3] += x.w;
+      s[4] += y.x; s[5] += y.y; s[6] += y.z; s[7] += y.w;
+    }
+    uint4 v;
+    v.x = pack_bf16x2(s[0], s[1]);
+    v.y = pack_bf16x2(s[2], s[3]);
+    v.z = pack_bf16x2(s[4], s[5]);
+    v.w = pack_bf16x2(s[6], s[7]);
+    *reinterpret_cast<uint4*>((is_w ? a.dw : a.du) + hrow * a.r + c) = v;
   }
 }
 
@@ -273,7 +309,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_expect_tx(kv_full, C::KVB);
       tma_load_3d(sb + C::OFF_K, &mK, kv_full, 0, k0, bh);
       tma_load_3d(sb + C::OFF_V, &mV, kv_full, 0, k0, bh);
-      if constexpr (RP > 0) tma_load_3d(sb + C::OFF_W, &mW, kv_full, 0, k0, bh);
+      if constexpr (RP > 0) tma_load_3d(sb + C::OFF_W, &mW, kv_full, 0, k0, bh % args.bias_heads);
       const float* l2 = args.lse2 + static_cast<size_t>(bh) * args.Npad;
       const float* dv = args.dvec + static_cast<size_t>(bh) * args.Npad;
       int i = 0;
@@ -284,7 +320,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_expect_tx(q_full(s), C::STAGE);
         tma_load_3d(st + C::S_Q, &mQ, q_full(s), 0, i * kTile, bh);
         tma_load_3d(st + C::S_DO, &mDO, q_full(s), 0, i * kTile, bh);
-        if constexpr (RP > 0) tma_load_3d(st + C::S_U, &mU, q_full(s), 0, i * kTile, bh);
+        if constexpr (RP > 0)
+          tma_load_3d(st + C::S_U, &mU, q_full(s), 0, i * kTile, bh % args.bias_heads);
         bulk_load(st + C::S_L2, l2 + i * kTile, 512, q_full(s));
         bulk_load(st + C::S_DV, dv + i * kTile, 512, q_full(s));
       }
@@ -573,7 +610,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if constexpr (RP > 0) {
           uint32_t gw[RP];
           tmem_ld_cols<RP>(tmem + lane_base + C::T_DW, gw);
-          if (key_ok) {
+          if (key_ok && args.dw_part != nullptr) {
+            // Shared factors: this window-head's fp32 dW rows, summed over the
+            // windows afterwards.
+            float4* dst = reinterpret_cast<float4*>(args.dw_part + r0 * args.r);
+            const float f = args.scale;
+#pragma unroll
+            for (int c = 0; c < RP; c += 4)
+              if (c < args.r)
+                dst[c >> 2] = make_float4(__uint_as_float(gw[c]) * f, __uint_as_float(gw[c + 1]) * f,
+                                          __uint_as_float(gw[c + 2]) * f,
+                                          __uint_as_float(gw[c + 3]) * f);
+          } else if (key_ok) {
             uint4* dst = reinterpret_cast<uint4*>(args.dw + r0 * args.r);
             const float f = args.scale;
 #pragma unroll

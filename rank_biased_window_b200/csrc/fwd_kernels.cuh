@@ -40,6 +40,10 @@ struct FwdArgs {
   int* err;          // device error word
   int BH;
   int N;
+  // Heads of the U / W tensors: BH (factors per window and head) or H (one
+  // pair per head, shared by all windows).  Window-head bh uses bias head
+  // bh % bias_heads (bh = b H + h).
+  int bias_heads;
   float scale_log2;  // s * log2(e)
   float inv_scale;   // 1 / s  (U' = bf16(U / s))
   uint64_t timeout_ns;
@@ -286,8 +290,19 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
         tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
         if constexpr (RP > 0) {
-          tma_load_3d(st + 3 * C::QB, &mU, in_full(s), 0, 0, w0);
-          tma_load_3d(st + 3 * C::QB + C::UB, &mW, in_full(s), 0, 0, w0);
+          if (args.bias_heads == args.BH) {
+            tma_load_3d(st + 3 * C::QB, &mU, in_full(s), 0, 0, w0);
+            tma_load_3d(st + 3 * C::QB + C::UB, &mW, in_full(s), 0, 0, w0);
+          } else {
+            // Shared factors: one copy per window (its bias head), since
+            // consecutive windows' bias heads wrap around at H.
+#pragma unroll
+            for (int i = 0; i < C::NW; ++i) {
+              const int z = (w0 + i) % args.bias_heads;
+              tma_load_3d(st + 3 * C::QB + i * (C::UB / C::NW), &mU, in_full(s), 0, 0, z);
+              tma_load_3d(st + 3 * C::QB + C::UB + i * (C::UB / C::NW), &mW, in_full(s), 0, 0, z);
+            }
+          }
         }
       }
       // Let the last copies land before the CTA can exit.
@@ -538,7 +553,8 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         mbar_expect_tx(q_full, 2 * (C::QB + C::UB));
         for (int t = 0; t < 2; ++t) {
           tma_load_3d(q_addr(t), &mQ, q_full, 0, q0 + t * kTile, bh);
-          if constexpr (RP > 0) tma_load_3d(u_addr(t), &mU, q_full, 0, q0 + t * kTile, bh);
+          if constexpr (RP > 0)
+            tma_load_3d(u_addr(t), &mU, q_full, 0, q0 + t * kTile, bh % args.bias_heads);
         }
         for (int j = 0; j < nkv; ++j, ++it) {
           const int s = it % NS;
@@ -550,7 +566,8 @@ __global__ void __launch_bounds__(kLongThreads, 1)
           mbar_expect_tx(kv_full(s), C::STAGE);
           tma_load_3d(st, &mK, kv_full(s), 0, j * kTile, bh);
           tma_load_3d(st + C::QB, &mV, kv_full(s), 0, j * kTile, bh);
-          if constexpr (RP > 0) tma_load_3d(st + 2 * C::QB, &mW, kv_full(s), 0, j * kTile, bh);
+          if constexpr (RP > 0)
+            tma_load_3d(st + 2 * C::QB, &mW, kv_full(s), 0, j * kTile, bh % args.bias_heads);
         }
       }
       // No copy may still be in flight when the CTA exits.

@@ -371,22 +371,27 @@ int dispatch_fwd_rp(int d, int rp, const Maps& m, const FwdArgs& a, int sms, cud
 
 // --------------------------------------------------------------- backward
 struct WsLayout {
-  size_t dvec, lse2, acc, uprime, total;
+  size_t dvec, lse2, acc, uprime, dw_part, total;
   int npad;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-WsLayout ws_layout(int B, int H, int N, int d, int r) {
+// Backward workspace: -D and -LSE log2(e) [BH, Npad] fp32, the fp32 dQ | dU
+// accumulator [BH, N, d + r], U' [bias heads, N, r] bf16 and, for shared
+// factors, the fp32 per-window dW [BH, N, r].
+WsLayout ws_layout(int B, int H, int N, int d, int r, bool shared = false) {
   WsLayout L{};
   const size_t bh = static_cast<size_t>(B) * H;
+  const size_t bias_heads = shared ? static_cast<size_t>(H) : bh;
   L.npad = (N + kTile - 1) / kTile * kTile;
   const size_t vec = align256(bh * L.npad * sizeof(float));
   L.dvec = 0;
   L.lse2 = vec;
   L.acc = 2 * vec;
   L.uprime = L.acc + align256(bh * N * static_cast<size_t>(d + r) * sizeof(float));
-  L.total = L.uprime + align256(bh * N * static_cast<size_t>(r) * 2);
+  L.dw_part = L.uprime + align256(bias_heads * N * static_cast<size_t>(r) * 2);
+  L.total = L.dw_part + (shared ? align256(bh * N * static_cast<size_t>(r) * sizeof(float)) : 0);
   return L;
 }
 
@@ -441,13 +446,12 @@ int noalloc_scratch(void** out) {
 }  // namespace
 }  // namespace rfb
 
-using namespace rfb;
-
-extern "C" {
-
-int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, const void* w,
-                 void* o, float* lse, int B, int H, int N, int d, int r, float scale,
-                 void* stream) {
+namespace rfb {
+namespace {
+// Forward of both entry points; `shared`: U, W are [H, N, r], one pair per head.
+int attn_fwd_impl(const void* q, const void* k, const void* v, const void* u, const void* w,
+                  void* o, float* lse, int B, int H, int N, int d, int r, float scale,
+                  void* stream, bool shared) {
   bool empty = false;
   if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
   if (empty) return RFB_OK;
@@ -469,8 +473,11 @@ int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, con
   int rc = encode_3d(&m.q, q, d, N, BH, d, rows, heads);
   if (!rc) rc = encode_3d(&m.k, k, d, N, BH, d, rows, heads);
   if (!rc) rc = encode_3d(&m.v, v, d, N, BH, d, rows, heads);
-  if (!rc && r > 0) rc = encode_3d(&m.u, u, r, N, BH, rp, rows, heads);
-  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, rp, rows, heads);
+  // Shared factors: [H, N, r], one window's rows per copy.
+  const int bias_heads = shared ? H : BH;
+  const int bias_box = shared ? 1 : heads;
+  if (!rc && r > 0) rc = encode_3d(&m.u, u, r, N, bias_heads, rp, rows, bias_box);
+  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, bias_heads, rp, rows, bias_box);
   if (rc) return rc;
   FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -478,22 +485,23 @@ int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, con
   a.err = dev.err_word;
   a.BH = BH;
   a.N = N;
+  a.bias_heads = bias_heads;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
   a.timeout_ns = kWaitTimeoutNs;
   return dispatch_fwd_rp(d, rp, m, a, dev.sms, static_cast<cudaStream_t>(stream));
 }
+}  // namespace
+}  // namespace rfb
 
-size_t rfb_attn_bwd_workspace_size(int B, int H, int N, int d, int r) {
-  bool empty = false;
-  if (check_shape(B, H, N, d, r, 1.0f, &empty) != RFB_OK || empty) return 0;
-  return ws_layout(B, H, N, d, r).total;
-}
-
-int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, const void* w,
-                 const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                 void* du, void* dw, void* workspace, size_t workspace_bytes, int B, int H,
-                 int N, int d, int r, float scale, void* stream) {
+namespace rfb {
+namespace {
+// Backward of both entry points; `shared`: U, W, dU, dW are [H, N, r] and dU,
+// dW are summed over the B windows.
+int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, const void* w,
+                  const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                  void* dv, void* du, void* dw, void* workspace, size_t workspace_bytes, int B,
+                  int H, int N, int d, int r, float scale, void* stream, bool shared) {
   bool empty = false;
   if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
   if (empty) return RFB_OK;
@@ -505,12 +513,13 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
     if (!aligned16(p)) return RFB_ERR_ALIGNMENT;
   if (r > 0 && (!aligned16(u) || !aligned16(w) || !aligned16(du) || !aligned16(dw)))
     return RFB_ERR_ALIGNMENT;
-  const WsLayout L = ws_layout(B, H, N, d, r);
+  const WsLayout L = ws_layout(B, H, N, d, r, shared);
   if (!workspace || workspace_bytes < L.total) return RFB_ERR_WORKSPACE;
   if (!aligned16(workspace)) return RFB_ERR_ALIGNMENT;
   DeviceInfo dev;
   if (int rc = device_info(&dev)) return rc;
   const int BH = B * H;
+  const int bias_heads = shared ? H : BH;
   const int rp = pad_rank(r);
   Maps m;
   std::memset(&m, 0, sizeof(m));
@@ -522,8 +531,9 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   // The backward stages U' = U / s once (bwd_pre) and tiles that copy.
   // With d = 64 the U' and W tiles are staged 64 columns wide (zero padded), so
   // they sit beside Q and K as one MMA operand each.
-  if (!rc && r > 0) rc = encode_3d(&m.u, ws + L.uprime, r, N, BH, d == 64 ? 64 : rp, kTile, 1);
-  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, BH, d == 64 ? 64 : rp, kTile, 1);
+  if (!rc && r > 0)
+    rc = encode_3d(&m.u, ws + L.uprime, r, N, bias_heads, d == 64 ? 64 : rp, kTile, 1);
+  if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, bias_heads, d == 64 ? 64 : rp, kTile, 1);
   if (!rc) rc = encode_acc_3d(&m.acc, ws + L.acc, d + r, N, BH);
   if (rc) return rc;
   BwdArgs a;
@@ -540,6 +550,8 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.du = static_cast<__nv_bfloat16*>(du);
   a.dw = static_cast<__nv_bfloat16*>(dw);
+  a.dw_part = shared ? reinterpret_cast<float*>(ws + L.dw_part) : nullptr;
+  a.bias_heads = bias_heads;
   a.err = dev.err_word;
   a.BH = BH;
   a.N = N;
@@ -562,8 +574,62 @@ int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, con
   {
     LaunchTimer timer(kIdBwdPost, st);
     bwd_post_kernel<<<grid_for(groups, 256, dev.sms), 256, 0, st>>>(a);
+    if (shared && r > 0) {
+      if ((rc = launch_status())) return rc;
+      const long long sgroups = 2LL * H * N * (r / 8);
+      bwd_post_shared_kernel<<<grid_for(sgroups, 256, dev.sms), 256, 0, st>>>(a);
+    }
   }
   return launch_status();
+}
+}  // namespace
+}  // namespace rfb
+
+using namespace rfb;
+
+extern "C" {
+
+
+int rfb_attn_fwd(const void* q, const void* k, const void* v, const void* u, const void* w,
+                 void* o, float* lse, int B, int H, int N, int d, int r, float scale,
+                 void* stream) {
+  return attn_fwd_impl(q, k, v, u, w, o, lse, B, H, N, d, r, scale, stream, false);
+}
+
+int rfb_attn_fwd_shared_bias(const void* q, const void* k, const void* v, const void* u,
+                             const void* w, void* o, float* lse, int B, int H, int N, int d,
+                             int r, float scale, void* stream) {
+  return attn_fwd_impl(q, k, v, u, w, o, lse, B, H, N, d, r, scale, stream, true);
+}
+
+size_t rfb_attn_bwd_workspace_size(int B, int H, int N, int d, int r) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, r, 1.0f, &empty) != RFB_OK || empty) return 0;
+  return ws_layout(B, H, N, d, r).total;
+}
+
+
+int rfb_attn_bwd(const void* q, const void* k, const void* v, const void* u, const void* w,
+                 const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                 void* du, void* dw, void* workspace, size_t workspace_bytes, int B, int H,
+                 int N, int d, int r, float scale, void* stream) {
+  return attn_bwd_impl(q, k, v, u, w, o, lse, dout, dq, dk, dv, du, dw, workspace,
+                       workspace_bytes, B, H, N, d, r, scale, stream, false);
+}
+
+size_t rfb_attn_bwd_shared_bias_workspace_size(int B, int H, int N, int d, int r) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, r, 1.0f, &empty) != RFB_OK || empty) return 0;
+  return ws_layout(B, H, N, d, r, true).total;
+}
+
+int rfb_attn_bwd_shared_bias(const void* q, const void* k, const void* v, const void* u,
+                             const void* w, const void* o, const float* lse, const void* dout,
+                             void* dq, void* dk, void* dv, void* du, void* dw, void* workspace,
+                             size_t workspace_bytes, int B, int H, int N, int d, int r,
+                             float scale, void* stream) {
+  return attn_bwd_impl(q, k, v, u, w, o, lse, dout, dq, dk, dv, du, dw, workspace,
+                       workspace_bytes, B, H, N, d, r, scale, stream, true);
 }
 
 int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* u,

@@ -74,6 +74,24 @@ def test_workspace_size(rfb_lib):
     assert need <= ws < need + 2 * B * H * 128 * 4 + 1024
 
 
+def test_shared_bias_host_checks_and_workspace(rfb_lib):
+    lib = rfb_lib.load_library()
+    n = None
+    assert lib.rfb_attn_fwd_shared_bias(n, n, n, n, n, n, n, 0, 4, 64, 32, 8, 0.1, n) == 0
+    assert lib.rfb_attn_fwd_shared_bias(n, n, n, n, n, n, n, 1, 1, 64, 32, 7, 0.1, n) == 2
+    assert lib.rfb_attn_fwd_shared_bias(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, 0.1, n) == 1
+    assert lib.rfb_attn_fwd_shared_bias(n, n, n, n, n, n, n, 1, 1, 64, 32, 8, 0.0, n) == 1
+    assert lib.rfb_attn_bwd_shared_bias(*([n] * 6 + [n] + [n] * 7 + [0, 1, 1, 64, 48, 8, 0.1, n])) == 2
+    assert lib.rfb_attn_bwd_shared_bias_workspace_size(0, 1, 64, 32, 8) == 0
+    B, H, N, d, r = 4, 8, 4096, 64, 32
+    ws = lib.rfb_attn_bwd_shared_bias_workspace_size(B, H, N, d, r)
+    # as the per-window layout, but U' holds one copy per head (H, not B H)
+    # and the per-window fp32 dW is added
+    need = (B * H * N * (d + r) * 4 + 2 * B * H * N * 4 + H * N * r * 2
+            + B * H * N * r * 4)
+    assert need <= ws < need + 2 * B * H * 128 * 4 + 2048
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     from rank_biased_window_b200 import binding
     # a fresh loader pointed at a missing file must raise, never fall back

@@ -1,8 +1,9 @@
-"""The multi-GPU path of bench.py on CPU: two `gloo` ranks exercise the
-cross-rank timing reduction (max over ranks) and the whole-job throughput, and
-the reference arm's rank > 0 exits without work.  The per-rank work itself is
-independent (weak scaling, no data-path collective), so nothing else crosses
-ranks."""
+"""The multi-GPU paths on CPU: two `gloo` ranks exercise bench.py's
+cross-rank timing reduction (max over ranks) and the whole-job throughput, the
+reference arm's rank > 0 exiting without work, and, for bias factors shared
+by all windows, the all-reduce that sums each rank's dU, dW over the ranks
+(the one data-path exchange; with per-window factors the ranks' work is
+independent)."""
 import os
 import socket
 
@@ -67,3 +68,64 @@ def test_reference_arm_nonzero_rank_exits_without_work(monkeypatch, capsys):
         steps, warmup, gpus = 1, 0, 2
     assert bench.run_reference(A(), WORKLOADS["train"], rank=1) == 0
     assert capsys.readouterr().out == ""
+
+
+def _dp_worker(rank, world, port, q):
+    """Data-parallel windows with shared bias factors: each rank holds half of
+    the windows, computes its windows' dU, dW (the fp64 oracle stands in for
+    the kernels on CPU) and sums them over the ranks with the package's
+    all-reduce helper."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from rank_biased_window_b200 import allreduce_bias_grads
+    from rank_biased_window_b200.inputs import make_inputs, to_f64
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H, N, d, r = 4, 2, 24, 8, 8
+        x = make_inputs(B, H, N, d, r, seed=123, with_dout=True)
+        f = {k: to_f64(v) for k, v in x.items()}
+        u = np.broadcast_to(f["u"][0][None], (B, H, N, r)).copy()   # shared factors
+        w = np.broadcast_to(f["w"][0][None], (B, H, N, r)).copy()
+        lo, hi = rank * B // world, (rank + 1) * B // world           # this rank's windows
+        _, _, _, du, dw = oracle.bwd(f["q"][lo:hi], f["k"][lo:hi], f["v"][lo:hi], u[lo:hi],
+                                     w[lo:hi], f["dout"][lo:hi], 0.35)
+        du_t = torch.from_numpy(du.sum(axis=0))
+        dw_t = torch.from_numpy(dw.sum(axis=0))
+        allreduce_bias_grads(du_t, dw_t)
+        q.put((rank, du_t.numpy(), dw_t.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shared_bias_gradients_all_reduced_over_two_gloo_ranks():
+    import numpy as np
+    import sys
+    sys.path.insert(0, ROOT)
+    import oracle
+    from rank_biased_window_b200.inputs import make_inputs, to_f64
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_dp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    B, H, N, d, r = 4, 2, 24, 8, 8
+    x = make_inputs(B, H, N, d, r, seed=123, with_dout=True)
+    f = {k: to_f64(v) for k, v in x.items()}
+    u = np.broadcast_to(f["u"][0][None], (B, H, N, r)).copy()
+    w = np.broadcast_to(f["w"][0][None], (B, H, N, r)).copy()
+    _, _, _, du, dw = oracle.bwd(f["q"], f["k"], f["v"], u, w, f["dout"], 0.35)
+    for _, du_r, dw_r in got:   # every rank ends with the sum over all windows
+        np.testing.assert_allclose(du_r, du.sum(axis=0), rtol=1e-5, atol=1e-6)
+        np.testing.assert_allclose(dw_r, dw.sum(axis=0), rtol=1e-5, atol=1e-6)
