@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", choices=("rfb", "reference"), default="rfb")
     ap.add_argument("--workload", default="train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense-bias", action="store_true",
+                    help="materialised-bias comparator: forward with the bias given as a "
+                         "dense bf16 [H, N, N] matrix (U[h] W[h]^T), forward only")
     ap.add_argument("--shared-bias", action="store_true",
                     help="one U, W pair per head shared by all windows; with several "
                          "ranks dU, dW are all-reduced (NCCL) inside the step")
@@ -289,7 +292,8 @@ def main():
     rfb.load_library()
 
     x = workload_inputs(wl, with_dout=True)
-    shared = args.shared_bias and wl.r > 0
+    shared = (args.shared_bias or args.dense_bias) and wl.r > 0
+    dense = args.dense_bias
     if shared:  # one factor pair per head: the first window's
         x["u"], x["w"] = x["u"][0].contiguous(), x["w"][0].contiguous()
     g = {k: v.to(dev) for k, v in x.items()}
@@ -305,8 +309,16 @@ def main():
     stream = torch.cuda.current_stream(dev)
     fwd_fn = rfb.attn_fwd_shared_bias if shared else rfb.attn_fwd
     bwd_fn = rfb.attn_bwd_shared_bias if shared else rfb.attn_bwd
+    dense_bias = None
+    if dense:  # the comparator's input: U[h] W[h]^T materialised once, outside timing
+        dense_bias = torch.einsum("hnr,hmr->hnm", g["u"].float(), g["w"].float()).to(
+            torch.bfloat16).contiguous()
 
     def step():
+        if dense:
+            rfb.attn_fwd_dense_bias(g["q"], g["k"], g["v"], dense_bias, s, out=o, lse=lse,
+                                    stream=stream)
+            return
         fwd_fn(g["q"], g["k"], g["v"], g["u"], g["w"], s, out=o, lse=lse, stream=stream)
         if wl.backward:
             bwd_fn(g["q"], g["k"], g["v"], g["u"], g["w"], o, lse, g["dout"], s,
@@ -365,12 +377,19 @@ def main():
         raise RuntimeError(f"device error word {err:#x} after the timed region")
 
     # ---- end-to-end through the public API with pinned host buffers
-    host_in = {k: v.pin_memory() for k, v in x.items()}
+    with_grads = wl.backward and not dense
+    if dense:  # the comparator's inputs include the dense bias itself
+        x["bias"] = dense_bias.cpu()
+        g["bias"] = dense_bias
+    used = ("q", "k", "v", "bias") if dense else \
+        (("q", "k", "v", "u", "w", "dout") if with_grads else ("q", "k", "v", "u", "w"))
+    host_in = {k: x[k].pin_memory() for k in used}
     host_out = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
                 "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
     names = ("dq", "dk", "dv", "du", "dw")
-    for n_, t_ in zip(names, grads):
-        host_out[n_] = torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True)
+    if with_grads:
+        for n_, t_ in zip(names, grads):
+            host_out[n_] = torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
 
@@ -380,8 +399,9 @@ def main():
         step()
         host_out["o"].copy_(o, non_blocking=True)
         host_out["lse"].copy_(lse, non_blocking=True)
-        for n_, t_ in zip(names, grads):
-            host_out[n_].copy_(t_, non_blocking=True)
+        if with_grads:
+            for n_, t_ in zip(names, grads):
+                host_out[n_].copy_(t_, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 10))
     e2e_step()
@@ -400,6 +420,11 @@ def main():
     ms_total, ms_e2e_total = max_over_ranks([ms_total, ms_e2e_total], dist, dev)
 
     fwd_f, bwd_f, fwd_b, bwd_b = work(wl)
+    if dense:
+        # forward only; counted with the factored forward's algorithmic flops for
+        # the same attention, so the two lines compare directly
+        bwd_f = 0.0
+        fwd_b += wl.H * wl.N * wl.N * 2  # the dense bias read once
     step_flops = fwd_f + bwd_f
     ms_step = ms_total / args.steps
     value = throughput_tflops(step_flops, world, ms_step)
@@ -451,7 +476,9 @@ def main():
                    "parallelism": (f"data parallel over windows x{world}, dU/dW all-reduced "
                                    f"(NCCL)" if shared and world > 1 else
                                    f"replicas x{world}" if world > 1 else "single GPU"),
-                   "bias": ("U, W [H, N, r] shared by all windows" if shared else
+                   "bias": ("dense [H, N, N] bf16 = U[h] W[h]^T (materialised-bias "
+                            "comparator, forward only)" if dense else
+                            "U, W [H, N, r] shared by all windows" if shared else
                             "U, W [B, H, N, r] per window and head"),
                    "l2": (f"inputs exceed L2 ({in_bytes / 2**20:.0f} MiB > 126 MiB), no flush"
                           if flush is None else

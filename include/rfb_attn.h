@@ -166,6 +166,26 @@ RFB_API int rfb_attn_bwd_shared_bias(const void* q, const void* k, const void* v
                                      size_t workspace_bytes, int B, int H, int N, int d, int r,
                                      float scale, void* stream);
 
+/*
+ * Materialised-bias comparator (not the method): the same attention with the
+ * bias given as a dense bf16 matrix per head,
+ *     O[b, h] = softmax(s Q[b, h] K[b, h]^T + bias[z]) V[b, h],
+ *     z = h (bias_heads == H, one matrix per head shared by all windows) or
+ *     z = b H + h (bias_heads == B H),
+ * i.e. the conventional form whose N x N read the rank-factorised bias avoids
+ * ("FlashBias: Fast Computation of Attention with Bias", Abstract: low-rank
+ * bias keeps attention fast where a materialised bias slows it down).  Forward
+ * only; used to measure that difference on this hardware.
+ *   bias : [bias_heads, N, N] bf16, row i holding the bias of query i.
+ *   q, k, v, o, lse, scale, stream : as rfb_attn_fwd (r = 0).
+ * Errors as rfb_attn_fwd; RFB_ERR_INVALID_ARG if bias_heads is neither H nor
+ * B*H; RFB_ERR_UNSUPPORTED if N is not a multiple of 8 (bias rows must be
+ * whole 16-byte units for the copy engine).
+ */
+RFB_API int rfb_attn_fwd_dense_bias(const void* q, const void* k, const void* v, const void* bias,
+                                    void* o, float* lse, int B, int H, int N, int d,
+                                    int bias_heads, float scale, void* stream);
+
 /* Human-readable text for a status code (static storage). */
 RFB_API const char* rfb_strerror(int status);
 

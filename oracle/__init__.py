@@ -218,3 +218,32 @@ def bwd_query_rows(q, k, v, u, w, dout, scale, bh, rows, *, nthreads: int = 0):
     if rc != 0:
         raise RuntimeError(f"oracle bwd_query_rows failed ({rc})")
     return dq, du, D
+
+
+def fwd_dense_bias(q, k, v, bias, scale):
+    """Forward with the bias given as a dense matrix (the materialised form the
+    rank-factorised bias replaces; "FlashBias: Fast Computation of Attention
+    with Bias", Abstract).  ``bias`` is ``[H, N, N]`` (one matrix per head,
+    used by every window) or ``[B, H, N, N]``.  Per batch-head, in float64::
+
+        S = s * Q @ K.T + Bias;  m = max_j S;  P = exp(S - m) / sum_j exp(S - m)
+        O = P @ V;  LSE = m + log(sum_j exp(S - m))
+
+    Returns ``(O, LSE)`` shaped ``[B, H, N, d]`` and ``[B, H, N]``.  Pinned in
+    ``tests/test_oracle_dense_bias.py`` against the factored oracle (``fwd``)
+    with ``Bias = U W^T``."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    bias = np.asarray(bias, dtype=np.float64)
+    B, H, N, d = q.shape
+    O = np.empty((B, H, N, d))
+    L = np.empty((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            bm = bias[h] if bias.ndim == 3 else bias[b, h]
+            S = scale * (q[b, h] @ k[b, h].T) + bm
+            m = S.max(axis=1, keepdims=True)
+            E = np.exp(S - m)
+            l = E.sum(axis=1, keepdims=True)
+            O[b, h] = (E @ v[b, h]) / l
+            L[b, h] = (m + np.log(l))[:, 0]
+    return O, L

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     attn_bwd_noalloc,
     attn_bwd_shared_bias,
     attn_fwd,
+    attn_fwd_dense_bias,
     attn_fwd_shared_bias,
     bwd_shared_bias_workspace_size,
     bwd_workspace_size,
@@ -28,6 +29,6 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "bwd_workspace_size", "rfb_attention", "RFBAttention",
-           "attn_fwd_shared_bias", "attn_bwd_shared_bias", "bwd_shared_bias_workspace_size",
+           "attn_fwd_shared_bias", "attn_fwd_dense_bias", "attn_bwd_shared_bias", "bwd_shared_bias_workspace_size",
            "rfb_attention_shared_bias", "RFBAttentionSharedBias", "allreduce_bias_grads",
            "last_device_error", "selftest_wait_timeout", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]

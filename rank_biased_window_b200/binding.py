@@ -35,6 +35,7 @@ SIGNATURES = {
     "rfb_attn_bwd_noalloc": (_i, [_vp] * 6 + [_fp] + [_vp] * 6 + [_i] * 5 + [_f, _vp]),
     "rfb_attn_fwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_i] * 5 + [_f, _vp]),
     "rfb_attn_bwd_shared_bias_workspace_size": (_sz, [_i] * 5),
+    "rfb_attn_fwd_dense_bias": (_i, [_vp] * 5 + [_fp] + [_i] * 5 + [_f, _vp]),
     "rfb_attn_bwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
     "rfb_strerror": (ctypes.c_char_p, [_i]),
     "rfb_last_device_error": (_i, []),
@@ -228,6 +229,37 @@ def attn_fwd_shared_bias(q, k, v, u=None, w=None, scale=None, *, out=None, lse=N
             ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, H, N, d, r, s,
             _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_fwd_shared_bias")
+    return o, l
+
+
+def attn_fwd_dense_bias(q, k, v, bias, scale=None, *, out=None, lse=None, stream=None):
+    """Materialised-bias comparator: O = softmax(s Q K^T + bias) V with a dense
+    bf16 bias, [H, N, N] (shared by the windows) or [B, H, N, N]."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = (int(x) for x in q.shape)
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_operand(name, t, (B, H, N, d), dev)
+    if tuple(bias.shape) == (H, N, N):
+        bias_heads = H
+    elif tuple(bias.shape) == (B, H, N, N):
+        bias_heads = B * H
+    else:
+        raise ValueError(f"bias must be [H, N, N] or [B, H, N, N], got {tuple(bias.shape)}")
+    _check_operand("bias", bias, tuple(bias.shape), dev)
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_operand("out", o, (B, H, N, d), dev)
+    if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    with _on_device(dev):
+        rc = load_library().rfb_attn_fwd_dense_bias(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, H, N, d, bias_heads, s,
+            _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_fwd_dense_bias")
     return o, l
 
 

@@ -33,6 +33,7 @@ namespace rfb {
 
 constexpr int kTile = 128;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2eF = 1.4426950408889634f;
 
 struct FwdArgs {
   __nv_bfloat16* o;  // [BH, N, D]
@@ -44,6 +45,12 @@ struct FwdArgs {
   // pair per head, shared by all windows).  Window-head bh uses bias head
   // bh % bias_heads (bh = b H + h).
   int bias_heads;
+  // Window kernel: how U / W reach shared memory.  kBiasTile: one copy per
+  // tile (per-window factors); kBiasWindow: one copy per window (shared
+  // factors); kBiasResident: all bias heads loaded once per CTA (shared
+  // factors that fit), followed by copies of heads 0 .. NW-2 so that any NW
+  // consecutive windows' heads are contiguous.
+  int bias_mode;
   float scale_log2;  // s * log2(e)
   float inv_scale;   // 1 / s  (U' = bf16(U / s))
   uint64_t timeout_ns;
@@ -182,6 +189,8 @@ __device__ __forceinline__ void issue_pv_ts(uint32_t o_tmem, uint32_t p_tmem, ui
 }
 
 // ============================================================ window regime
+constexpr int kBiasTile = 0, kBiasWindow = 1, kBiasResident = 2;
+
 template <int D, int RP, int NP>
 struct WinCfg {
   static constexpr int NW = kTile / NP;       // windows packed per tile
@@ -194,9 +203,13 @@ struct WinCfg {
   // TMEM columns: S_a at 128 a, O_a at 256 + D a, P_a (packed bf16) at 384 + 64 a.
   static constexpr int T_O = 256, T_P = 384;
   // in_full[NS] u_ready[NS] in_empty[NS] s_full[2] s_empty[2] p_full[2] o_full[2]
-  // acc_empty[2] drain
-  static constexpr int NBAR = 3 * NS + 11;
+  // acc_empty[2] drain res_full res_ready
+  static constexpr int NBAR = 3 * NS + 13;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  // Resident shared factors start after the barriers; one head's U or W rows.
+  static constexpr int OFF_RES = (OFF_BAR + NBAR * 8 + 16 + 1023) / 1024 * 1024;
+  static constexpr int HB = NP * RP * 2;
+  static constexpr int res_bytes(int heads) { return 2 * (heads + NW - 1) * HB; }
   static_assert(NS >= 2, "not enough shared memory for two input stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
   static_assert(QB % 1024 == 0 && UB % 1024 == 0, "tile alignment");
@@ -230,6 +243,11 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   auto o_full = [&](int a) { return bar0 + 8u * (3 * NS + 6 + a); };
   auto acc_empty = [&](int a) { return bar0 + 8u * (3 * NS + 8 + a); };
   const uint32_t drain_bar = bar0 + 8u * (3 * NS + 10);
+  const uint32_t res_full = bar0 + 8u * (3 * NS + 11);   // resident factors landed
+  const uint32_t res_ready = bar0 + 8u * (3 * NS + 12);  // resident U' scaled
+  const bool resident = RP > 0 && args.bias_mode == kBiasResident;
+  const int res_heads = args.bias_heads + C::NW - 1;
+  const uint32_t res_u = sb + C::OFF_RES, res_w = res_u + res_heads * C::HB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -252,6 +270,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       mbar_init(acc_empty(a), 128);
     }
     mbar_init(drain_bar, 2);
+    mbar_init(res_full, 1);
+    mbar_init(res_ready, 8);  // one arrival per softmax warp
     fence_mbar_init();
   }
   if (warp == 8 && lane == 0) {
@@ -279,18 +299,30 @@ __global__ void __launch_bounds__(kWinThreads, 1)
    if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      if (resident) {
+        // Every bias head once (head hh % H at slot hh), for the whole kernel.
+        mbar_expect_tx(res_full, C::res_bytes(args.bias_heads));
+        for (int hh = 0; hh < res_heads; ++hh) {
+          const int z = hh % args.bias_heads;
+          tma_load_3d(res_u + hh * C::HB, &mU, res_full, 0, 0, z);
+          tma_load_3d(res_w + hh * C::HB, &mW, res_full, 0, 0, z);
+        }
+      }
+      const uint32_t stage_tx = resident ? 3 * C::QB : C::STAGE;
       int it = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
         const int s = it % NS;
         if (it >= NS && !wait_bounded(in_empty(s), ((it / NS) + 1) & 1, g, 1)) break;
         const uint32_t st = sb + s * C::STAGE;
-        mbar_expect_tx(in_full(s), C::STAGE);
+        mbar_expect_tx(in_full(s), stage_tx);
         const int w0 = t * C::NW;
         tma_load_3d(st, &mQ, in_full(s), 0, 0, w0);
         tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
         tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
         if constexpr (RP > 0) {
-          if (args.bias_heads == args.BH) {
+          if (resident) {
+            // factors already resident
+          } else if (args.bias_mode == kBiasTile) {
             tma_load_3d(st + 3 * C::QB, &mU, in_full(s), 0, 0, w0);
             tma_load_3d(st + 3 * C::QB + C::UB, &mW, in_full(s), 0, 0, w0);
           } else {
@@ -306,22 +338,29 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         }
       }
       // Let the last copies land before the CTA can exit.
+      if (resident) wait_drain(res_full, 0, args.timeout_ns);
       for (int j = (it > NS ? it - NS : 0); j < it; ++j)
         wait_drain(in_full(j % NS), (j / NS) & 1, args.timeout_ns);
     }
    } else if (warp == 9) {
     // --------------------------------------------------- score MMA issue
     bool ok = true;
+    if (resident) ok = wait_warp(res_ready, 0, g, 9);
     int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, ++it) {
       const int s = it % NS, a = it & 1;
-      // Inputs landed (and, with a bias, U' scaled in place).
-      if (!wait_warp(RP > 0 ? u_ready(s) : in_full(s), (it / NS) & 1, g, 2)) { ok = false; break; }
+      // Inputs landed (and, with per-tile factors, U' scaled in place).
+      const uint32_t ready = (RP > 0 && !resident) ? u_ready(s) : in_full(s);
+      if (!wait_warp(ready, (it / NS) & 1, g, 2)) { ok = false; break; }
       // S_a is free once the softmax of tile it - 2 has loaded it.
       if (it >= 2 && !wait_warp(s_empty(a), ((it >> 1) + 1) & 1, g, 4)) { ok = false; break; }
       tc_fence_after();
       const uint32_t st = sb + s * C::STAGE;
-      issue_scores<D, RP>(tmem + a * 128, st, st + C::QB, st + 3 * C::QB, st + 3 * C::QB + C::UB);
+      // Resident factors: the NW windows' heads are contiguous from head w0 % H.
+      const uint32_t hoff = resident ? ((t * C::NW) % args.bias_heads) * C::HB : 0u;
+      const uint32_t ua = resident ? res_u + hoff : st + 3 * C::QB;
+      const uint32_t wa = resident ? res_w + hoff : st + 3 * C::QB + C::UB;
+      issue_scores<D, RP>(tmem + a * 128, st, st + C::QB, ua, wa);
       umma_commit(s_full(a));
     }
     (void)ok;
@@ -347,7 +386,10 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     __syncwarp();
    } else {
     // ------------------------------------------------- U' = U / s in place
-    if constexpr (RP > 0) {
+    if (RP > 0 && resident) {
+      // The softmax warpgroups scale the resident U (they are idle until the
+      // first scores).
+    } else if constexpr (RP > 0) {
       int it = 0;
       for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
         const int s = it % NS;
@@ -373,6 +415,24 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     const uint32_t p_tm = tmem + lane_base + C::T_P + a * 64;
     const int N = args.N;
     const float sl2 = args.scale_log2;
+    if (resident) {
+      // U' = U / s for the resident factors, 16 bytes per thread per step.
+      if (wait_warp(res_full, 0, g, 10)) {
+        const uint32_t bytes = res_heads * C::HB;
+        for (uint32_t off = threadIdx.x * 16u; off < bytes; off += 256u * 16u) {
+          uint4 v = ld_shared_v4(res_u + off);
+          uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            wv[e] = pack_bf16x2(__uint_as_float(wv[e] << 16) * args.inv_scale,
+                                __uint_as_float(wv[e] & 0xFFFF0000u) * args.inv_scale);
+          st_shared_v4(res_u + off, wv[0], wv[1], wv[2], wv[3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(res_ready);
+      }
+    }
     // P_a starts at zero: each row only ever writes its own window's block of
     // NP / 2 columns, so the other blocks stay zero (block-diagonal P).
     {
@@ -424,11 +484,17 @@ __global__ void __launch_bounds__(kWinThreads, 1)
 }
 
 // ============================================================== long regime
-template <int D, int RP>
+// DENSE: the materialised-bias comparator (no factors; each K/V stage also
+// holds the two query tiles' 128 x 128 bf16 bias tiles, each as two 64-column
+// 128-byte-swizzled halves).
+template <int D, int RP, bool DENSE = false>
 struct LongCfg {
+  static_assert(!DENSE || RP == 0, "the dense-bias comparator takes no factors");
   static constexpr int QB = kTile * D * 2;
   static constexpr int UB = kTile * RP * 2;
-  static constexpr int STAGE = 2 * QB + UB;  // K, V, W
+  static constexpr int BT = DENSE ? kTile * kTile * 2 : 0;  // one query tile's bias tile
+  static constexpr int OFF_BIAS = 2 * QB + UB;                // within a stage
+  static constexpr int STAGE = 2 * QB + UB + 2 * BT;        // K, V, W, bias tiles
   // Two query tiles per CTA: Q0 U0 Q1 U1, then the KV stages.  P lives in TMEM.
   static constexpr int OFF_Q = 0;            // Q tile t at OFF_Q + t * (QB + UB), U right after
   static constexpr int OFF_STAGE = 2 * (QB + UB);
@@ -465,12 +531,14 @@ constexpr int kLongSoftPairs = 1;
 // the other's loads, maxima and waits, and each K/V tile serves 256 query rows.
 // Barrier phases run on across units, so the K/V loads and the scores of the
 // next unit start while the current unit's last tiles and epilogue finish.
-template <int D, int RP>
+// With DENSE (the comparator) mU is the map of the dense bias [bias heads, N,
+// N] (box 64 x 128) and mW is unused.
+template <int D, int RP, bool DENSE = false>
 __global__ void __launch_bounds__(kLongThreads, 1)
     fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
                     const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
-  using C = LongCfg<D, RP>;
+  using C = LongCfg<D, RP, DENSE>;
   constexpr int NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
@@ -525,10 +593,8 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     tma_prefetch(&mQ);
     tma_prefetch(&mK);
     tma_prefetch(&mV);
-    if constexpr (RP > 0) {
-      tma_prefetch(&mU);
-      tma_prefetch(&mW);
-    }
+    if constexpr (RP > 0 || DENSE) tma_prefetch(&mU);
+    if constexpr (RP > 0) tma_prefetch(&mW);
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -568,6 +634,16 @@ __global__ void __launch_bounds__(kLongThreads, 1)
           tma_load_3d(st + C::QB, &mV, kv_full(s), 0, j * kTile, bh);
           if constexpr (RP > 0)
             tma_load_3d(st + 2 * C::QB, &mW, kv_full(s), 0, j * kTile, bh % args.bias_heads);
+          if constexpr (DENSE) {
+            // bias[q0 + 128 t + row, 128 j + col] for both query tiles, in two
+            // 64-column halves each
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d(st + C::OFF_BIAS + t * C::BT + c * (C::BT / 2), &mU, kv_full(s),
+                            j * kTile + c * 64, q0 + t * kTile, bh % args.bias_heads);
+          }
         }
       }
       // No copy may still be in flight when the CTA exits.
@@ -635,8 +711,10 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     const uint32_t s_tm = tmem + lane_base + t * 128;
     const uint32_t o_tm = tmem + lane_base + C::T_O + t * D;
     const uint32_t p_tm = tmem + lane_base + C::T_P + t * 64;
-    const float sl2 = args.scale_log2;
-    int jt = 0;  // S tiles of this query tile so far
+    // Scores are accumulator * sl2 in log2 units; the comparator adds its bias
+    // to the scaled scores first and then uses a unit factor.
+    const float sl2 = DENSE ? 1.0f : args.scale_log2;
+    int jt = 0;  // S tiles of this query tile so far (= K/V tiles of the CTA)
     bool ok = true;
     for (int u = first; ok && u < nunits; u += stride) {
       const int bh = u / npairs, q0 = (u % npairs) * 2 * kTile;
@@ -648,6 +726,28 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         tmem_ld_cols<128>(s_tm, sv);
         tc_fence_before();
         mbar_arrive(s_empty(t));
+        if constexpr (DENSE) {
+          // s_j = acc_j s log2(e) + bias_j log2(e), the bias row from this K/V
+          // tile's stage (its copy is awaited here too; it landed with K / V).
+          const int s = jt % NS;
+          if (!wait_warp(kv_full(s), (jt / NS) & 1, g, 20)) { ok = false; break; }
+          const uint32_t bt = sb + C::OFF_STAGE + s * C::STAGE + C::OFF_BIAS + t * C::BT;
+          const float sl = args.scale_log2;
+#pragma unroll
+          for (int c = 0; c < 128; c += 8) {
+            const uint4 bv = ld_shared_v4(bt + (c >> 6) * (C::BT / 2) + row * 128 +
+                                          ((((c & 63) >> 3) ^ (row & 7)) << 4));
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              sv[c + 2 * e] = __float_as_uint(fmaf(__uint_as_float(sv[c + 2 * e]), sl,
+                                                   __uint_as_float(bw[e] << 16) * kLog2eF));
+              sv[c + 2 * e + 1] = __float_as_uint(
+                  fmaf(__uint_as_float(sv[c + 2 * e + 1]), sl,
+                       __uint_as_float(bw[e] & 0xFFFF0000u) * kLog2eF));
+            }
+          }
+        }
         const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
         if (kvalid < kTile) mask_tail<128>(sv, kvalid);
         const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);

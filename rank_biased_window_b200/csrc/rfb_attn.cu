@@ -332,11 +332,24 @@ template <int D, int RP, int NP>
 int launch_window(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   using C = WinCfg<D, RP, NP>;
   static std::atomic<uint64_t> done{0};
-  if (int rc = ensure_smem(fwd_window_kernel<D, RP, NP>, C::SMEM, done)) return rc;
+  constexpr int kMaxSmem = 232448;
+  if (int rc = ensure_smem(fwd_window_kernel<D, RP, NP>, kMaxSmem, done)) return rc;
   const int tiles = (a.BH + C::NW - 1) / C::NW;
   const int grid = tiles < sms ? tiles : sms;
+  FwdArgs args = a;
+  int smem = C::SMEM;
+  if (RP > 0 && args.bias_mode == kBiasWindow) {
+    // Shared factors: keep every head resident in shared memory when they fit
+    // beside the input ring (every CTA would otherwise re-read the same few
+    // lines of U and W for each tile).
+    const long long need = C::OFF_RES + static_cast<long long>(C::res_bytes(args.bias_heads)) + 1024;
+    if (need <= kMaxSmem) {
+      args.bias_mode = kBiasResident;
+      smem = static_cast<int>(need);
+    }
+  }
   LaunchTimer timer(kIdFwd, st);
-  fwd_window_kernel<D, RP, NP><<<grid, kWinThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  fwd_window_kernel<D, RP, NP><<<grid, kWinThreads, smem, st>>>(m.q, m.k, m.v, m.u, m.w, args);
   return launch_status();
 }
 
@@ -350,6 +363,19 @@ int launch_long(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
   LaunchTimer timer(kIdFwd, st);
   fwd_long_kernel<D, RP><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  return launch_status();
+}
+
+// The materialised-bias comparator (long kernel, DENSE).
+template <int D>
+int launch_long_dense(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
+  using C = LongCfg<D, 0, true>;
+  static std::atomic<uint64_t> done{0};
+  if (int rc = ensure_smem(fwd_long_kernel<D, 0, true>, C::SMEM, done)) return rc;
+  const long long units = static_cast<long long>((a.N + 2 * kTile - 1) / (2 * kTile)) * a.BH;
+  const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
+  LaunchTimer timer(kIdFwd, st);
+  fwd_long_kernel<D, 0, true><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
 }
 
@@ -486,6 +512,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const void* u, co
   a.BH = BH;
   a.N = N;
   a.bias_heads = bias_heads;
+  a.bias_mode = shared ? kBiasWindow : kBiasTile;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
   a.timeout_ns = kWaitTimeoutNs;
@@ -600,6 +627,43 @@ int rfb_attn_fwd_shared_bias(const void* q, const void* k, const void* v, const 
                              const void* w, void* o, float* lse, int B, int H, int N, int d,
                              int r, float scale, void* stream) {
   return attn_fwd_impl(q, k, v, u, w, o, lse, B, H, N, d, r, scale, stream, true);
+}
+
+int rfb_attn_fwd_dense_bias(const void* q, const void* k, const void* v, const void* bias,
+                            void* o, float* lse, int B, int H, int N, int d, int bias_heads,
+                            float scale, void* stream) {
+  bool empty = false;
+  if (int rc = check_shape(B, H, N, d, 0, scale, &empty)) return rc;
+  if (empty) return RFB_OK;
+  if (!q || !k || !v || !bias || !o || !lse) return RFB_ERR_INVALID_ARG;
+  const int BH = B * H;
+  if (bias_heads != H && bias_heads != BH) return RFB_ERR_INVALID_ARG;
+  if (N % 8 != 0) return RFB_ERR_UNSUPPORTED;  // bias rows must be 16-byte multiples
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) || !aligned16(o) ||
+      !aligned16(lse))
+    return RFB_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  Maps m;
+  std::memset(&m, 0, sizeof(m));
+  int rc = encode_3d(&m.q, q, d, N, BH, d, kTile, 1);
+  if (!rc) rc = encode_3d(&m.k, k, d, N, BH, d, kTile, 1);
+  if (!rc) rc = encode_3d(&m.v, v, d, N, BH, d, kTile, 1);
+  if (!rc) rc = encode_3d(&m.u, bias, N, N, bias_heads, 64, kTile, 1);
+  if (rc) return rc;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.err = dev.err_word;
+  a.BH = BH;
+  a.N = N;
+  a.bias_heads = bias_heads;
+  a.bias_mode = kBiasTile;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.inv_scale = 1.0f / scale;
+  a.timeout_ns = kWaitTimeoutNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 32 ? launch_long_dense<32>(m, a, dev.sms, st) : launch_long_dense<64>(m, a, dev.sms, st);
 }
 
 size_t rfb_attn_bwd_workspace_size(int B, int H, int N, int d, int r) {

@@ -92,6 +92,14 @@ def test_shared_bias_host_checks_and_workspace(rfb_lib):
     assert need <= ws < need + 2 * B * H * 128 * 4 + 2048
 
 
+def test_dense_bias_host_checks(rfb_lib):
+    lib = rfb_lib.load_library()
+    n = None
+    assert lib.rfb_attn_fwd_dense_bias(n, n, n, n, n, n, 0, 2, 64, 32, 2, 0.1, n) == 0
+    assert lib.rfb_attn_fwd_dense_bias(n, n, n, n, n, n, 1, 2, 64, 32, 2, 0.1, n) == 1  # nulls
+    assert lib.rfb_attn_fwd_dense_bias(n, n, n, n, n, n, 1, 2, 64, 48, 2, 0.1, n) == 2  # d
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     from rank_biased_window_b200 import binding
     # a fresh loader pointed at a missing file must raise, never fall back

@@ -33,7 +33,10 @@ def _expand(t, B):
 
 
 CASES = [
-    (2, 3, 64, 32, 16),   # two windows per tile whose bias heads wrap (2, 0)
+    (2, 3, 64, 32, 16),   # two windows per tile whose bias heads wrap (2, 0); resident
+    (1, 1, 64, 32, 8),    # one window: as many bias heads as window-heads
+    (2, 9, 64, 32, 16),   # too many heads to keep resident: one copy per window, wrapping
+    (2, 3, 100, 64, 64),  # one window per tile, copied per window
     (3, 1, 49, 64, 8),    # ragged window
     (2, 2, 200, 64, 32),  # long regime
     (2, 3, 130, 32, 16),
