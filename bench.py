@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", choices=("rfb", "reference"), default="rfb")
     ap.add_argument("--workload", default="train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--factorize", action="store_true",
+                    help="time the low-rank factoriser of a dense relative-position bias "
+                         "(the step before the path) on this workload's window, r = its rank")
     ap.add_argument("--dense-bias", action="store_true",
                     help="materialised-bias comparator: forward with the bias given as a "
                          "dense bf16 [H, N, N] matrix (U[h] W[h]^T), forward only")
@@ -263,6 +266,43 @@ def cpu_sample_fixed(wl, R, x64):
 
 
 # ------------------------------------------------------------------ GPU arm
+def run_factorize(args, wl, rank):
+    """Times rank_biased_window_b200.factorize_bias on a synthetic
+    relative-position bias of this workload's window ([H, N, N], square
+    windows) at rank r, and reports the relative error against the best
+    possible rank-r error (the oracle's truncated SVD)."""
+    import math
+    import torch
+    from rank_biased_window_b200.factorize import factorize_bias, relative_position_bias
+    side = int(round(math.sqrt(wl.N)))
+    if side * side != wl.N or rank != 0:
+        return
+    dev = torch.device("cuda", 0)
+    bias = relative_position_bias(wl.H, side, side, seed=wl.seed, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        factorize_bias(bias, wl.r)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        _, _, err = factorize_bias(bias, wl.r)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    line = {"metric": "low-rank factoriser of a dense bias: ms per call", "value": ms,
+            "unit": "ms", "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "data": "synthetic smooth relative-position bias",
+            "config": {"workload": wl.name, "H": wl.H, "N": wl.N, "r": wl.r,
+                       "window": f"{side}x{side}"},
+            "rel_err": [round(float(v), 5) for v in err.tolist()]}
+    if not args.no_cpu_baseline:
+        sys.path.insert(0, ROOT)
+        import oracle
+        _, _, opt = oracle.factorize_bias(bias.double().cpu().numpy(), wl.r)
+        line["oracle_rel_err"] = [round(float(v), 5) for v in opt.tolist()]
+    print(json.dumps(line))
+
+
 def main():
     args = parse_args()
     from rank_biased_window_b200.inputs import WORKLOADS, workload_inputs
@@ -276,6 +316,8 @@ def main():
     import torch
     import rank_biased_window_b200 as rfb
     from rank_biased_window_b200 import build as rfb_build
+    if args.factorize:
+        return run_factorize(args, wl, rank)
 
     dist = None
     if world > 1:

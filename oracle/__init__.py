@@ -247,3 +247,29 @@ def fwd_dense_bias(q, k, v, bias, scale):
             O[b, h] = (E @ v[b, h]) / l
             L[b, h] = (m + np.log(l))[:, 0]
     return O, L
+
+
+def factorize_bias(bias, r):
+    """Best rank-r factors of each head's bias matrix (Eckart-Young: the
+    truncated SVD), the step that turns a materialised bias into the factored
+    form ("FlashBias: Fast Computation of Attention with Bias", Abstract: a
+    low-rank bias keeps attention fast).  ``bias`` ``[H, N, N]`` float64.
+    With Bias_h = X S Y^T (singular values S descending)::
+
+        U_h = X[:, :r] sqrt(S[:r]),   W_h = Y[:, :r] sqrt(S[:r])
+
+    so U_h W_h^T is the rank-r truncation.  Returns ``(U, W, rel_err)`` with
+    ``rel_err[h] = ||Bias_h - U_h W_h^T||_F / ||Bias_h||_F``.  Pinned in
+    ``tests/test_factorize.py``."""
+    bias = np.asarray(bias, dtype=np.float64)
+    H, N, _ = bias.shape
+    U = np.empty((H, N, r))
+    W = np.empty((H, N, r))
+    err = np.empty(H)
+    for h in range(H):
+        X, S, Yt = np.linalg.svd(bias[h])
+        root = np.sqrt(S[:r])
+        U[h] = X[:, :r] * root
+        W[h] = Yt[:r].T * root
+        err[h] = np.linalg.norm(bias[h] - U[h] @ W[h].T) / np.linalg.norm(bias[h])
+    return U, W, err

@@ -1,0 +1,90 @@
+"""Low-rank factoriser of a materialised bias: the oracle's truncated SVD is
+pinned by the Eckart-Young closed form, exact recovery of rank-r input and a
+diagonal case; the randomised factoriser (torch, any device) is checked
+against the oracle's optimal error."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rank_biased_window_b200.factorize import factorize_bias, relative_position_bias
+
+
+def test_oracle_error_is_eckart_young():
+    """||B - B_r||_F^2 = sum of the eigenvalues of B^T B beyond the r largest
+    (eigenvalues from a separate symmetric solver)."""
+    rng = np.random.default_rng(5)
+    B = rng.standard_normal((3, 20, 20))
+    for r in (1, 5, 12):
+        _, _, err = oracle.factorize_bias(B, r)
+        for h in range(3):
+            lam = np.sort(np.linalg.eigvalsh(B[h].T @ B[h]))[::-1]
+            want = np.sqrt(lam[r:].sum() / lam.sum())
+            assert abs(err[h] - want) < 1e-10
+
+
+def test_oracle_recovers_exact_low_rank_and_diagonal():
+    rng = np.random.default_rng(6)
+    U0, W0 = rng.standard_normal((2, 16, 3)), rng.standard_normal((2, 16, 3))
+    B = np.einsum("hnr,hmr->hnm", U0, W0)
+    U, W, err = oracle.factorize_bias(B, 3)
+    np.testing.assert_allclose(np.einsum("hnr,hmr->hnm", U, W), B, atol=1e-10)
+    assert err.max() < 1e-12
+    d = np.array([5.0, 4.0, 3.0, 2.0, 1.0])
+    _, _, err = oracle.factorize_bias(np.diag(d)[None], 2)
+    assert abs(err[0] - np.sqrt((d[2:] ** 2).sum() / (d ** 2).sum())) < 1e-14
+
+
+@pytest.mark.parametrize("r", [4, 8, 16])
+def test_randomised_factoriser_near_optimal_cpu(r):
+    B = relative_position_bias(3, 8, 8, seed=11)
+    U, W, err = factorize_bias(B, r, out_dtype=torch.float32)
+    assert U.shape == (3, 64, r) and W.shape == (3, 64, r)
+    _, _, opt = oracle.factorize_bias(B.double().numpy(), r)
+    # within 2 % of the best possible rank-r error (power iterations converge fast)
+    assert (err.numpy() <= opt * 1.02 + 1e-5).all(), (err, opt)
+    # reported error matches the factors returned
+    R = B - torch.bmm(U, W.transpose(1, 2))
+    np.testing.assert_allclose(err.numpy(), (torch.linalg.matrix_norm(R) /
+                                             torch.linalg.matrix_norm(B)).numpy(), rtol=1e-4)
+
+
+def test_randomised_factoriser_exact_rank_and_bf16_output():
+    g = torch.Generator().manual_seed(3)
+    U0, W0 = torch.randn((2, 48, 8), generator=g), torch.randn((2, 48, 8), generator=g)
+    B = torch.bmm(U0, W0.transpose(1, 2))
+    U, W, err = factorize_bias(B, 8)                       # bf16 factors
+    assert U.dtype == torch.bfloat16
+    assert err.max().item() < 1e-2                          # bf16 rounding of the factors
+    _, _, err32 = factorize_bias(B, 8, out_dtype=torch.float32)
+    assert err32.max().item() < 1e-5
+
+
+def test_factoriser_argument_checks():
+    with pytest.raises(ValueError):
+        factorize_bias(torch.zeros(2, 4, 5), 2)
+    with pytest.raises(ValueError):
+        factorize_bias(torch.zeros(2, 4, 4), 0)
+
+
+@pytest.mark.gpu
+def test_factorised_bias_feeds_the_kernels(rfb_lib, cuda_dev):
+    """On the GPU: factorise a window bias, then run the factored kernel with
+    the factors and the dense comparator with their product U W^T; the two
+    compute the same attention (up to bf16 rounding of the product)."""
+    from rank_biased_window_b200.inputs import make_inputs
+    H, wh, ww, r, B = 4, 16, 16, 32, 3
+    bias = relative_position_bias(H, wh, ww, seed=21, device=cuda_dev)
+    U, W, err = factorize_bias(bias, r)
+    _, _, opt = oracle.factorize_bias(bias.double().cpu().numpy(), r)
+    assert (err.cpu().numpy() <= opt * 1.05 + 4e-3).all()   # bf16 factors
+    N, d = wh * ww, 32
+    x = make_inputs(B, H, N, d, 0, seed=22)
+    g = {k: v.to(cuda_dev) for k, v in x.items()}
+    o1, _ = rfb_lib.attn_fwd_shared_bias(g["q"], g["k"], g["v"], U, W)
+    prod = torch.bmm(U.float(), W.float().transpose(1, 2)).to(torch.bfloat16).contiguous()
+    o2, _ = rfb_lib.attn_fwd_dense_bias(g["q"], g["k"], g["v"], prod)
+    torch.cuda.synchronize()
+    assert rfb_lib.last_device_error() == 0
+    diff = (o1.float() - o2.float()).abs().max().item()
+    assert diff < 3e-2, diff
