@@ -273,3 +273,57 @@ def factorize_bias(bias, r):
         W[h] = Yt[:r].T * root
         err[h] = np.linalg.norm(bias[h] - U[h] @ W[h].T) / np.linalg.norm(bias[h])
     return U, W, err
+
+
+def _shift_regions(n, win, shift):
+    """Region id along one axis of the cyclically shifted map (the shifted-window
+    mask: positions that were not neighbours before the roll get different ids)."""
+    ids = np.zeros(n, dtype=np.int64)
+    if shift > 0:
+        ids[n - win:n - shift] = 1
+        ids[n - shift:] = 2
+    return ids
+
+
+def fwd_image_windows(q, k, v, u, w, scale, win, shift):
+    """Shifted-window attention over feature maps, written out step by step
+    (the window attention of SR transformers such as SwinIR, with the bias in
+    the rank-factorised form of "Rank-Factorized Implicit Neural Bias",
+    Abstract).  ``q, k, v`` ``[B, Hs, Ws, heads, d]``; ``u, w`` ``[heads,
+    win*win, r]`` indexed by the token's raster position inside its window
+    (one pair per head, shared by all windows), or None.
+
+    1. roll the maps by (-shift, -shift) over (Hs, Ws);
+    2. cut the rolled maps into win x win windows (raster order);
+    3. per window and head: S = s Q K^T + U W^T, with S = -inf between tokens
+       whose regions of the rolled map differ (when shift > 0);
+       P = softmax(S), O = P V, LSE = log sum exp S;
+    4. put every token's O and LSE back at its position before the roll.
+
+    Returns ``(O [B, Hs, Ws, heads, d], LSE [B, Hs, Ws, heads])`` in float64."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    B, Hs, Ws, nh, d = q.shape
+    qs, ks, vs = (np.roll(x, (-shift, -shift), axis=(1, 2)) for x in (q, k, v))
+    ry, rx = _shift_regions(Hs, win, shift), _shift_regions(Ws, win, shift)
+    O = np.zeros_like(qs)
+    L = np.zeros((B, Hs, Ws, nh))
+    N = win * win
+    for b in range(B):
+        for y0 in range(0, Hs, win):
+            for x0 in range(0, Ws, win):
+                ys, xs = np.meshgrid(np.arange(y0, y0 + win), np.arange(x0, x0 + win), indexing="ij")
+                ys, xs = ys.reshape(-1), xs.reshape(-1)           # raster order in the window
+                region = 3 * ry[ys] + rx[xs]
+                allowed = region[:, None] == region[None, :]
+                for h in range(nh):
+                    Qw, Kw, Vw = qs[b, ys, xs, h], ks[b, ys, xs, h], vs[b, ys, xs, h]
+                    S = scale * (Qw @ Kw.T)
+                    if u is not None:
+                        S = S + np.asarray(u, dtype=np.float64)[h] @ np.asarray(w, dtype=np.float64)[h].T
+                    S = np.where(allowed, S, -np.inf)
+                    m = S.max(axis=1, keepdims=True)
+                    E = np.exp(S - m)
+                    l = E.sum(axis=1, keepdims=True)
+                    O[b, ys, xs, h] = (E @ Vw) / l
+                    L[b, ys, xs, h] = (m + np.log(l))[:, 0]
+    return (np.roll(O, (shift, shift), axis=(1, 2)), np.roll(L, (shift, shift), axis=(1, 2)))
