@@ -186,6 +186,35 @@ RFB_API int rfb_attn_fwd_dense_bias(const void* q, const void* k, const void* v,
                                     void* o, float* lse, int B, int H, int N, int d,
                                     int bias_heads, float scale, void* stream);
 
+/*
+ * Shifted-window attention straight from feature maps (forward): the window
+ * partition and the cyclic shift of SR window transformers happen in the copy
+ * engine's addressing, with the bias in the rank-factorised form of
+ * "Rank-Factorized Implicit Neural Bias" (Abstract).  For each image b, the
+ * map rolled by (-shift, -shift) is cut into win x win windows (raster order);
+ * per window and head h,
+ *     O = softmax(s Q K^T + U[h] W[h]^T + M) V,
+ * where M is 0 between tokens of the same region of the rolled map and -inf
+ * between tokens of different regions (regions: rows [0, H-win), [H-win,
+ * H-shift), [H-shift, H) times the same split of columns; all one region when
+ * shift == 0); every token's O and LSE are written at its place in the
+ * unrolled map.  Nothing is copied or rolled in memory.
+ *   q, k, v, o : [B, img_h, img_w, heads, d] bf16 (channels-last maps).
+ *   u, w       : [heads, win*win, r] bf16, row = raster position in the
+ *                window (one pair per head for all windows); NULL iff r == 0.
+ *   lse        : [B, img_h, img_w, heads] fp32 (natural log).
+ *   win        : 8 (64 tokens per window); shift : 0 or 4.
+ *   img_h, img_w : multiples of 8.
+ * Errors as rfb_attn_fwd; RFB_ERR_UNSUPPORTED for other win / shift / map
+ * sizes, or when the factors of all heads do not fit in shared memory at once
+ * ((heads + 1) * 64 * r_pad * 4 bytes beside the input ring; e.g. up to 20
+ * heads at r <= 16, 9 at r = 32, 4 at r = 64 for d = 32).
+ */
+RFB_API int rfb_attn_fwd_image_windows(const void* q, const void* k, const void* v,
+                                       const void* u, const void* w, void* o, float* lse, int B,
+                                       int img_h, int img_w, int heads, int d, int r, int win,
+                                       int shift, float scale, void* stream);
+
 /* Human-readable text for a status code (static storage). */
 RFB_API const char* rfb_strerror(int status);
 

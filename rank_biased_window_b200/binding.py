@@ -36,6 +36,7 @@ SIGNATURES = {
     "rfb_attn_fwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_i] * 5 + [_f, _vp]),
     "rfb_attn_bwd_shared_bias_workspace_size": (_sz, [_i] * 5),
     "rfb_attn_fwd_dense_bias": (_i, [_vp] * 5 + [_fp] + [_i] * 5 + [_f, _vp]),
+    "rfb_attn_fwd_image_windows": (_i, [_vp] * 6 + [_fp] + [_i] * 8 + [_f, _vp]),
     "rfb_attn_bwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
     "rfb_strerror": (ctypes.c_char_p, [_i]),
     "rfb_last_device_error": (_i, []),
@@ -260,6 +261,38 @@ def attn_fwd_dense_bias(q, k, v, bias, scale=None, *, out=None, lse=None, stream
             ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, H, N, d, bias_heads, s,
             _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_fwd_dense_bias")
+    return o, l
+
+
+def attn_fwd_image_windows(q, k, v, u=None, w=None, scale=None, *, win=8, shift=0, out=None,
+                           lse=None, stream=None):
+    """Shifted-window attention from feature maps q, k, v [B, H, W, heads, d]
+    with shared factors u, w [heads, win*win, r]: returns O [B, H, W, heads, d]
+    and LSE [B, H, W, heads] at the tokens' map positions."""
+    if q.dim() != 5:
+        raise ValueError("q must be [B, H, W, heads, d]")
+    B, Hs, Ws, nh, d = (int(x) for x in q.shape)
+    r = 0 if u is None else int(u.shape[-1])
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_operand(name, t, (B, Hs, Ws, nh, d), dev)
+    if r > 0:
+        _check_operand("u", u, (nh, win * win, r), dev)
+        _check_operand("w", w, (nh, win * win, r), dev)
+    else:
+        u = w = None
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, Hs, Ws, nh), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_operand("out", o, (B, Hs, Ws, nh, d), dev)
+    if l.dtype != torch.float32 or tuple(l.shape) != (B, Hs, Ws, nh) or not l.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, W, heads]")
+    with _on_device(dev):
+        rc = load_library().rfb_attn_fwd_image_windows(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(l.data_ptr()), _fp), B, Hs, Ws, nh, d, r, int(win),
+            int(shift), s, _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_fwd_image_windows")
     return o, l
 
 

@@ -45,6 +45,10 @@ struct FwdArgs {
   // pair per head, shared by all windows).  Window-head bh uses bias head
   // bh % bias_heads (bh = b H + h).
   int bias_heads;
+  // Image-window mode of the window kernel (feature maps [B, img_h, img_w,
+  // img_heads, D], 8 x 8 windows of the map rolled by -shift): window-head
+  // bh = ((b * (img_h / 8) + wy) * (img_w / 8) + wx) * img_heads + h.
+  int img_h, img_w, img_heads, shift;
   // Window kernel: how U / W reach shared memory.  kBiasTile: one copy per
   // tile (per-window factors); kBiasWindow: one copy per window (shared
   // factors); kBiasResident: all bias heads loaded once per CTA (shared
@@ -191,12 +195,15 @@ __device__ __forceinline__ void issue_pv_ts(uint32_t o_tmem, uint32_t p_tmem, ui
 // ============================================================ window regime
 constexpr int kBiasTile = 0, kBiasWindow = 1, kBiasResident = 2;
 
-template <int D, int RP, int NP>
+// IMG: windows gathered from feature maps (8 x 8 windows, NP = 64), factors
+// always resident, so a stage holds only Q, K, V.
+template <int D, int RP, int NP, bool IMG = false>
 struct WinCfg {
+  static_assert(!IMG || NP == 64, "image windows are 8 x 8");
   static constexpr int NW = kTile / NP;       // windows packed per tile
   static constexpr int QB = kTile * D * 2;    // bytes of a Q / K / V tile
   static constexpr int UB = kTile * RP * 2;   // bytes of a U / W tile
-  static constexpr int STAGE = 3 * QB + 2 * UB;
+  static constexpr int STAGE = 3 * QB + (IMG ? 0 : 2 * UB);
   static constexpr int NS_FIT = (224 * 1024) / STAGE;
   static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
   static constexpr int OFF_BAR = NS * STAGE;
@@ -223,12 +230,17 @@ constexpr uint32_t kWinSoftmaxRegs = 208, kWinControlRegs = 56;
 static_assert(2 * 128 * kWinSoftmaxRegs + 128 * kWinControlRegs <= kWinThreads * 168,
               "register split exceeds the launch budget");
 
-template <int D, int RP, int NP>
+// With IMG the Q / K / V maps are 5-D over the feature maps (D, heads, W, H, B)
+// with a 4 x 4-token box, and U / W 4-D (r, 8, 8, heads) with a 4 x 4 box:
+// each window is copied as four 4 x 4 quadrants, so inside the kernel its
+// tokens are in quadrant-major order (row 16 q + 4 (y % 4) + x % 4, q = 2 (y /
+// 4) + x / 4) for Q, K, V, U and W alike; O and LSE go back to map positions.
+template <int D, int RP, int NP, bool IMG = false>
 __global__ void __launch_bounds__(kWinThreads, 1)
     fwd_window_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                       const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
                       const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
-  using C = WinCfg<D, RP, NP>;
+  using C = WinCfg<D, RP, NP, IMG>;
   constexpr int NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
@@ -245,7 +257,16 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (3 * NS + 10);
   const uint32_t res_full = bar0 + 8u * (3 * NS + 11);   // resident factors landed
   const uint32_t res_ready = bar0 + 8u * (3 * NS + 12);  // resident U' scaled
-  const bool resident = RP > 0 && args.bias_mode == kBiasResident;
+  const bool resident = RP > 0 && (IMG || args.bias_mode == kBiasResident);
+  // Image windows: map coordinates of window-head bh.
+  const int nwx = IMG ? args.img_w / 8 : 1, nwy = IMG ? args.img_h / 8 : 1;
+  auto window_of = [&](int bh, int& b, int& wy, int& wx, int& h) {
+    h = bh % args.img_heads;
+    const int bw = bh / args.img_heads;
+    wx = bw % nwx;
+    wy = (bw / nwx) % nwy;
+    b = bw / (nwx * nwy);
+  };
   const int res_heads = args.bias_heads + C::NW - 1;
   const uint32_t res_u = sb + C::OFF_RES, res_w = res_u + res_heads * C::HB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
@@ -304,8 +325,17 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         mbar_expect_tx(res_full, C::res_bytes(args.bias_heads));
         for (int hh = 0; hh < res_heads; ++hh) {
           const int z = hh % args.bias_heads;
-          tma_load_3d(res_u + hh * C::HB, &mU, res_full, 0, 0, z);
-          tma_load_3d(res_w + hh * C::HB, &mW, res_full, 0, 0, z);
+          if constexpr (IMG) {
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+              const uint32_t off = hh * C::HB + qd * (16 * RP * 2);
+              tma_load_4d(res_u + off, &mU, res_full, 0, 4 * (qd & 1), 4 * (qd >> 1), z);
+              tma_load_4d(res_w + off, &mW, res_full, 0, 4 * (qd & 1), 4 * (qd >> 1), z);
+            }
+          } else {
+            tma_load_3d(res_u + hh * C::HB, &mU, res_full, 0, 0, z);
+            tma_load_3d(res_w + hh * C::HB, &mW, res_full, 0, 0, z);
+          }
         }
       }
       const uint32_t stage_tx = resident ? 3 * C::QB : C::STAGE;
@@ -316,10 +346,30 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         const uint32_t st = sb + s * C::STAGE;
         mbar_expect_tx(in_full(s), stage_tx);
         const int w0 = t * C::NW;
-        tma_load_3d(st, &mQ, in_full(s), 0, 0, w0);
-        tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
-        tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
-        if constexpr (RP > 0) {
+        if constexpr (IMG) {
+          // Each window as four 4 x 4 quadrants of the rolled map, taken from
+          // the unrolled map at (row + shift, column + shift) mod size.  A
+          // missing last window repeats the previous one (not stored).
+#pragma unroll
+          for (int i = 0; i < C::NW; ++i) {
+            int b, wy, wx, h;
+            window_of(min(w0 + i, args.BH - 1), b, wy, wx, h);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+              const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
+              const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+              const uint32_t off = i * (NP * D * 2) + qd * (16 * D * 2);
+              tma_load_5d(st + off, &mQ, in_full(s), 0, h, x, y, b);
+              tma_load_5d(st + C::QB + off, &mK, in_full(s), 0, h, x, y, b);
+              tma_load_5d(st + 2 * C::QB + off, &mV, in_full(s), 0, h, x, y, b);
+            }
+          }
+        } else {
+          tma_load_3d(st, &mQ, in_full(s), 0, 0, w0);
+          tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
+          tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
+        }
+        if constexpr (RP > 0 && !IMG) {
           if (resident) {
             // factors already resident
           } else if (args.bias_mode == kBiasTile) {
@@ -452,6 +502,26 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       tc_fence_before();
       mbar_arrive(s_empty(a));
       if (N < NP) mask_tail<NP>(sv, N);
+      if constexpr (IMG) {
+        // Shifted-window mask: in the last window row (column) of the rolled
+        // map the two quadrant rows (columns) come from opposite edges of the
+        // unrolled map; keys of another region are excluded.
+        if (args.shift > 0) {
+          int b, wy, wx, h;
+          window_of(min(t * C::NW + wl, args.BH - 1), b, wy, wx, h);
+          const int qq = n >> 4;
+          const bool split_y = wy == nwy - 1, split_x = wx == nwx - 1;
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            const bool ok_key = (!split_y || (kq >> 1) == (qq >> 1)) &&
+                                (!split_x || (kq & 1) == (qq & 1));
+            if (!ok_key) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sv[kq * 16 + e] = 0xFF800000u;
+            }
+          }
+        }
+      }
       const float m = row_max<NP>(sv) * sl2;
       // P_a was last read by PV(it - 2), complete since this warpgroup saw
       // o_full for that tile.
@@ -468,7 +538,16 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       mbar_arrive(acc_empty(a));
       const int win = t * C::NW + wl;
       if (win < args.BH && n < N) {
-        const size_t r = static_cast<size_t>(win) * N + n;
+        size_t r = static_cast<size_t>(win) * N + n;
+        if constexpr (IMG) {
+          // back to the token's place in the unrolled map
+          int b, wy, wx, h;
+          window_of(win, b, wy, wx, h);
+          const int qq = n >> 4;
+          const int y = (wy * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift) % args.img_h;
+          const int x = (wx * 8 + 4 * (qq & 1) + (n & 3) + args.shift) % args.img_w;
+          r = ((static_cast<size_t>(b) * args.img_h + y) * args.img_w + x) * args.img_heads + h;
+        }
         store_o_row<D>(args.o + r * D, ov, 1.0f / l);
         args.lse[r] = (m + __log2f(l)) * kLn2;
       }

@@ -247,6 +247,20 @@ int encode_acc_3d_uncached(CUtensorMap* m, void* ptr, int cols, int N, int BH) {
   return rc == CUDA_SUCCESS ? RFB_OK : cuda_fail(static_cast<int>(rc), kSiteEncode);
 }
 
+// bf16 map of any rank (dims innermost first, strides in bytes for dims 1..),
+// not cached (the image-window maps).
+int encode_nd(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return cuda_fail(0, kSiteEncoder);
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult rc = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle_for(static_cast<int>(box[0]) * 2),
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? RFB_OK : cuda_fail(static_cast<int>(rc), kSiteEncode);
+}
+
 int pad_rank(int r) { return r == 0 ? 0 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -364,6 +378,33 @@ int launch_long(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   LaunchTimer timer(kIdFwd, st);
   fwd_long_kernel<D, RP><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
+}
+
+// Shifted windows gathered from feature maps (window kernel, IMG).
+template <int D, int RP>
+int launch_window_img(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
+  using C = WinCfg<D, RP, 64, true>;
+  static std::atomic<uint64_t> done{0};
+  constexpr int kMaxSmem = 232448;
+  if (int rc = ensure_smem(fwd_window_kernel<D, RP, 64, true>, kMaxSmem, done)) return rc;
+  const long long need =
+      RP > 0 ? C::OFF_RES + static_cast<long long>(C::res_bytes(a.bias_heads)) + 1024 : C::SMEM;
+  if (need > kMaxSmem) return RFB_ERR_UNSUPPORTED;  // factors of all heads must stay resident
+  const int tiles = (a.BH + C::NW - 1) / C::NW;
+  const int grid = tiles < sms ? tiles : sms;
+  LaunchTimer timer(kIdFwd, st);
+  fwd_window_kernel<D, RP, 64, true><<<grid, kWinThreads, static_cast<int>(need), st>>>(
+      m.q, m.k, m.v, m.u, m.w, a);
+  return launch_status();
+}
+
+int dispatch_window_img(int d, int rp, const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
+#define RFB_IMG_CASE(DD, RR) \
+  if (d == DD && rp == RR) return launch_window_img<DD, RR>(m, a, sms, st);
+  RFB_IMG_CASE(32, 0) RFB_IMG_CASE(32, 16) RFB_IMG_CASE(32, 32) RFB_IMG_CASE(32, 64)
+  RFB_IMG_CASE(64, 0) RFB_IMG_CASE(64, 16) RFB_IMG_CASE(64, 32) RFB_IMG_CASE(64, 64)
+#undef RFB_IMG_CASE
+  return RFB_ERR_UNSUPPORTED;
 }
 
 // The materialised-bias comparator (long kernel, DENSE).
@@ -664,6 +705,66 @@ int rfb_attn_fwd_dense_bias(const void* q, const void* k, const void* v, const v
   a.timeout_ns = kWaitTimeoutNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 32 ? launch_long_dense<32>(m, a, dev.sms, st) : launch_long_dense<64>(m, a, dev.sms, st);
+}
+
+int rfb_attn_fwd_image_windows(const void* q, const void* k, const void* v, const void* u,
+                               const void* w, void* o, float* lse, int B, int img_h, int img_w,
+                               int heads, int d, int r, int win, int shift, float scale,
+                               void* stream) {
+  bool empty = false;
+  if (int rc = check_shape(B, heads, 64, d, r, scale, &empty)) return rc;
+  if (B < 0 || img_h < 0 || img_w < 0) return RFB_ERR_INVALID_ARG;
+  if (win != 8 || (shift != 0 && shift != 4)) return RFB_ERR_UNSUPPORTED;
+  if (img_h % 8 != 0 || img_w % 8 != 0) return RFB_ERR_UNSUPPORTED;
+  if (empty || img_h == 0 || img_w == 0) return RFB_OK;
+  if (!q || !k || !v || !o || !lse || (r > 0 && (!u || !w))) return RFB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (r > 0 && (!aligned16(u) || !aligned16(w))))
+    return RFB_ERR_ALIGNMENT;
+  const long long bh = static_cast<long long>(B) * (img_h / 8) * (img_w / 8) * heads;
+  if (bh > 0x7fffffffLL) return RFB_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  const int rp = pad_rank(r);
+  Maps m;
+  std::memset(&m, 0, sizeof(m));
+  // Q, K, V: (d, heads, W, H, B), a 4 x 4-token box of one head.
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(img_w), static_cast<cuuint64_t>(img_h),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
+  const cuuint64_t strides[4] = {row, row * heads, row * heads * img_w,
+                                 row * heads * img_w * img_h};
+  const cuuint32_t box[5] = {static_cast<cuuint32_t>(d), 1, 4, 4, 1};
+  int rc = encode_nd(&m.q, q, 5, dims, strides, box);
+  if (!rc) rc = encode_nd(&m.k, k, 5, dims, strides, box);
+  if (!rc) rc = encode_nd(&m.v, v, 5, dims, strides, box);
+  if (!rc && r > 0) {
+    // U, W [heads, 64, r] as (r, 8, 8, heads), a 4 x 4 box.
+    const cuuint64_t udims[4] = {static_cast<cuuint64_t>(r), 8, 8, static_cast<cuuint64_t>(heads)};
+    const cuuint64_t urow = static_cast<cuuint64_t>(r) * 2;
+    const cuuint64_t ustr[3] = {urow, urow * 8, urow * 64};
+    const cuuint32_t ubox[4] = {static_cast<cuuint32_t>(rp), 4, 4, 1};
+    rc = encode_nd(&m.u, u, 4, udims, ustr, ubox);
+    if (!rc) rc = encode_nd(&m.w, w, 4, udims, ustr, ubox);
+  }
+  if (rc) return rc;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.err = dev.err_word;
+  a.BH = static_cast<int>(bh);
+  a.N = 64;
+  a.bias_heads = heads;
+  a.bias_mode = kBiasResident;
+  a.img_h = img_h;
+  a.img_w = img_w;
+  a.img_heads = heads;
+  a.shift = shift;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.inv_scale = 1.0f / scale;
+  a.timeout_ns = kWaitTimeoutNs;
+  return dispatch_window_img(d, rp, m, a, dev.sms, static_cast<cudaStream_t>(stream));
 }
 
 size_t rfb_attn_bwd_workspace_size(int B, int H, int N, int d, int r) {
