@@ -16,8 +16,12 @@ bias matrix added to the query-key scores) and "Rank-Factorized Implicit Neural
 Bias" (Abstract: a low-rank bias U W^T).  The backward is the plain chain rule
 through the same definition (see ``rfb_oracle.c``).
 
-The arithmetic lives in ``rfb_oracle.c`` (plain C, fp64, OpenMP over output
-rows).  This module only compiles it with gcc and marshals numpy arrays.
+The arithmetic of ``fwd`` / ``bwd`` / ``bwd_query_rows`` lives in
+``rfb_oracle.c`` (plain C, fp64, OpenMP over output rows); this module compiles
+it with gcc and marshals numpy arrays.  Three further definitions are written
+here in plain numpy (fp64, one head at a time): ``fwd_dense_bias`` (the bias
+as a dense matrix), ``factorize_bias`` (best rank-r factors of a dense bias)
+and ``fwd_image_windows`` (shifted-window attention over feature maps).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against library special
 cases (torch SDPA and autograd in fp64), brute force with ``math.fsum``,
