@@ -19,6 +19,13 @@
  *     bias.
  *   - The scale s multiplies Q K^T only (the bias is added after scaling).
  *
+ * Entry points: the per-window forward / backward (rfb_attn_fwd,
+ * rfb_attn_bwd, rfb_attn_bwd_noalloc); variants with one factor pair per head
+ * shared by all windows (rfb_attn_*_shared_bias); shifted-window attention read
+ * straight from feature maps (rfb_attn_fwd_image_windows); a dense-bias
+ * comparator (rfb_attn_fwd_dense_bias); diagnostics.  Each declaration below
+ * states what differs from these conventions.
+ *
  * Conventions for every entry point
  *   - Layout: all tensors are contiguous row-major.  Q, K, V, O, dO and their
  *     gradients are [B, H, N, d] bf16; U, W, dU, dW are [B, H, N, r] bf16;
