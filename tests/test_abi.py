@@ -100,6 +100,48 @@ def test_dense_bias_host_checks(rfb_lib):
     assert lib.rfb_attn_fwd_dense_bias(n, n, n, n, n, n, 1, 2, 64, 48, 2, 0.1, n) == 2  # d
 
 
+def test_image_windows_host_checks(rfb_lib):
+    lib = rfb_lib.load_library()
+    n = None
+    f = lib.rfb_attn_fwd_image_windows
+    # B, img_h, img_w, heads, d, r, win, shift, scale
+    assert f(n, n, n, n, n, n, n, 0, 16, 16, 2, 32, 8, 8, 0, 0.1, n) == 0   # empty
+    assert f(n, n, n, n, n, n, n, 1, 16, 16, 2, 32, 8, 16, 0, 0.1, n) == 2  # window 16
+    assert f(n, n, n, n, n, n, n, 1, 16, 16, 2, 32, 8, 8, 2, 0.1, n) == 2   # shift 2
+    assert f(n, n, n, n, n, n, n, 1, 12, 16, 2, 32, 8, 8, 4, 0.1, n) == 2   # 12 rows
+    assert f(n, n, n, n, n, n, n, 1, 16, 16, 2, 48, 8, 8, 4, 0.1, n) == 2   # d
+    assert f(n, n, n, n, n, n, n, 1, 16, 16, 2, 32, 8, 8, 4, 0.1, n) == 1   # null pointers
+    assert f(n, n, n, n, n, n, n, 1, 16, 16, 2, 32, 8, 8, 4, 0.0, n) == 1   # scale
+
+
+def test_bench_accounting_helpers(tmp_path, monkeypatch):
+    """bench.py's algorithmic flop / byte counts and the traffic record's
+    source-hash gate."""
+    import json
+    import bench
+    from rank_biased_window_b200.inputs import WORKLOADS
+    wl = WORKLOADS["train"]
+    fwd, bwd, fb, bb = bench.work(wl)
+    BH, N, d, r = wl.B * wl.H, wl.N, wl.d, wl.r
+    assert fwd == 2.0 * BH * N * N * (2 * d + r)
+    assert bwd == 2.0 * BH * N * N * (5 * d + 3 * r)
+    assert fb == BH * N * (2 * (3 * d + 2 * r + d) + 4)
+    assert bench.work(WORKLOADS["swinir"])[1] == 0.0          # forward-only workload
+    assert bench.throughput_tflops(1e12, 2, 1000.0) == 2.0    # weak scaling: all ranks' work
+    # a traffic record is used only while the kernel sources are unchanged
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "rank_biased_window_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k.cu").write_text("kernel one")
+    rec = {"source_hash": bench.kernel_source_hash(), "dram_bytes_per_launch": 123.0}
+    (tmp_path / "profiles" / "k_w_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("k", "w") == 123.0
+    (src / "k.cu").write_text("kernel two")
+    assert bench.ncu_traffic("k", "w") is None
+    assert bench.ncu_traffic("missing", "w") is None
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     from rank_biased_window_b200 import binding
     # a fresh loader pointed at a missing file must raise, never fall back
