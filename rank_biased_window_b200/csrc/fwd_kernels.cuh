@@ -134,16 +134,17 @@ __device__ __forceinline__ float row_max(const uint32_t (&sv)[NC]) {
 // p_j = 2^(s_j * sl2 - m) for the NC scores of this thread's row, written as
 // packed bf16 pairs into its TMEM lane (column p_tm + c / 2 holds keys c and
 // c + 1), where the PV MMA reads them as its A operand; returns sum_j p_j
-// (fp32, 4 partial sums).  Masked scores are -inf and give p = 0.  SOFT_PAIRS
+// (fp32; the arguments and four partial sums in packed f32x2 arithmetic, one
+// instruction per pair).  Masked scores are -inf and give p = 0.  SOFT_PAIRS
 // of every 4 pairs of exponentials use the software exp2 (FMA / integer pipes)
 // instead of the MUFU unit.  The stores are not awaited (tmem_st_wait()).
 template <int NC, int SOFT_PAIRS = 0>
 __device__ __forceinline__ float exp_row_to_tmem(const uint32_t (&sv)[NC], float sl2, float m,
                                                  uint32_t p_tm) {
   constexpr int HW = 8 - 2 * SOFT_PAIRS;
-  float l[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) l[e] = 0.f;
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
   for (int c0 = 0; c0 < NC; c0 += 32) {
     uint32_t pk[16];
@@ -151,19 +152,23 @@ __device__ __forceinline__ float exp_row_to_tmem(const uint32_t (&sv)[NC], float
     for (int c = c0; c < c0 + 32; c += 8) {
       float p[8];
 #pragma unroll
-      for (int e = 0; e < HW; ++e) p[e] = fast_exp2(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
-#pragma unroll
-      for (int e = HW; e < 8; e += 2)
-        soft_exp2_x2(fmaf(__uint_as_float(sv[c + e]), sl2, -m),
-                     fmaf(__uint_as_float(sv[c + e + 1]), sl2, -m), p[e], p[e + 1]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) l[e & 3] += p[e];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) pk[(c - c0 + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+      for (int e = 0; e < 8; e += 2) {
+        const uint64_t x2 = static_cast<uint64_t>(sv[c + e + 1]) << 32 | sv[c + e];
+        const float2 a = f2_unpack(f2_fma(x2, sl2x2, nm2));
+        if (e < HW) {
+          p[e] = fast_exp2(a.x);
+          p[e + 1] = fast_exp2(a.y);
+        } else {
+          soft_exp2_x2(a.x, a.y, p[e], p[e + 1]);
+        }
+        l2[e >> 1] = f2_add(l2[e >> 1], f2_pack(p[e], p[e + 1]));
+        pk[(c - c0 + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+      }
     }
     tmem_st16_nowait(p_tm + (c0 >> 1), pk);
   }
-  return (l[0] + l[1]) + (l[2] + l[3]);
+  const float2 a = f2_unpack(f2_add(l2[0], l2[1])), b = f2_unpack(f2_add(l2[2], l2[3]));
+  return (a.x + a.y) + (b.x + b.y);
 }
 
 // Issue the score MMAs  S(tmem) = Q.K^T + U'.W^T  for one 128x128 tile.
