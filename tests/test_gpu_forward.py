@@ -120,3 +120,26 @@ def test_repeat_calls_identical(rfb_lib, cuda_dev):
     o1, l1 = _run_gpu(rfb_lib, x, cuda_dev, 0.125, 32)
     o2, l2 = _run_gpu(rfb_lib, x, cuda_dev, 0.125, 32)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_forward_growing_row_max(rfb_lib, oracle_mod, cuda_dev, d):
+    """A bias that ramps along the keys, rising for some query rows and falling
+    for others, so that the running max grows past the lazy-rescale threshold
+    on every key tile for half the rows of each warp (the tile is exponentiated
+    again with the new max and O rescaled) and never for the rest."""
+    B, H, N, r = 1, 2, 700, 16
+    x = make_inputs(B, H, N, d, r, seed=77 + d)
+    n = torch.arange(N, dtype=torch.float32)
+    u = torch.zeros(B, H, N, r)
+    w = torch.zeros(B, H, N, r)
+    u[..., 0] = torch.where(n % 2 == 0, 1.0, -1.0) * (0.5 + (n % 7) / 8.0)
+    w[..., 0] = 0.06 * n
+    x["u"], x["w"] = u.to(torch.bfloat16), w.to(torch.bfloat16)
+    # A power-of-two scale keeps U / s exact in bf16 at these bias magnitudes.
+    s = 0.125
+    o, lse = _run_gpu(rfb_lib, x, cuda_dev, s, r)
+    f = {k: to_f64(v) for k, v in x.items()}
+    ro, rl = oracle_mod.fwd(f["q"], f["k"], f["v"], f["u"], f["w"], s)
+    assert_close("O", o, ro)
+    assert_close("LSE", lse, rl)
