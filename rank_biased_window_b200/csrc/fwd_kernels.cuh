@@ -24,7 +24,8 @@
 //     tile 0 / 1 (running out of phase), warp 8 TMA, warps 9 / 10 MMA issue
 //     for tile 0 / 1; P goes back into TMEM as packed bf16 and the PV MMA
 //     reads it from there.  The softmax warpgroups take registers from the
-//     control warpgroup (setmaxnreg).
+//     control warpgroup (setmaxnreg).  With d = 32 the row sums of P come
+//     out of the PV MMA (a block of ones beside V), not from the softmax.
 // Operands are staged by TMA with the swizzle that matches their row width.
 #pragma once
 #include "sm100.cuh"
@@ -194,6 +195,19 @@ __device__ __forceinline__ void issue_pv_ts(uint32_t o_tmem, uint32_t p_tmem, ui
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
     umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_mnmajor(v + kk * 16 * (D * 2), D * 2, 128 * D * 2),
+                 id, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// O'(tmem) (+)= P . [V | 1] (N = D + 16): the second MN block of B is a
+// constant block of ones `ones_off` bytes after V, so columns D .. D + 15 of
+// O' accumulate the row sums of P.
+template <int D>
+__device__ __forceinline__ void issue_pv_ts_ones(uint32_t o_tmem, uint32_t p_tmem, uint32_t v,
+                                                 uint32_t ones_off, bool accumulate) {
+  constexpr uint32_t id = idesc_bf16_f32(128, D + 16, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_mnmajor(v + kk * 16 * (D * 2), D * 2, ones_off),
                  id, (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -582,11 +596,20 @@ struct LongCfg {
   // Two query tiles per CTA: Q0 U0 Q1 U1, then the KV stages.  P lives in TMEM.
   static constexpr int OFF_Q = 0;            // Q tile t at OFF_Q + t * (QB + UB), U right after
   static constexpr int OFF_STAGE = 2 * (QB + UB);
-  static constexpr int NS_FIT = (226 * 1024 - OFF_STAGE) / STAGE;
+  // With d = 32 the row sums come out of the PV MMA: B is [V | 1] (a constant
+  // 128 x 32 block of ones as a second MN block, N = d + 16), so column d of
+  // the O accumulator collects sum_j bf16(p_j) and the softmax adds nothing.
+  static constexpr bool LCOL = (D == 32);
+  static constexpr int OD = LCOL ? D + 16 : D;  // O accumulator columns per query tile
+  static constexpr int ONES = LCOL ? kTile * 64 : 0;
+  static constexpr int NS_FIT = (226 * 1024 - OFF_STAGE - ONES) / STAGE;
   static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
-  static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
-  // TMEM columns: S_t at 128 t, O_t at 256 + D t, P_t (packed bf16) at 384 + 64 t.
+  static constexpr int OFF_ONES = OFF_STAGE + NS * STAGE;  // 1024-byte aligned
+  static constexpr int OFF_BAR = OFF_ONES + ONES;
+  // TMEM columns: S_t at 128 t, O_t at 256 + OD t, P_t (packed bf16) at 384 + 64 t.
   static constexpr int T_O = 256, T_P = 384;
+  static_assert(T_O + 2 * OD <= T_P, "TMEM budget");
+  static_assert(OFF_ONES % 1024 == 0, "ones block alignment");
   // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
   // q_empty o_empty[2]
   static constexpr int NBAR = 2 * NS + 13;
@@ -610,7 +633,7 @@ constexpr int kLongSoftPairs = 1;
 // Long regime: a persistent CTA per SM works through units (head, pair of
 // 128-query tiles), each a loop over 128-key tiles.  Each query tile of a unit
 // has its own softmax warpgroup, MMA-issuing warp, S buffer (TMEM columns
-// t*128), O accumulator (TMEM 256 + t*D) and P buffer (TMEM 384 + 64 t); the two
+// t*128), O accumulator (TMEM 256 + t*OD) and P buffer (TMEM 384 + 64 t); the two
 // pipelines run independently and out of phase, so one's exponentials overlap
 // the other's loads, maxima and waits, and each K/V tile serves 256 query rows.
 // Barrier phases run on across units, so the K/V loads and the scores of the
@@ -672,6 +695,14 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     }
     mbar_init(drain_bar, 2);
     fence_mbar_init();
+  }
+  if constexpr (C::LCOL) {
+    // bf16 1.0 everywhere (so the swizzle pattern of the block is immaterial);
+    // the fence makes the stores visible to the tensor core (async proxy).
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::OFF_ONES);
+    for (int i = threadIdx.x; i < C::ONES / 16; i += kLongThreads)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_async_smem();
   }
   if (warp == 8 && lane == 0) {
     tma_prefetch(&mQ);
@@ -756,8 +787,12 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       const int s = itj % NS;
       if (!wait_warp(p_full(t), jtj & 1, g, 15)) return false;
       tc_fence_after();
-      issue_pv_ts<D>(tmem + C::T_O + t * D, tmem + C::T_P + t * 64,
-                     sb + C::OFF_STAGE + s * C::STAGE + C::QB, !first_of_unit);
+      const uint32_t v = sb + C::OFF_STAGE + s * C::STAGE + C::QB;
+      if constexpr (C::LCOL)
+        issue_pv_ts_ones<D>(tmem + C::T_O + t * C::OD, tmem + C::T_P + t * 64, v,
+                            sb + C::OFF_ONES - v, !first_of_unit);
+      else
+        issue_pv_ts<D>(tmem + C::T_O + t * D, tmem + C::T_P + t * 64, v, !first_of_unit);
       umma_commit(pv_done(t));
       umma_commit(kv_empty(s));
       return true;
@@ -793,7 +828,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     const int row = threadIdx.x & 127;   // TMEM lane == query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_tm = tmem + lane_base + t * 128;
-    const uint32_t o_tm = tmem + lane_base + C::T_O + t * D;
+    const uint32_t o_tm = tmem + lane_base + C::T_O + t * C::OD;
     const uint32_t p_tm = tmem + lane_base + C::T_P + t * 64;
     // Scores are accumulator * sl2 in log2 units; the comparator adds its bias
     // to the scaled scores first and then uses a unit factor.
@@ -847,13 +882,21 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         // The P buffer of this tile and O: the previous PV must have finished.
         if (jt >= 1 && !wait_warp(pv_done(t), (jt - 1) & 1, g, 17)) { ok = false; break; }
         tc_fence_after();
-        l += exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
+        if constexpr (C::LCOL) exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
+        else l += exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
         if (fix_o) {
           uint32_t ov[D];
           tmem_ld_cols<D>(o_tm, ov);
 #pragma unroll
           for (int c = 0; c < D; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
           tmem_st_cols<D>(o_tm, ov);
+          if constexpr (C::LCOL) {  // the row-sum columns
+            uint32_t lv[16];
+            tmem_ld_cols<16>(o_tm + D, lv);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) lv[c] = __float_as_uint(__uint_as_float(lv[c]) * alpha);
+            tmem_st_cols<16>(o_tm + D, lv);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -864,6 +907,11 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       tc_fence_after();
       uint32_t ov[D];
       tmem_ld_cols<D>(o_tm, ov);
+      if constexpr (C::LCOL) {
+        uint32_t lv[16];
+        tmem_ld_cols<16>(o_tm + D, lv);
+        l = __uint_as_float(lv[0]);
+      }
       tc_fence_before();
       mbar_arrive(o_empty(t));
       const int q = q0 + t * kTile + row;
