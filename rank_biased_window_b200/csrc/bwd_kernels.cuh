@@ -23,7 +23,8 @@
 //              the partial dQ|dU tile goes to TMEM columns of its own (when
 //              they fit), which the compute warps stage in 128-byte-swizzled
 //              shared memory and add into the fp32 accumulator with TMA bulk
-//              tensor reductions.  The reduction of tile i runs after the
+//              tensor reductions, each warp its own 32 query rows (no barrier
+//              spans a warpgroup).  The reduction of tile i runs after the
 //              softmax of tile i + 1, overlapping tile i + 1's MMAs.  Each
 //              query half (one warpgroup's 64 columns) has barriers of its
 //              own: S^T / dP^T of a half (N = 64 MMAs) and its dV / dK / dW
@@ -212,9 +213,8 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_STG = OFF_DS + NDS * PB;
   static constexpr int OFF_BAR = OFF_STG + NSTG * STG;
-  // kv_full q_full[NS] q_empty[NS] sdp_full[2] ds_full[2] dq_full dq_free drain wg_sync[2]
-  // a_done[2]
-  static constexpr int NBAR = 2 * NS + 12;
+  // kv_full q_full[NS] q_empty[NS] sdp_full[2] ds_full[2] dq_full dq_free drain a_done[2]
+  static constexpr int NBAR = 2 * NS + 10;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(NS >= 1, "shared memory budget");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
@@ -250,9 +250,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t dq_full = bar0 + 8u * (5 + 2 * NS);
   const uint32_t dq_free = bar0 + 8u * (6 + 2 * NS);
   const uint32_t drain_bar = bar0 + 8u * (7 + 2 * NS);
-  // Per-warpgroup barriers (128 arrivals) guarding the dQ staging buffers.
-  auto wg_bar = [&](int w) { return bar0 + 8u * (8 + 2 * NS + w); };
-  auto a_done = [&](int h) { return bar0 + 8u * (10 + 2 * NS + h); };
+  auto a_done = [&](int h) { return bar0 + 8u * (8 + 2 * NS + h); };
   auto ds_buf = [&](int i) { return sb + C::OFF_DS + (C::NDS == 2 ? (i & 1) : 0) * C::PB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -274,7 +272,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int h = 0; h < 2; ++h) {
       mbar_init(sdp_full(h), 1);
       mbar_init(ds_full(h), 128);
-      mbar_init(wg_bar(h), 128);
       mbar_init(a_done(h), 1);
     }
     mbar_init(dq_full, 1);
@@ -458,17 +455,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const bool key_ok = (k0 + row) < N;
     const uint64_t sl2x2 = f2_pack(args.scale_log2, args.scale_log2);
-    const bool leader = (threadIdx.x & 127) == 0;  // issues this warpgroup's reductions
     const uint32_t stg = sb + C::OFF_STG + (C::NSTG == 2 ? wg : 0) * C::STG;
     const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
-    uint32_t wg_phase = 0;
-    // Bounded barrier over this warpgroup's 128 threads.
-    auto wg_sync = [&]() -> bool {
-      mbar_arrive(wg_bar(wg));
-      const bool r = wait_warp(wg_bar(wg), wg_phase & 1u, g, 40);
-      ++wg_phase;
-      return r;
-    };
     // P^T = 2^(S^T s log2e - LSE log2e), dS^T = P^T o (dP^T - D) for this
     // warpgroup's 64 query columns of tile i; P^T and dS^T go back into TMEM in
     // place (packed bf16, columns wg*64 + [0, 32)), dS^T also into shared memory.
@@ -482,12 +470,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // Block wg of this dS buffer staged this warpgroup's first dQ | dU chunk
         // of tile i - 2; the last reductions issued are reduce_dq(i - 2)'s, so
         // only its later chunks (from the staging buffer) may still be read.
+        // A warp writes the same 32 rows of the block that it staged and
+        // reduced, so it waits on its own copies only.
         if (i >= 2) {
-          if (leader) {
+          if (lane == 0) {
             if (my_chunks >= 2) bulk_wait_read<1>();
             else bulk_wait_read<0>();
           }
-          if (!wg_sync()) return false;
+          __syncwarp();
         }
       }
       const int qvalid = N - i * kTile;
@@ -538,8 +528,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     // Partial dQ | dU of tile j (TMEM lane = query row): this warpgroup reads its
     // chunks (wg, wg + 2, ... of 32 columns), frees the TMEM columns, then
-    // stages each chunk in its 128-byte-swizzled buffer and reduces it into the
-    // fp32 accumulator with one TMA bulk tensor reduction.
+    // stages each chunk in its 128-byte-swizzled buffer; each warp adds its 32
+    // rows into the fp32 accumulator with a TMA bulk tensor reduction of its
+    // own (32 x 32 box) issued by its lane 0, whose bulk groups are the only
+    // ones that warp ever waits for.  Rows entirely past N issue no copy but
+    // still commit a (empty) group, so the wait counts hold.
     auto reduce_dq = [&](int j) -> bool {
       if (!wait_warp(dq_full, j & 1, g, 39)) return false;
       tc_fence_after();
@@ -563,11 +556,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // and the reduction staged there earlier was awaited by softmax(j).
           buf = ds_buf(j) + wg * (kTile * 128);
         } else {
-          if (leader) {
+          if (lane == 0) {
             if (C::DEFER) bulk_wait_read<1>();  // only this tile's first chunk may still read
             else bulk_wait_read_all();
           }
-          if (!wg_sync()) return false;
+          __syncwarp();
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -581,9 +574,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        __float_as_uint(v4[1]), __float_as_uint(v4[2]), __float_as_uint(v4[3]));
         }
         fence_async_smem();
-        if (!wg_sync()) return false;
-        if (leader) {
-          tma_reduce_add_3d(&mAcc, buf, ch * 32, j * kTile, bh);
+        __syncwarp();
+        if (lane == 0) {
+          const int wq = (warp & 3) * 32;  // this warp's 32 query rows
+          if (j * kTile + wq < N)
+            tma_reduce_add_3d(&mAcc, buf + wq * 128, ch * 32, j * kTile + wq, bh);
           bulk_commit();
         }
       }
@@ -643,7 +638,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (key_ok) store_o_row<D>(args.dk + r0 * D, gk, args.scale);
       }
     }
-    if (leader) bulk_wait_all();  // reductions complete before the CTA exits
+    if (lane == 0) bulk_wait_all();  // reductions complete before the CTA exits
   }
 
   tc_fence_before();

@@ -217,8 +217,9 @@ int encode_3d_uncached(CUtensorMap* m, const void* ptr, int cols, int N, int BH,
   return rc == CUDA_SUCCESS ? RFB_OK : cuda_fail(static_cast<int>(rc), kSiteEncode);
 }
 
-// 3-D fp32 map over the [BH, N, cols] dQ|dU accumulator, box (32, 128, 1),
-// 128-byte swizzle (32 fp32 per row); used for bulk reductions.
+// 3-D fp32 map over the [BH, N, cols] dQ|dU accumulator, box (32, 32, 1),
+// 128-byte swizzle (32 fp32 per row); used for the bulk reductions, one per
+// warp and chunk (32 query rows each).
 int encode_acc_3d_uncached(CUtensorMap* m, void* ptr, int cols, int N, int BH);
 
 int encode_acc_3d(CUtensorMap* m, void* ptr, int cols, int N, int BH) {
@@ -239,7 +240,7 @@ int encode_acc_3d_uncached(CUtensorMap* m, void* ptr, int cols, int N, int BH) {
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4,
                                  static_cast<cuuint64_t>(cols) * 4 * static_cast<cuuint64_t>(N)};
-  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t box[3] = {32, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult rc = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
