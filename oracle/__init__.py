@@ -20,8 +20,9 @@ The arithmetic of ``fwd`` / ``bwd`` / ``bwd_query_rows`` lives in
 ``rfb_oracle.c`` (plain C, fp64, OpenMP over output rows); this module compiles
 it with gcc and marshals numpy arrays.  Three further definitions are written
 here in plain numpy (fp64, one head at a time): ``fwd_dense_bias`` (the bias
-as a dense matrix), ``factorize_bias`` (best rank-r factors of a dense bias)
-and ``fwd_image_windows`` (shifted-window attention over feature maps).
+as a dense matrix), ``factorize_bias`` (best rank-r factors of a dense bias),
+``fwd_image_windows`` (shifted-window attention over feature maps) and
+``bwd_image_windows`` (its gradients).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against library special
 cases (torch SDPA and autograd in fp64), brute force with ``math.fsum``,
@@ -331,3 +332,56 @@ def fwd_image_windows(q, k, v, u, w, scale, win, shift):
                     O[b, ys, xs, h] = (E @ Vw) / l
                     L[b, ys, xs, h] = (m + np.log(l))[:, 0]
     return (np.roll(O, (shift, shift), axis=(1, 2)), np.roll(L, (shift, shift), axis=(1, 2)))
+
+
+def bwd_image_windows(q, k, v, u, w, dout, scale, win, shift):
+    """Gradients of ``fwd_image_windows`` for an upstream gradient ``dout``
+    ``[B, Hs, Ws, heads, d]``, by the chain rule through the same steps.  The
+    roll and the window cut only move tokens, so every window's gradients are
+    those of its own masked attention, carried back to the tokens' places;
+    ``u, w`` are shared by all windows, so their gradients are sums over the
+    windows.  Per window and head, with P the masked softmax of step 3 (P = 0
+    between regions):
+
+        dP = dO V^T,   D_i = sum_j P_ij dP_ij,   dS = P o (dP - D),
+        dQ = s dS K,   dK = s dS^T Q,   dV = P^T dO,
+        dU[h] += dS W[h],   dW[h] += dS^T U[h].
+
+    Returns ``(dQ, dK, dV, dU, dW)`` in float64; ``dU, dW`` ``[heads, win*win,
+    r]`` or None without factors."""
+    q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    B, Hs, Ws, nh, d = q.shape
+    qs, ks, vs, dos = (np.roll(x, (-shift, -shift), axis=(1, 2)) for x in (q, k, v, do))
+    ry, rx = _shift_regions(Hs, win, shift), _shift_regions(Ws, win, shift)
+    dQ, dK, dV = np.zeros_like(qs), np.zeros_like(qs), np.zeros_like(qs)
+    uu = None if u is None else np.asarray(u, dtype=np.float64)
+    ww = None if w is None else np.asarray(w, dtype=np.float64)
+    dU = None if uu is None else np.zeros_like(uu)
+    dW = None if ww is None else np.zeros_like(ww)
+    for b in range(B):
+        for y0 in range(0, Hs, win):
+            for x0 in range(0, Ws, win):
+                ys, xs = np.meshgrid(np.arange(y0, y0 + win), np.arange(x0, x0 + win), indexing="ij")
+                ys, xs = ys.reshape(-1), xs.reshape(-1)           # raster order in the window
+                region = 3 * ry[ys] + rx[xs]
+                allowed = region[:, None] == region[None, :]
+                for h in range(nh):
+                    Qw, Kw, Vw = qs[b, ys, xs, h], ks[b, ys, xs, h], vs[b, ys, xs, h]
+                    dOw = dos[b, ys, xs, h]
+                    S = scale * (Qw @ Kw.T)
+                    if uu is not None:
+                        S = S + uu[h] @ ww[h].T
+                    S = np.where(allowed, S, -np.inf)
+                    E = np.exp(S - S.max(axis=1, keepdims=True))
+                    P = E / E.sum(axis=1, keepdims=True)
+                    dP = dOw @ Vw.T
+                    Dv = (P * dP).sum(axis=1, keepdims=True)
+                    dS = P * (dP - Dv)
+                    dQ[b, ys, xs, h] = scale * (dS @ Kw)
+                    dK[b, ys, xs, h] = scale * (dS.T @ Qw)
+                    dV[b, ys, xs, h] = P.T @ dOw
+                    if uu is not None:
+                        dU[h] += dS @ ww[h]
+                        dW[h] += dS.T @ uu[h]
+    back = lambda x: np.roll(x, (shift, shift), axis=(1, 2))
+    return back(dQ), back(dK), back(dV), dU, dW

@@ -63,3 +63,74 @@ def test_interior_shifted_window_needs_no_mask():
     P = np.exp(S - S.max(1, keepdims=True))
     want = (P @ V) / P.sum(1, keepdims=True)
     np.testing.assert_allclose(o[0, 12:20, 12:20, 0].reshape(64, d), want, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ backward
+
+def test_backward_finite_differences_shifted():
+    """Central differences of L = sum(dO o O) through the oracle's own forward,
+    on a 16 x 16 map shifted by 4 (masked windows in the last row and column)."""
+    B, Hs, Ws, nh, d, r = 1, 16, 16, 2, 4, 2
+    q, k, v, u, w = _maps(B, Hs, Ws, nh, d, r, seed=21)
+    rng = np.random.default_rng(5)
+    do = rng.standard_normal(q.shape)
+    s, shift = 0.45, 4
+    grads = oracle.bwd_image_windows(q, k, v, u, w, do, s, 8, shift)
+    args = [q, k, v, u, w]
+
+    def loss(a):
+        o, _ = oracle.fwd_image_windows(*a, s, 8, shift)
+        return float((do * o).sum())
+
+    h = 1e-6
+    for t, g in enumerate(grads):
+        flat = args[t].reshape(-1)
+        for idx in rng.choice(flat.size, size=10, replace=False):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[t].reshape(-1)[idx] += h
+            minus[t].reshape(-1)[idx] -= h
+            fd = (loss(plus) - loss(minus)) / (2 * h)
+            an = g.reshape(-1)[idx]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (t, idx, fd, an)
+
+
+def test_backward_unshifted_equals_factored_oracle_on_partitioned_windows():
+    """Without a shift: the C oracle's backward on windows cut by reshapes, with
+    the shared factors' gradients summed over the windows."""
+    B, Hs, Ws, nh, d, r = 2, 16, 8, 2, 8, 4
+    q, k, v, u, w = _maps(B, Hs, Ws, nh, d, r, seed=22)
+    do = np.random.default_rng(6).standard_normal(q.shape)
+    dq, dk, dv, du, dw = oracle.bwd_image_windows(q, k, v, u, w, do, 0.35, 8, 0)
+
+    def part(x):
+        c = x.shape[-1]
+        x = x.reshape(B, Hs // 8, 8, Ws // 8, 8, nh, c).transpose(0, 1, 3, 5, 2, 4, 6)
+        return x.reshape(-1, nh, 64, c)
+
+    nw = B * (Hs // 8) * (Ws // 8)
+    ub = np.broadcast_to(u[None], (nw, nh, 64, r)).copy()
+    wb = np.broadcast_to(w[None], (nw, nh, 64, r)).copy()
+    rq, rk, rv, ru, rw = oracle.bwd(part(q), part(k), part(v), ub, wb, part(do), 0.35)
+    for got, want in ((dq, rq), (dk, rk), (dv, rv)):
+        np.testing.assert_allclose(part(got), want, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(du, ru.sum(axis=0), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dw, rw.sum(axis=0), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_shift_on_one_window_is_four_region_backwards():
+    """An 8 x 8 map shifted by 4: the gradients of each 4 x 4 block are those of
+    plain attention inside the block (the C oracle on 16 tokens)."""
+    nh, d = 2, 8
+    q, k, v, _, _ = _maps(1, 8, 8, nh, d, 0, seed=23)
+    do = np.random.default_rng(7).standard_normal(q.shape)
+    dq, dk, dv, _, _ = oracle.bwd_image_windows(q, k, v, None, None, do, 0.5, 8, 4)
+    for y0 in (0, 4):
+        for x0 in (0, 4):
+            for h in range(nh):
+                sl = (0, slice(y0, y0 + 4), slice(x0, x0 + 4), h)
+                blk = [t[sl].reshape(1, 1, 16, d) for t in (q, k, v, do)]
+                rq, rk, rv, _, _ = oracle.bwd(blk[0], blk[1], blk[2], None, None, blk[3], 0.5)
+                for got, want in ((dq, rq), (dk, rk), (dv, rv)):
+                    np.testing.assert_allclose(got[sl].reshape(16, d), want[0, 0], rtol=1e-10,
+                                               atol=1e-12)
