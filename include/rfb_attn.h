@@ -21,8 +21,8 @@
  *
  * Entry points: the per-window forward / backward (rfb_attn_fwd,
  * rfb_attn_bwd, rfb_attn_bwd_noalloc); variants with one factor pair per head
- * shared by all windows (rfb_attn_*_shared_bias); shifted-window attention read
- * straight from feature maps (rfb_attn_fwd_image_windows); a dense-bias
+ * shared by all windows (rfb_attn_*_shared_bias); shifted-window attention on
+ * feature maps (rfb_attn_fwd_image_windows, rfb_attn_bwd_image_windows); a dense-bias
  * comparator (rfb_attn_fwd_dense_bias); diagnostics.  Each declaration below
  * states what differs from these conventions.
  *
@@ -221,6 +221,43 @@ RFB_API int rfb_attn_fwd_image_windows(const void* q, const void* k, const void*
                                        const void* u, const void* w, void* o, float* lse, int B,
                                        int img_h, int img_w, int heads, int d, int r, int win,
                                        int shift, float scale, void* stream);
+
+/*
+ * Backward of rfb_attn_fwd_image_windows: dQ, dK, dV at the tokens' map
+ * positions and dU, dW of the shared factors, summed over all windows (the
+ * chain rule through the roll, the window cut and the masked window
+ * attention; the mask gives P = 0 between regions).  The maps are gathered
+ * into window tensors (the rolled window cut, raster order inside each
+ * window) in the workspace, the shared-factor backward runs on them with the
+ * shifted-window mask, and dQ, dK, dV are scattered back.
+ *   q, k, v, o, dout   : [B, img_h, img_w, heads, d] bf16; o and lse as
+ *                        written by rfb_attn_fwd_image_windows for the same
+ *                        inputs, win and shift.
+ *   u, w               : [heads, win*win, r] bf16 (raster position in the
+ *                        window); NULL iff r == 0.
+ *   lse                : [B, img_h, img_w, heads] fp32.
+ *   dq, dk, dv         : [B, img_h, img_w, heads, d] bf16 outputs.
+ *   du, dw             : [heads, win*win, r] bf16 outputs (fp32 sums over the
+ *                        windows, rounded once); NULL iff r == 0.
+ *   workspace          : device, 16-byte aligned, at least
+ *                        rfb_attn_bwd_image_windows_workspace_size() bytes
+ *                        (eight bf16 window tensors, the gathered LSE and the
+ *                        shared-factor backward's workspace); the caller owns
+ *                        it and may reuse it once the call has completed on
+ *                        the stream.
+ *   win = 8, shift = 0 or 4, img_h and img_w multiples of 8.
+ * Errors as rfb_attn_bwd_shared_bias; RFB_ERR_UNSUPPORTED for other win /
+ * shift / map sizes.
+ */
+RFB_API size_t rfb_attn_bwd_image_windows_workspace_size(int B, int img_h, int img_w, int heads,
+                                                         int d, int r);
+RFB_API int rfb_attn_bwd_image_windows(const void* q, const void* k, const void* v,
+                                       const void* u, const void* w, const void* o,
+                                       const float* lse, const void* dout, void* dq, void* dk,
+                                       void* dv, void* du, void* dw, void* workspace,
+                                       size_t workspace_bytes, int B, int img_h, int img_w,
+                                       int heads, int d, int r, int win, int shift, float scale,
+                                       void* stream);
 
 /* Human-readable text for a status code (static storage). */
 RFB_API const char* rfb_strerror(int status);

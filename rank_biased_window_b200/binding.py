@@ -37,6 +37,9 @@ SIGNATURES = {
     "rfb_attn_bwd_shared_bias_workspace_size": (_sz, [_i] * 5),
     "rfb_attn_fwd_dense_bias": (_i, [_vp] * 5 + [_fp] + [_i] * 5 + [_f, _vp]),
     "rfb_attn_fwd_image_windows": (_i, [_vp] * 6 + [_fp] + [_i] * 8 + [_f, _vp]),
+    "rfb_attn_bwd_image_windows_workspace_size": (_sz, [_i] * 6),
+    "rfb_attn_bwd_image_windows": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 8
+                                   + [_f, _vp]),
     "rfb_attn_bwd_shared_bias": (_i, [_vp] * 6 + [_fp] + [_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp]),
     "rfb_strerror": (ctypes.c_char_p, [_i]),
     "rfb_last_device_error": (_i, []),
@@ -294,6 +297,50 @@ def attn_fwd_image_windows(q, k, v, u=None, w=None, scale=None, *, win=8, shift=
             int(shift), s, _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_fwd_image_windows")
     return o, l
+
+
+def bwd_image_windows_workspace_size(B, img_h, img_w, heads, d, r) -> int:
+    return int(load_library().rfb_attn_bwd_image_windows_workspace_size(B, img_h, img_w, heads,
+                                                                         d, r))
+
+
+def attn_bwd_image_windows(q, k, v, u, w, o, lse, dout, scale=None, *, win=8, shift=0,
+                           workspace=None, grads=None, stream=None):
+    """Backward of attn_fwd_image_windows: dQ, dK, dV [B, H, W, heads, d] at
+    the tokens' map positions and dU, dW [heads, win*win, r] summed over all
+    windows (None when r == 0)."""
+    if q.dim() != 5:
+        raise ValueError("q must be [B, H, W, heads, d]")
+    B, Hs, Ws, nh, d = (int(x) for x in q.shape)
+    r = 0 if u is None else int(u.shape[-1])
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_operand(name, t, (B, Hs, Ws, nh, d), dev)
+    if r > 0:
+        _check_operand("u", u, (nh, win * win, r), dev)
+        _check_operand("w", w, (nh, win * win, r), dev)
+    else:
+        u = w = None
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hs, Ws, nh) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, W, heads]")
+    s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    if grads is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        du = torch.empty_like(u) if r else None
+        dw = torch.empty_like(w) if r else None
+    else:
+        dq, dk, dv, du, dw = grads
+    nbytes = bwd_image_windows_workspace_size(B, Hs, Ws, nh, d, r)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    with _on_device(dev):
+        rc = load_library().rfb_attn_bwd_image_windows(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
+            ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, Hs, Ws, nh, d,
+            r, int(win), int(shift), s, _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_bwd_image_windows")
+    return dq, dk, dv, du, dw
 
 
 def bwd_shared_bias_workspace_size(B, H, N, d, r) -> int:

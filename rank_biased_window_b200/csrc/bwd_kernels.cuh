@@ -61,7 +61,51 @@ struct BwdArgs {
   float scale_log2;  // s log2(e)
   float inv_scale;   // 1/s
   uint64_t timeout_ns;
+  // Shifted-window mask of image windows (N = 64, tokens in raster order
+  // inside each 8 x 8 window; 0 = no mask): window-head bh is window
+  // (bh / mask_heads) of a map of mask_nwy x mask_nwx windows per image.
+  int mask_shift, mask_nwx, mask_nwy, mask_heads;
 };
+
+// Image windows <-> window tensors.  Window-head bh = ((b * nwy + wy) * nwx +
+// wx) * heads + h, token n = 8 ty + tx (raster order inside the window) is the
+// map token (b, (8 wy + ty + shift) mod img_h, (8 wx + tx + shift) mod img_w)
+// of head h: the window cut of the map rolled by (-shift, -shift).  Moves
+// `ntensor` bf16 tensors (and optionally the fp32 LSE) between the map layout
+// [B, img_h, img_w, heads, d] and the window layout [BH, 64, d], in either
+// direction; every position is written exactly once.
+struct ImgMoveArgs {
+  const __nv_bfloat16* src[5];
+  __nv_bfloat16* dst[5];
+  const float* lse_src;  // NULL: no LSE to move
+  float* lse_dst;
+  int ntensor, BH, img_h, img_w, heads, d, shift;
+  int to_windows;  // 1: maps -> windows, 0: windows -> maps
+};
+
+__global__ void __launch_bounds__(256) img_move_kernel(const ImgMoveArgs a) {
+  const int G = a.d / 8;  // 16-byte pieces per token row
+  const long long total = static_cast<long long>(a.BH) * 64 * G;
+  const int nwx = a.img_w / 8, nwy = a.img_h / 8;
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int g = static_cast<int>(t % G);
+    const long long wrow = t / G;  // bh * 64 + n
+    const int n = static_cast<int>(wrow % 64);
+    const int bh = static_cast<int>(wrow / 64);
+    const int h = bh % a.heads, bw = bh / a.heads;
+    const int wx = bw % nwx, wy = (bw / nwx) % nwy, b = bw / (nwx * nwy);
+    const int y = (wy * 8 + (n >> 3) + a.shift) % a.img_h;
+    const int x = (wx * 8 + (n & 7) + a.shift) % a.img_w;
+    const long long mrow = ((static_cast<long long>(b) * a.img_h + y) * a.img_w + x) * a.heads + h;
+    const long long srow = a.to_windows ? mrow : wrow, drow = a.to_windows ? wrow : mrow;
+    for (int i = 0; i < a.ntensor; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(a.src[i] + srow * a.d)[g];
+      reinterpret_cast<uint4*>(a.dst[i] + drow * a.d)[g] = v;
+    }
+    if (g == 0 && a.lse_src != nullptr) a.lse_dst[drow] = a.lse_src[srow];
+  }
+}
 
 // ------------------------------------------------------------------ bwd_pre
 // Thread group of G = D/8 lanes per row (16-byte loads); rows grid-strided.
@@ -456,6 +500,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool key_ok = (k0 + row) < N;
     const uint64_t sl2x2 = f2_pack(args.scale_log2, args.scale_log2);
     const uint32_t stg = sb + C::OFF_STG + (C::NSTG == 2 ? wg : 0) * C::STG;
+    // Shifted-window mask: in the last window row (column) of a shifted map the
+    // top and bottom (left and right) 4-token halves are different regions, so
+    // key k and query q interact only if ((k ^ q) & mask_bits) == 0 (bit 5 of
+    // the raster index selects the half of rows, bit 2 the half of columns).
+    int mask_bits = 0;
+    if (args.mask_shift > 0) {
+      const int bw = bh / args.mask_heads;
+      const int wx = bw % args.mask_nwx, wy = (bw / args.mask_nwx) % args.mask_nwy;
+      mask_bits = (wy == args.mask_nwy - 1 ? 32 : 0) | (wx == args.mask_nwx - 1 ? 4 : 0);
+    }
     const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
     // P^T = 2^(S^T s log2e - LSE log2e), dS^T = P^T o (dP^T - D) for this
     // warpgroup's 64 query columns of tile i; P^T and dS^T go back into TMEM in
@@ -491,6 +545,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (!key_ok || c + e >= qvalid) xy[e] = 0xFF800000u;
+        }
+        if (mask_bits != 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if ((((k0 + row) ^ (i * kTile + c + e)) & mask_bits) != 0) xy[e] = 0xFF800000u;
         }
         uint32_t pk[16], dk[16];
 #pragma unroll

@@ -570,7 +570,8 @@ namespace {
 int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, const void* w,
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
                   void* dv, void* du, void* dw, void* workspace, size_t workspace_bytes, int B,
-                  int H, int N, int d, int r, float scale, void* stream, bool shared) {
+                  int H, int N, int d, int r, float scale, void* stream, bool shared,
+                  const int* img_mask = nullptr) {
   bool empty = false;
   if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
   if (empty) return RFB_OK;
@@ -631,6 +632,11 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
   a.timeout_ns = kWaitTimeoutNs;
+  // img_mask = {shift, windows per map row, windows per map column, heads}
+  a.mask_shift = img_mask ? img_mask[0] : 0;
+  a.mask_nwx = img_mask ? img_mask[1] : 1;
+  a.mask_nwy = img_mask ? img_mask[2] : 1;
+  a.mask_heads = img_mask ? img_mask[3] : 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long rows = static_cast<long long>(BH) * L.npad;
   {
@@ -650,6 +656,46 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
     }
   }
   return launch_status();
+}
+
+// Image-window backward workspace: the eight window tensors (Q, K, V, O, dO
+// gathered; dQ, dK, dV before their scatter), the gathered LSE, then the
+// shared-factor backward's own workspace.
+struct ImgWsLayout {
+  size_t win[8], lse, inner, total;
+};
+
+ImgWsLayout img_ws_layout(long long BH, int heads, int d, int r) {
+  ImgWsLayout L;
+  const size_t t = align256(static_cast<size_t>(BH) * 64 * d * 2);
+  size_t off = 0;
+  for (int i = 0; i < 8; ++i) {
+    L.win[i] = off;
+    off += t;
+  }
+  L.lse = off;
+  off += align256(static_cast<size_t>(BH) * 64 * sizeof(float));
+  L.inner = off;
+  off += ws_layout(static_cast<int>(BH / heads), heads, 64, d, r, true).total;
+  L.total = off;
+  return L;
+}
+
+// Shape checks shared by the image-window entry points; *bh receives the
+// number of window-heads (0: nothing to do).
+int check_image_windows(int B, int img_h, int img_w, int heads, int d, int r, int win, int shift,
+                        float scale, long long* bh) {
+  bool empty = false;
+  *bh = 0;
+  if (int rc = check_shape(B, heads, 64, d, r, scale, &empty)) return rc;
+  if (B < 0 || img_h < 0 || img_w < 0) return RFB_ERR_INVALID_ARG;
+  if (win != 8 || (shift != 0 && shift != 4)) return RFB_ERR_UNSUPPORTED;
+  if (img_h % 8 != 0 || img_w % 8 != 0) return RFB_ERR_UNSUPPORTED;
+  if (empty || img_h == 0 || img_w == 0) return RFB_OK;
+  const long long n = static_cast<long long>(B) * (img_h / 8) * (img_w / 8) * heads;
+  if (n > 0x7fffffffLL / 64) return RFB_ERR_UNSUPPORTED;
+  *bh = n;
+  return RFB_OK;
 }
 }  // namespace
 }  // namespace rfb
@@ -796,6 +842,84 @@ int rfb_attn_bwd_shared_bias(const void* q, const void* k, const void* v, const 
                              float scale, void* stream) {
   return attn_bwd_impl(q, k, v, u, w, o, lse, dout, dq, dk, dv, du, dw, workspace,
                        workspace_bytes, B, H, N, d, r, scale, stream, true);
+}
+
+size_t rfb_attn_bwd_image_windows_workspace_size(int B, int img_h, int img_w, int heads, int d,
+                                                  int r) {
+  long long bh = 0;
+  if (check_image_windows(B, img_h, img_w, heads, d, r, 8, 0, 1.0f, &bh) != RFB_OK || bh == 0)
+    return 0;
+  return img_ws_layout(bh, heads, d, r).total;
+}
+
+int rfb_attn_bwd_image_windows(const void* q, const void* k, const void* v, const void* u,
+                               const void* w, const void* o, const float* lse, const void* dout,
+                               void* dq, void* dk, void* dv, void* du, void* dw, void* workspace,
+                               size_t workspace_bytes, int B, int img_h, int img_w, int heads,
+                               int d, int r, int win, int shift, float scale, void* stream) {
+  long long bh = 0;
+  if (int rc = check_image_windows(B, img_h, img_w, heads, d, r, win, shift, scale, &bh))
+    return rc;
+  if (bh == 0) return RFB_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv ||
+      (r > 0 && (!u || !w || !du || !dw)))
+    return RFB_ERR_INVALID_ARG;
+  const void* all[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void* p : all)
+    if (!aligned16(p)) return RFB_ERR_ALIGNMENT;
+  const ImgWsLayout L = img_ws_layout(bh, heads, d, r);
+  if (!workspace || workspace_bytes < L.total) return RFB_ERR_WORKSPACE;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto wt = [&](int i) { return reinterpret_cast<__nv_bfloat16*>(ws + L.win[i]); };
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long pieces = bh * 64 * (d / 8);
+  // 1. maps -> windows: Q, K, V, O, dO and the LSE.
+  ImgMoveArgs g;
+  std::memset(&g, 0, sizeof(g));
+  const void* srcs[5] = {q, k, v, o, dout};
+  for (int i = 0; i < 5; ++i) {
+    g.src[i] = static_cast<const __nv_bfloat16*>(srcs[i]);
+    g.dst[i] = wt(i);
+  }
+  g.lse_src = lse;
+  g.lse_dst = reinterpret_cast<float*>(ws + L.lse);
+  g.ntensor = 5;
+  g.BH = static_cast<int>(bh);
+  g.img_h = img_h;
+  g.img_w = img_w;
+  g.heads = heads;
+  g.d = d;
+  g.shift = shift;
+  g.to_windows = 1;
+  img_move_kernel<<<grid_for(pieces, 256, dev.sms), 256, 0, st>>>(g);
+  if (int rc = launch_status()) return rc;
+  // 2. the shared-factor backward on the windows, with the shifted-window mask.
+  const int mask[4] = {shift, img_w / 8, img_h / 8, heads};
+  const int nwin = static_cast<int>(bh / heads);
+  if (int rc = attn_bwd_impl(wt(0), wt(1), wt(2), u, w, wt(3), reinterpret_cast<float*>(ws + L.lse),
+                             wt(4), wt(5), wt(6), wt(7), du, dw, ws + L.inner, L.total - L.inner,
+                             nwin, heads, 64, d, r, scale, stream, true, mask))
+    return rc;
+  // 3. windows -> maps: dQ, dK, dV.
+  ImgMoveArgs sc;
+  std::memset(&sc, 0, sizeof(sc));
+  void* dsts[3] = {dq, dk, dv};
+  for (int i = 0; i < 3; ++i) {
+    sc.src[i] = wt(5 + i);
+    sc.dst[i] = static_cast<__nv_bfloat16*>(dsts[i]);
+  }
+  sc.ntensor = 3;
+  sc.BH = static_cast<int>(bh);
+  sc.img_h = img_h;
+  sc.img_w = img_w;
+  sc.heads = heads;
+  sc.d = d;
+  sc.shift = shift;
+  sc.to_windows = 0;
+  img_move_kernel<<<grid_for(pieces, 256, dev.sms), 256, 0, st>>>(sc);
+  return launch_status();
 }
 
 int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* u,

@@ -114,6 +114,30 @@ def test_image_windows_host_checks(rfb_lib):
     assert f(n, n, n, n, n, n, n, 1, 16, 16, 2, 32, 8, 8, 4, 0.0, n) == 1   # scale
 
 
+def test_image_windows_backward_host_checks(rfb_lib):
+    lib = rfb_lib.load_library()
+    n = None
+    f = lib.rfb_attn_bwd_image_windows
+    size = lib.rfb_attn_bwd_image_windows_workspace_size
+    # 8 pointers, 5 outputs, workspace, bytes, B, img_h, img_w, heads, d, r, win, shift, scale
+    args = lambda B, Hs, Ws, d, win, shift, scale, ws=0: (
+        [n] * 13 + [n, ws, B, Hs, Ws, 2, d, 8, win, shift, scale, n])
+    assert f(*args(0, 16, 16, 32, 8, 0, 0.1)) == 0        # empty
+    assert f(*args(1, 16, 16, 32, 16, 0, 0.1)) == 2       # window 16
+    assert f(*args(1, 16, 16, 32, 8, 2, 0.1)) == 2        # shift 2
+    assert f(*args(1, 12, 16, 32, 8, 4, 0.1)) == 2        # 12 rows
+    assert f(*args(1, 16, 16, 48, 8, 4, 0.1)) == 2        # d
+    assert f(*args(1, 16, 16, 32, 8, 4, 0.1)) == 1        # null pointers
+    assert f(*args(1, 16, 16, 32, 8, 4, 0.0)) == 1        # scale
+    # workspace: eight bf16 window tensors, the LSE and the shared-factor backward's
+    nwin, heads, d, r = 2 * 2 * 3, 2, 32, 8
+    base = lib.rfb_attn_bwd_shared_bias_workspace_size(nwin, heads, 64, d, r)
+    t = -(-(nwin * heads * 64 * d * 2) // 256) * 256
+    lse = -(-(nwin * heads * 64 * 4) // 256) * 256
+    assert size(2, 16, 24, heads, d, r) == 8 * t + lse + base
+    assert size(0, 16, 24, heads, d, r) == 0 and size(1, 12, 24, heads, d, r) == 0
+
+
 def test_bench_accounting_helpers(tmp_path, monkeypatch):
     """bench.py's algorithmic flop / byte counts and the traffic record's
     source-hash gate."""

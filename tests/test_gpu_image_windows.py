@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from rank_biased_window_b200.inputs import make_inputs, to_f64
-from tests._parity import assert_close
+from tests._parity import MAX_ABS, assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -74,3 +74,43 @@ def test_image_windows_reject_unsupported(rfb_lib, cuda_dev):
     q, k, v, u, w = (t.to(cuda_dev) for t in _maps(1, 16, 16, 2, 32, 8, seed=2))
     with pytest.raises(RuntimeError, match="unsupported"):
         rfb_lib.attn_fwd_image_windows(q, k, v, u, w, shift=2)
+
+
+BWD_CASES = [
+    (2, 16, 24, 3, 32, 16, 0),
+    (2, 16, 24, 3, 32, 16, 4),   # masks in the last window row and column
+    (1, 8, 8, 2, 64, 8, 4),      # one window: four regions
+    (1, 24, 16, 6, 32, 8, 4),    # SwinIR-like heads
+    (2, 16, 16, 1, 64, 0, 4),    # no bias
+    (1, 16, 16, 2, 64, 32, 4),
+]
+
+
+@pytest.mark.parametrize("shape", BWD_CASES, ids=[f"B{b}H{hs}W{ws}h{nh}d{d}r{r}s{sh}"
+                                                  for b, hs, ws, nh, d, r, sh in BWD_CASES])
+def test_image_windows_backward_match_oracle(rfb_lib, oracle_mod, cuda_dev, shape):
+    B, Hs, Ws, nh, d, r, shift = shape
+    q, k, v, u, w = _maps(B, Hs, Ws, nh, d, r, seed=8300 + Hs + Ws + d + r + shift)
+    g = torch.Generator().manual_seed(8400 + Hs + d + shift)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    s = 1.0 / math.sqrt(d)
+    dev = lambda t: None if t is None else t.to(cuda_dev)
+    o, lse = rfb_lib.attn_fwd_image_windows(dev(q), dev(k), dev(v), dev(u), dev(w), s,
+                                            shift=shift)
+    got = rfb_lib.attn_bwd_image_windows(dev(q), dev(k), dev(v), dev(u), dev(w), o, lse, dev(do),
+                                         s, shift=shift)
+    torch.cuda.synchronize()
+    assert rfb_lib.last_device_error() == 0
+    f = lambda t: None if t is None else to_f64(t)
+    want = oracle_mod.bwd_image_windows(f(q), f(k), f(v), f(u), f(w), f(do), s, 8, shift)
+    for name, a, b in zip(("dQ", "dK", "dV", "dU", "dW"), got, want):
+        if b is None:
+            assert a is None
+            continue
+        # dU, dW are sums over all windows of a map (magnitudes up to ~8 here):
+        # the bf16 operands of the tensor-core products (dS, U', W) and the bf16
+        # output each carry a relative error of 2^-9, so the absolute bound, set
+        # for outputs of order 1, is scaled to one bf16 step at the largest
+        # magnitude (2^-7 max|x|); the rel-L2 bound is unchanged.
+        ma = MAX_ABS if name in ("dQ", "dK", "dV") else max(MAX_ABS, 2.0 ** -7 * np.abs(b).max())
+        assert_close(name, a, b, max_abs=ma)
