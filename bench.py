@@ -57,6 +57,10 @@ def parse_args():
     ap.add_argument("--shared-bias", action="store_true",
                     help="one U, W pair per head shared by all windows; with several "
                          "ranks dU, dW are all-reduced (NCCL) inside the step")
+    ap.add_argument("--image-windows", action="store_true",
+                    help="shifted-window attention on feature maps (SwinIR-sized: 4 maps of "
+                         "128 x 128 tokens, 6 heads, d = 32, r = 8, 8 x 8 windows, shift 4), "
+                         "forward + backward from the maps")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall seconds of the CPU-baseline sample")
     return ap.parse_args()
@@ -303,6 +307,67 @@ def run_factorize(args, wl, rank):
     print(json.dumps(line))
 
 
+def run_image_windows(args, rank):
+    """Forward + backward of shifted-window attention read from channels-last
+    maps (attn_fwd_image_windows, attn_bwd_image_windows), L2 flushed clean
+    before every step; flops as the window workload's (N = 64 per window)."""
+    import torch
+    import rank_biased_window_b200 as rfb
+    if rank != 0:
+        return
+    B, Hs, Ws, nh, d, r, shift = 4, 128, 128, 6, 32, 8, 4
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(20260306)
+    mk = lambda *shape, std=1.0: (torch.randn(shape, generator=g) * std).to(torch.bfloat16).to(dev)
+    q, k, v, do = (mk(B, Hs, Ws, nh, d) for _ in range(4))
+    u, w = mk(nh, 64, r, std=r ** -0.5), mk(nh, 64, r, std=r ** -0.5)
+    s = d ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hs, Ws, nh), dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(u),
+             torch.empty_like(w))
+    ws = torch.empty(rfb.bwd_image_windows_workspace_size(B, Hs, Ws, nh, d, r), dtype=torch.uint8,
+                     device=dev)
+    fwd = lambda: rfb.attn_fwd_image_windows(q, k, v, u, w, s, shift=shift, out=o, lse=lse)
+    bwd = lambda: rfb.attn_bwd_image_windows(q, k, v, u, w, o, lse, do, s, shift=shift,
+                                             workspace=ws, grads=grads)
+    for _ in range(max(args.warmup, 3)):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    assert rfb.last_device_error() == 0
+    flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev)
+    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        flush_sum.copy_(flush.view(torch.float32).sum())
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        fwd()
+        e[1].record()
+        bwd()
+        e[2].record()
+        evs.append(e)
+    torch.cuda.synchronize(dev)
+    t_f = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_b = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    BH, N = B * (Hs // 8) * (Ws // 8) * nh, 64
+    fl_f = 2.0 * BH * N * N * (2 * d + r)
+    fl_b = 2.0 * BH * N * N * (5 * d + 3 * r)
+    line = {"metric": "shifted-window attention on maps, fwd+bwd TFLOP/s (bf16)",
+            "value": (fl_f + fl_b) / ((t_f + t_b) * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "higher_is_better": True, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_f + t_b, "fwd_ms": t_f, "bwd_ms": t_b,
+            "windows_per_s": B * (Hs // 8) * (Ws // 8) / ((t_f + t_b) * 1e-3),
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) maps, N(0,1/r) factors)",
+            "config": {"workload": "image windows", "B": B, "img_h": Hs, "img_w": Ws,
+                       "heads": nh, "d": d, "r": r, "win": 8, "shift": shift,
+                       "l2": "flushed clean before every step"}}
+    print(json.dumps(line))
+
+
 def main():
     args = parse_args()
     from rank_biased_window_b200.inputs import WORKLOADS, workload_inputs
@@ -318,6 +383,8 @@ def main():
     from rank_biased_window_b200 import build as rfb_build
     if args.factorize:
         return run_factorize(args, wl, rank)
+    if args.image_windows:
+        return run_image_windows(args, rank)
 
     dist = None
     if world > 1:

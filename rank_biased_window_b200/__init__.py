@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     LIB_PATH,
     RFBAttention,
     RFBAttentionSharedBias,
+    RFBImageWindows,
     allreduce_bias_grads,
     attn_bwd,
     attn_bwd_image_windows,
@@ -26,6 +27,7 @@ from .binding import (  # noqa: F401
     profile_enable,
     profile_read,
     rfb_attention,
+    rfb_attention_image_windows,
     rfb_attention_shared_bias,
     selftest_wait_timeout,
     strerror,
@@ -35,6 +37,7 @@ from .factorize import factorize_bias, relative_position_bias  # noqa: F401
 __all__ = ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "bwd_workspace_size", "rfb_attention", "RFBAttention",
            "attn_fwd_shared_bias", "attn_fwd_dense_bias", "attn_fwd_image_windows", "attn_bwd_image_windows",
            "bwd_image_windows_workspace_size", "attn_bwd_shared_bias", "bwd_shared_bias_workspace_size",
-           "rfb_attention_shared_bias", "RFBAttentionSharedBias", "allreduce_bias_grads",
+           "rfb_attention_shared_bias", "RFBAttentionSharedBias",
+           "rfb_attention_image_windows", "RFBImageWindows", "allreduce_bias_grads",
            "factorize_bias", "relative_position_bias",
            "last_device_error", "selftest_wait_timeout", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]

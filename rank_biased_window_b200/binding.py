@@ -511,6 +511,25 @@ class RFBAttentionSharedBias(torch.autograd.Function):
         return dq, dk, dv, du, dw, None
 
 
+class RFBImageWindows(torch.autograd.Function):
+    """Autograd wrapper for shifted-window attention on maps q, k, v [B, H, W,
+    heads, d] with shared factors u, w [heads, 64, r]."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, u, w, scale, shift):
+        o, lse = attn_fwd_image_windows(q, k, v, u, w, scale, shift=shift)
+        ctx.save_for_backward(q, k, v, u, w, o, lse)
+        ctx.scale, ctx.shift = scale, shift
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, u, w, o, lse = ctx.saved_tensors
+        dq, dk, dv, du, dw = attn_bwd_image_windows(q, k, v, u, w, o, lse, dout.contiguous(),
+                                                    ctx.scale, shift=ctx.shift)
+        return dq, dk, dv, du, dw, None, None
+
+
 def rfb_attention(q, k, v, u, w, scale=None):
     s = (1.0 / math.sqrt(q.shape[-1])) if scale is None else float(scale)
     return RFBAttention.apply(q, k, v, u, w, s)
@@ -520,3 +539,10 @@ def rfb_attention_shared_bias(q, k, v, u, w, scale=None):
     """As rfb_attention with u, w [H, N, r] shared by all windows."""
     s = (1.0 / math.sqrt(q.shape[-1])) if scale is None else float(scale)
     return RFBAttentionSharedBias.apply(q, k, v, u, w, s)
+
+
+def rfb_attention_image_windows(q, k, v, u, w, scale=None, shift=0):
+    """Shifted-window attention (8 x 8 windows, shift 0 or 4) on feature maps,
+    differentiable in q, k, v, u, w."""
+    s = (1.0 / math.sqrt(q.shape[-1])) if scale is None else float(scale)
+    return RFBImageWindows.apply(q, k, v, u, w, s, int(shift))

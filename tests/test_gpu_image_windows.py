@@ -114,3 +114,19 @@ def test_image_windows_backward_match_oracle(rfb_lib, oracle_mod, cuda_dev, shap
         # magnitude (2^-7 max|x|); the rel-L2 bound is unchanged.
         ma = MAX_ABS if name in ("dQ", "dK", "dV") else max(MAX_ABS, 2.0 ** -7 * np.abs(b).max())
         assert_close(name, a, b, max_abs=ma)
+
+
+def test_image_windows_autograd(rfb_lib, oracle_mod, cuda_dev):
+    """Gradients through torch autograd (both passes run the CUDA kernels)."""
+    B, Hs, Ws, nh, d, r, shift = 1, 16, 24, 2, 32, 16, 4
+    q, k, v, u, w = _maps(B, Hs, Ws, nh, d, r, seed=8500)
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(8501)).to(torch.bfloat16)
+    leaves = [t.to(cuda_dev).requires_grad_() for t in (q, k, v, u, w)]
+    o = rfb_lib.rfb_attention_image_windows(*leaves, 0.2, shift)
+    o.backward(do.to(cuda_dev))
+    torch.cuda.synchronize()
+    assert rfb_lib.last_device_error() == 0
+    want = oracle_mod.bwd_image_windows(*(to_f64(t) for t in (q, k, v, u, w, do)), 0.2, 8, shift)
+    for name, t, b in zip(("dQ", "dK", "dV", "dU", "dW"), leaves, want):
+        ma = MAX_ABS if name in ("dQ", "dK", "dV") else max(MAX_ABS, 2.0 ** -7 * np.abs(b).max())
+        assert_close(name, t.grad, b, max_abs=ma)
