@@ -1,5 +1,6 @@
 """Pins of the oracle's shifted-window attention over feature maps."""
 import numpy as np
+import pytest
 
 import oracle
 from rank_biased_window_b200.inputs import make_inputs, to_f64
@@ -134,3 +135,56 @@ def test_backward_shift_on_one_window_is_four_region_backwards():
                 for got, want in ((dq, rq), (dk, rk), (dv, rv)):
                     np.testing.assert_allclose(got[sl].reshape(16, d), want[0, 0], rtol=1e-10,
                                                atol=1e-12)
+
+
+# Plausible mistakes planted in a copy of the oracle's image-window backward
+# (text substitution in its source); the pins above must reject every one.
+BWD_MUTANTS = [
+    ("mask_dropped", "S = np.where(allowed, S, -np.inf)\n                    E = np.exp",
+     "S = S\n                    E = np.exp"),
+    ("not_rolled_back", "return back(dQ), back(dK), back(dV), dU, dW",
+     "return dQ, dK, dV, dU, dW"),
+    ("du_not_summed", "dU[h] += dS @ ww[h]", "dU[h] = dS @ ww[h]"),
+    ("d_missing", "dS = P * (dP - Dv)", "dS = P * dP"),
+    ("dk_unscaled", "dK[b, ys, xs, h] = scale * (dS.T @ Qw)", "dK[b, ys, xs, h] = dS.T @ Qw"),
+    ("dw_wrong_operand", "dW[h] += dS.T @ uu[h]", "dW[h] += dS.T @ ww[h]"),
+    ("dv_uses_ds", "dV[b, ys, xs, h] = P.T @ dOw", "dV[b, ys, xs, h] = dS.T @ dOw"),
+]
+
+
+def _planted_bwd(old, new):
+    import inspect
+    src = inspect.getsource(oracle.bwd_image_windows)
+    assert src.count(old) == 1, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<planted>", "exec"), ns)
+    return ns["bwd_image_windows"]
+
+
+def _fd_pin_holds(bwd):
+    B, Hs, Ws, nh, d, r = 1, 16, 16, 2, 4, 2
+    q, k, v, u, w = _maps(B, Hs, Ws, nh, d, r, seed=31)
+    rng = np.random.default_rng(8)
+    do = rng.standard_normal(q.shape)
+    s, shift, h = 0.45, 4, 1e-6
+    grads = bwd(q, k, v, u, w, do, s, 8, shift)
+    args = [q, k, v, u, w]
+    loss = lambda a: float((do * oracle.fwd_image_windows(*a, s, 8, shift)[0]).sum())
+    for t, g in enumerate(grads):
+        for idx in rng.choice(args[t].size, size=6, replace=False):
+            plus, minus = [a.copy() for a in args], [a.copy() for a in args]
+            plus[t].reshape(-1)[idx] += h
+            minus[t].reshape(-1)[idx] -= h
+            fd = (loss(plus) - loss(minus)) / (2 * h)
+            if abs(fd - g.reshape(-1)[idx]) > 1e-6 * max(1.0, abs(fd)):
+                return False
+    return True
+
+
+def test_backward_pins_hold_for_the_unmodified_copy():
+    assert _fd_pin_holds(_planted_bwd("dS = P * (dP - Dv)", "dS = P * (dP - Dv)"))
+
+
+@pytest.mark.parametrize("name,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
+def test_backward_pins_catch_planted_mistake(name, old, new):
+    assert not _fd_pin_holds(_planted_bwd(old, new)), name
