@@ -188,3 +188,46 @@ def test_backward_pins_hold_for_the_unmodified_copy():
 @pytest.mark.parametrize("name,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
 def test_backward_pins_catch_planted_mistake(name, old, new):
     assert not _fd_pin_holds(_planted_bwd(old, new)), name
+
+
+# The same for the forward: mistakes planted in a copy of fwd_image_windows
+# must fail at least one of the forward pins above.
+FWD_MUTANTS = [
+    ("mask_dropped", "S = np.where(allowed, S, -np.inf)\n                    m = S.max",
+     "S = S\n                    m = S.max"),
+    ("rolled_the_wrong_way", "np.roll(x, (-shift, -shift), axis=(1, 2)) for x in (q, k, v)",
+     "np.roll(x, (shift, shift), axis=(1, 2)) for x in (q, k, v)"),
+    ("not_rolled_back", "return (np.roll(O, (shift, shift), axis=(1, 2)), np.roll(L, (shift, shift), axis=(1, 2)))",
+     "return (O, L)"),
+    ("bias_transposed", "np.asarray(u, dtype=np.float64)[h] @ np.asarray(w, dtype=np.float64)[h].T",
+     "np.asarray(w, dtype=np.float64)[h] @ np.asarray(u, dtype=np.float64)[h].T"),
+]
+
+
+def _planted_fwd(old, new):
+    import inspect
+    src = inspect.getsource(oracle.fwd_image_windows)
+    assert src.count(old) == 1, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<planted>", "exec"), ns)
+    return ns["fwd_image_windows"]
+
+
+def _fwd_pins_hold(fwd, monkeypatch):
+    monkeypatch.setattr(oracle, "fwd_image_windows", fwd)
+    try:
+        test_unshifted_equals_factored_oracle_on_partitioned_windows()
+        test_shift_on_one_window_splits_it_into_four_regions()
+        test_interior_shifted_window_needs_no_mask()
+    except AssertionError:
+        return False
+    return True
+
+
+def test_forward_pins_hold_for_the_unmodified_copy(monkeypatch):
+    assert _fwd_pins_hold(_planted_fwd("m = S.max", "m = S.max"), monkeypatch)
+
+
+@pytest.mark.parametrize("name,old,new", FWD_MUTANTS, ids=[m[0] for m in FWD_MUTANTS])
+def test_forward_pins_catch_planted_mistake(name, old, new, monkeypatch):
+    assert not _fwd_pins_hold(_planted_fwd(old, new), monkeypatch), name
