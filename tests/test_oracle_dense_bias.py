@@ -1,6 +1,7 @@
 """Pins of the oracle's dense-bias forward (the materialised-bias form used by
 the comparator kernel) against the independently written factored oracle."""
 import numpy as np
+import pytest
 
 import oracle
 from rank_biased_window_b200.inputs import make_inputs, to_f64
@@ -47,3 +48,42 @@ def test_dense_bias_row_constant_shift():
     o2, l2 = oracle.fwd_dense_bias(f["q"], f["k"], f["v"], np.zeros((H, N, N)), 0.4)
     np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(l1, l2 + c[None, None, :], rtol=1e-12, atol=1e-12)
+
+
+# Mistakes planted in a copy of fwd_dense_bias must fail one of the pins above.
+MUTANTS = [
+    ("bias_transposed", "S = scale * (q[b, h] @ k[b, h].T) + bm", "S = scale * (q[b, h] @ k[b, h].T) + bm.T"),
+    ("bias_scaled", "S = scale * (q[b, h] @ k[b, h].T) + bm", "S = scale * (q[b, h] @ k[b, h].T + bm)"),
+    ("bias_of_another_head", "bm = bias[h] if bias.ndim == 3 else bias[b, h]",
+     "bm = bias[0] if bias.ndim == 3 else bias[b, 0]"),
+    ("lse_without_max", "L[b, h] = (m + np.log(l))[:, 0]", "L[b, h] = np.log(l)[:, 0]"),
+]
+
+
+def _planted(old, new):
+    import inspect
+    src = inspect.getsource(oracle.fwd_dense_bias)
+    assert src.count(old) == 1, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<planted>", "exec"), ns)
+    return ns["fwd_dense_bias"]
+
+
+def _pins_hold(fn, monkeypatch):
+    monkeypatch.setattr(oracle, "fwd_dense_bias", fn)
+    try:
+        test_dense_bias_equals_factored_oracle()
+        test_dense_bias_shared_per_head_and_zero_bias()
+        test_dense_bias_row_constant_shift()
+    except AssertionError:
+        return False
+    return True
+
+
+def test_pins_hold_for_the_unmodified_copy(monkeypatch):
+    assert _pins_hold(_planted("L[b, h] =", "L[b, h] ="), monkeypatch)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(name, old, new, monkeypatch):
+    assert not _pins_hold(_planted(old, new), monkeypatch), name
