@@ -35,6 +35,42 @@ def test_oracle_recovers_exact_low_rank_and_diagonal():
     assert abs(err[0] - np.sqrt((d[2:] ** 2).sum() / (d ** 2).sum())) < 1e-14
 
 
+# Mistakes planted in a copy of the oracle's factoriser must fail its pins.
+MUTANTS = [
+    ("w_from_left_vectors", "W[h] = Yt[:r].T * root", "W[h] = X[:, :r] * root"),
+    ("singular_values_not_split", "root = np.sqrt(S[:r])", "root = S[:r]"),
+    ("right_vectors_not_transposed", "W[h] = Yt[:r].T * root", "W[h] = Yt[:, :r] * root"),
+]
+
+
+def _planted(old, new):
+    import inspect
+    src = inspect.getsource(oracle.factorize_bias)
+    assert src.count(old) == 1, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<planted>", "exec"), ns)
+    return ns["factorize_bias"]
+
+
+def _pins_hold(fn, monkeypatch):
+    monkeypatch.setattr(oracle, "factorize_bias", fn)
+    try:
+        test_oracle_error_is_eckart_young()
+        test_oracle_recovers_exact_low_rank_and_diagonal()
+    except AssertionError:
+        return False
+    return True
+
+
+def test_oracle_pins_hold_for_the_unmodified_copy(monkeypatch):
+    assert _pins_hold(_planted("root = np.sqrt(S[:r])", "root = np.sqrt(S[:r])"), monkeypatch)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_oracle_pins_catch_planted_mistake(name, old, new, monkeypatch):
+    assert not _pins_hold(_planted(old, new), monkeypatch), name
+
+
 @pytest.mark.parametrize("r", [4, 8, 16])
 def test_randomised_factoriser_near_optimal_cpu(r):
     B = relative_position_bias(3, 8, 8, seed=11)
