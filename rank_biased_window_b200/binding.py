@@ -133,6 +133,50 @@ def _check_operand(name, t, shape, device):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_f32(name, t, shape, device):
+    """fp32 tensors the kernels write or read (LSE): dtype, device, shape,
+    contiguity -- a wrong one would hand the kernels a bad pointer."""
+    if (isinstance(t, torch.Tensor) and t.dtype is torch.float32 and t.device == device
+            and t.shape == shape and t.is_contiguous()):
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32, got {t.dtype}")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must live on {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(workspace, nbytes, device):
+    """The caller's workspace (or a new one) and its size in bytes; its size
+    is checked by the library (RFB_ERR_WORKSPACE), its device and layout here."""
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    if (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda
+            or workspace.device != device or not workspace.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def _grads(grads, q, u, r, device):
+    """Gradient outputs: new tensors, or the caller's after checking that each
+    has its input's shape, dtype and device."""
+    if grads is None:
+        return (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q),
+                torch.empty_like(u) if r else None, torch.empty_like(u) if r else None)
+    dq, dk, dv, du, dw = grads
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_operand(name, t, tuple(q.shape), device)
+    if r > 0:
+        _check_operand("du", du, tuple(u.shape), device)
+        _check_operand("dw", dw, tuple(u.shape), device)
+        return dq, dk, dv, du, dw
+    return dq, dk, dv, None, None
+
+
 def _dims(q, u):
     if q.dim() != 4:
         raise ValueError("q must be [B, H, N, d]")
@@ -156,8 +200,7 @@ def attn_fwd(q, k, v, u=None, w=None, scale=None, *, out=None, lse=None, stream=
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
     _check_operand("out", o, (B, H, N, d), dev)
-    if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_f32("lse", l, (B, H, N), dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_fwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
@@ -183,23 +226,16 @@ def attn_bwd(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=None, grads=N
         _check_operand("w", w, (B, H, N, r), dev)
     else:
         u = w = None
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_f32("lse", lse, (B, H, N), dev)
     s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
-    if grads is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        du = torch.empty_like(u) if r else None
-        dw = torch.empty_like(w) if r else None
-    else:
-        dq, dk, dv, du, dw = grads
+    dq, dk, dv, du, dw = _grads(grads, q, u, r, dev)
     nbytes = bwd_workspace_size(B, H, N, d, r)
-    if workspace is None:
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    workspace, ws_bytes = _workspace(workspace, nbytes, dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_bwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
             ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
-            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, H, N, d, r, s,
+            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), ws_bytes, B, H, N, d, r, s,
             _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_bwd")
     return dq, dk, dv, du, dw
@@ -225,8 +261,7 @@ def attn_fwd_shared_bias(q, k, v, u=None, w=None, scale=None, *, out=None, lse=N
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
     _check_operand("out", o, (B, H, N, d), dev)
-    if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_f32("lse", l, (B, H, N), dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_fwd_shared_bias(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
@@ -256,8 +291,7 @@ def attn_fwd_dense_bias(q, k, v, bias, scale=None, *, out=None, lse=None, stream
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
     _check_operand("out", o, (B, H, N, d), dev)
-    if l.dtype != torch.float32 or tuple(l.shape) != (B, H, N) or not l.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_f32("lse", l, (B, H, N), dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_fwd_dense_bias(
             _ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(o),
@@ -288,8 +322,7 @@ def attn_fwd_image_windows(q, k, v, u=None, w=None, scale=None, *, win=8, shift=
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, Hs, Ws, nh), dtype=torch.float32, device=dev) if lse is None else lse
     _check_operand("out", o, (B, Hs, Ws, nh, d), dev)
-    if l.dtype != torch.float32 or tuple(l.shape) != (B, Hs, Ws, nh) or not l.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, W, heads]")
+    _check_f32("lse", l, (B, Hs, Ws, nh), dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_fwd_image_windows(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
@@ -321,23 +354,16 @@ def attn_bwd_image_windows(q, k, v, u, w, o, lse, dout, scale=None, *, win=8, sh
         _check_operand("w", w, (nh, win * win, r), dev)
     else:
         u = w = None
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hs, Ws, nh) or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, W, heads]")
+    _check_f32("lse", lse, (B, Hs, Ws, nh), dev)
     s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
-    if grads is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        du = torch.empty_like(u) if r else None
-        dw = torch.empty_like(w) if r else None
-    else:
-        dq, dk, dv, du, dw = grads
+    dq, dk, dv, du, dw = _grads(grads, q, u, r, dev)
     nbytes = bwd_image_windows_workspace_size(B, Hs, Ws, nh, d, r)
-    if workspace is None:
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    workspace, ws_bytes = _workspace(workspace, nbytes, dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_bwd_image_windows(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
             ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
-            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, Hs, Ws, nh, d,
+            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), ws_bytes, B, Hs, Ws, nh, d,
             r, int(win), int(shift), s, _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_bwd_image_windows")
     return dq, dk, dv, du, dw
@@ -363,23 +389,16 @@ def attn_bwd_shared_bias(q, k, v, u, w, o, lse, dout, scale=None, *, workspace=N
         _check_operand("w", w, (H, N, r), dev)
     else:
         u = w = None
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_f32("lse", lse, (B, H, N), dev)
     s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
-    if grads is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        du = torch.empty_like(u) if r else None
-        dw = torch.empty_like(w) if r else None
-    else:
-        dq, dk, dv, du, dw = grads
+    dq, dk, dv, du, dw = _grads(grads, q, u, r, dev)
     nbytes = bwd_shared_bias_workspace_size(B, H, N, d, r)
-    if workspace is None:
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    workspace, ws_bytes = _workspace(workspace, nbytes, dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_bwd_shared_bias(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),
             ctypes.cast(ctypes.c_void_p(lse.data_ptr()), _fp), _ptr(dout), _ptr(dq), _ptr(dk),
-            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), workspace.numel(), B, H, N, d, r, s,
+            _ptr(dv), _ptr(du), _ptr(dw), _ptr(workspace), ws_bytes, B, H, N, d, r, s,
             _stream_ptr(stream, dev))
     _check(rc, "rfb_attn_bwd_shared_bias")
     return dq, dk, dv, du, dw
@@ -416,15 +435,9 @@ def attn_bwd_noalloc(q, k, v, u, w, o, lse, dout, scale=None, *, grads=None, str
         _check_operand("w", w, (B, H, N, r), dev)
     else:
         u = w = None
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_f32("lse", lse, (B, H, N), dev)
     s = (1.0 / math.sqrt(d)) if scale is None else float(scale)
-    if grads is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        du = torch.empty_like(u) if r else None
-        dw = torch.empty_like(w) if r else None
-    else:
-        dq, dk, dv, du, dw = grads
+    dq, dk, dv, du, dw = _grads(grads, q, u, r, dev)
     with _on_device(dev):
         rc = load_library().rfb_attn_bwd_noalloc(
             _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(w), _ptr(o),

@@ -138,6 +138,27 @@ def test_image_windows_backward_host_checks(rfb_lib):
     assert size(0, 16, 24, heads, d, r) == 0 and size(1, 12, 24, heads, d, r) == 0
 
 
+def test_binding_rejects_bad_outputs_before_the_library():
+    """Output, LSE, gradient and workspace tensors the caller hands in are
+    checked on the host (dtype, device, shape, layout) before any pointer
+    reaches the kernels."""
+    import torch
+    from rank_biased_window_b200 import binding as b
+    dev = torch.device("cuda", 0)
+    lse = torch.zeros(2, 3, dtype=torch.float32)
+    with pytest.raises(ValueError, match="must live on"):
+        b._check_f32("lse", lse, (2, 3), dev)
+    with pytest.raises(TypeError, match="float32"):
+        b._check_f32("lse", lse.double(), (2, 3), dev)
+    with pytest.raises(ValueError, match="workspace"):
+        b._workspace(torch.zeros(64, dtype=torch.uint8), 64, dev)
+    q = torch.zeros(1, 2, 16, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="must live on"):
+        b._grads((q, q, q, None, None), q, None, 0, dev)
+    with pytest.raises(TypeError, match="bfloat16"):
+        b._grads((q.float(), q, q, None, None), q, None, 0, dev)
+
+
 def test_bench_accounting_helpers(tmp_path, monkeypatch):
     """bench.py's algorithmic flop / byte counts and the traffic record's
     source-hash gate."""
