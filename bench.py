@@ -2,7 +2,7 @@
 """Throughput of the rank-factorised-bias attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {rfb,reference}]
-                    [--workload train] [--no-cpu-baseline]
+                    [--workload train] [--no-cpu-baseline] [--no-configs]
 
 A step is one pass of the whole hot path -- forward (O, LSE) and backward
 (dQ, dK, dV, dU, dW) -- over one batch of the training workload: B=2 images of a
@@ -11,9 +11,18 @@ synthetic inputs (rank_biased_window_b200/inputs.py).  The metric is
 algorithmic bf16 TFLOP/s of that step (forward 2*BH*N^2*(2d+r) plus backward
 2*BH*N^2*(5d+3r) flops, r counted unpadded), with windows/s beside it.
 
-Multi-GPU (launched with torchrun): every rank runs its own full workload on
-its own GPU (independent problems, weak scaling, no data-path collective);
-the step time is the max over ranks and `value` counts the work of all ranks.
+The same JSON line carries, under "configs", the forward-only workloads (one
+8x8 window; 1024 SwinIR-style 8x8 windows; 64 windows of 32x32 tokens; a
+64x64 map), each timed with CUDA events with L2 flushed before every step,
+with its TFLOP/s, windows/s and binding roof (HBM for windows of <= 128
+tokens, the bf16 tensor peak otherwise; launch latency for the single
+window).
+
+Multi-GPU: every rank runs its own full workload on its own GPU (independent
+problems, weak scaling, no data-path collective); the step time is the max over
+ranks and `value` counts the work of all ranks.  `--gpus N` without a torchrun
+environment re-launches this script under torch.distributed.run with N local
+ranks (127.0.0.1).
 
 `--impl reference` times the fp64 CPU oracle (oracle/) on the host cores on a
 bounded sample of the same workload; it is a deliberately slow reference, not
@@ -48,6 +57,8 @@ def parse_args():
     ap.add_argument("--impl", choices=("rfb", "reference"), default="rfb")
     ap.add_argument("--workload", default="train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the forward-only workloads reported under 'configs'")
     ap.add_argument("--factorize", action="store_true",
                     help="time the low-rank factoriser of a dense relative-position bias "
                          "(the step before the path) on this workload's window, r = its rank")
@@ -224,7 +235,43 @@ def cpu_sample(wl, seconds, x64=None):
     return flops, t, R, oracle.max_threads(), x64
 
 
-def run_reference(args, wl, rank):
+def input_bytes(wl, shared=False, dense=False):
+    """Bytes of the step's device inputs (Q, K, V, the factors or the dense
+    bias, and dO when the step has a backward)."""
+    BH = wl.B * wl.H
+    n = 3 * BH * wl.N * wl.d * 2
+    if dense:
+        n += wl.H * wl.N * wl.N * 2
+    elif wl.r > 0:
+        n += 2 * (wl.H if shared else BH) * wl.N * wl.r * 2
+    if wl.backward and not dense:
+        n += BH * wl.N * wl.d * 2
+    return n
+
+
+def workload_config(wl, world, *, shared=False, dense=False):
+    """The `config` object of the JSON line.  Both arms build it here, so for
+    the same workload and rank count the two lines carry identical configs."""
+    nbytes = input_bytes(wl, shared, dense)
+    return {
+        "workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r,
+        "global_batch": wl.B * world, "seq_len": wl.N,
+        "parallelism": (f"data parallel over windows x{world}, dU/dW all-reduced (NCCL)"
+                        if shared and world > 1 else
+                        f"replicas x{world}" if world > 1 else "single GPU"),
+        "bias": ("dense [H, N, N] bf16 = U[h] W[h]^T (materialised-bias comparator, "
+                 "forward only)" if dense else
+                 "U, W [H, N, r] shared by all windows" if shared else
+                 "U, W [B, H, N, r] per window and head"),
+        "l2": (f"inputs exceed L2 ({nbytes / 2**20:.0f} MiB > 126 MiB), no flush"
+               if nbytes > L2_BYTES else
+               f"inputs {nbytes / 2**20:.0f} MiB fit in L2: before each step a 512 MiB "
+               f"write then read flushes L2 (clean lines), outside the timed events"),
+        "note": wl.note,
+    }
+
+
+def run_reference(args, wl, rank, world=1):
     if rank != 0:
         return 0
     per_step = max(1.0, 150.0 / max(args.steps + args.warmup, 1))
@@ -237,14 +284,15 @@ def run_reference(args, wl, rank):
     t_step = statistics.mean(times) if times else t
     value = flops / t_step / 1e12
     sample = (f"fp64 oracle, head 0 of {wl.B * wl.H}, {R} of {wl.N} query rows against all keys: "
-              f"forward + query-side backward (dQ, dU)")
+              f"forward" + (" + query-side backward (dQ, dU)" if wl.backward else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r,
-                   "parallelism": "cpu", "note": wl.note},
+        "config": workload_config(wl, world, shared=getattr(args, "shared_bias", False),
+                                  dense=getattr(args, "dense_bias", False)),
+        "device": "host cores (fp64 oracle, rank 0 only)",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -368,15 +416,119 @@ def run_image_windows(args, rank):
     print(json.dumps(line))
 
 
+SWEEP = ("tiny", "swinir", "large", "global")
+
+
+def config_roofline(wl, kernel_ms, peaks):
+    """Binding roof of a forward-only workload's kernel: launch latency for a
+    single window, HBM for windows of <= 128 tokens, else the bf16 tensor peak
+    (burst figure: these kernels run alone, for well under a second)."""
+    fl, _, fb, _ = work(wl)
+    if wl.B * wl.H == 1:
+        return {"bound": "launch", "achieved": kernel_ms * 1e3, "unit": "us per launch",
+                "peak": None, "frac": None}
+    if wl.N <= 128:
+        ach = fb / (kernel_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "peak_kind": f"HBM copy, {peaks['source']}",
+                "traffic": ncu_traffic("fwd", wl.name)}
+    ach = fl / (kernel_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": ach / peaks["bf16_tflops"], "peak_kind": f"bf16 burst, {peaks['source']}",
+            "traffic": ncu_traffic("fwd", wl.name)}
+
+
+def run_configs(rfb, torch, dev, stream, dist, world, peaks, steps, warmup):
+    """Forward-only workloads (one 8x8 window, SwinIR-style windows, 32x32
+    windows, a 64x64 map): per workload `steps` forwards, each preceded by an
+    L2 flush (512 MiB written then read, outside the timed events), timed with
+    CUDA events on the launching stream and by the library's per-launch
+    events; max over ranks."""
+    from rank_biased_window_b200.inputs import WORKLOADS, workload_inputs
+    flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev)
+    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
+    out = {}
+    for name in SWEEP:
+        wl = WORKLOADS[name]
+        g = {k: v.to(dev) for k, v in workload_inputs(wl, with_dout=False).items()}
+        o = torch.empty_like(g["q"])
+        lse = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device=dev)
+        u, w = (g["u"], g["w"]) if wl.r else (None, None)
+
+        def fwd():
+            rfb.attn_fwd(g["q"], g["k"], g["v"], u, w, wl.scale, out=o, lse=lse, stream=stream)
+
+        for _ in range(max(warmup, 3)):
+            fwd()
+        torch.cuda.synchronize(dev)
+        if rfb.last_device_error() != 0:
+            raise RuntimeError(f"device error word set by the {name} forward")
+        rfb.profile_read()
+        rfb.profile_enable(True)
+        evs = []
+        for _ in range(steps):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                flush_sum.copy_(flush.view(torch.float32).sum())
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fwd()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        rfb.profile_enable(False)
+        prof = rfb.profile_read()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        kms = prof["fwd"][0] / max(prof["fwd"][1], 1)
+        ms, kms = max_over_ranks([ms, kms], dist, dev)
+        fl, _, fb, _ = work(wl)
+        out[name] = {
+            "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r, "pass": "fwd",
+            "ms_per_step": ms, "kernel_ms": kms,
+            "tflops": throughput_tflops(fl, world, ms),
+            "kernel_tflops": fl / (kms * 1e-3) / 1e12,
+            "windows_per_s": wl.B * world / (ms * 1e-3),
+            "pct_of_bf16_peak": fl / (kms * 1e-3) / 1e12 / peaks["bf16_tflops"] * 100.0,
+            "algorithmic_bytes": fb,
+            "roofline": config_roofline(wl, kms, peaks),
+            "steps": steps, "warmup": max(warmup, 3),
+            "l2": "flushed (512 MiB write then read) before every step, outside the timed events",
+            "note": wl.note,
+        }
+    return out
+
+
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_argv(argv, n, port):
+    """Command that runs this script under torch.distributed.run with n local
+    ranks (one per GPU) on 127.0.0.1."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.join(ROOT, "bench.py"), *argv]
+
+
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # One process per GPU: re-launch under torchrun (rank 0 prints the line).
+        import subprocess
+        return subprocess.call(relaunch_argv(sys.argv[1:], args.gpus, free_port()))
     from rank_biased_window_b200.inputs import WORKLOADS, workload_inputs
     wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; "
+                         f"reporting the {world} ranks that run\n")
     if args.impl == "reference":
-        return run_reference(args, wl, rank)
+        return run_reference(args, wl, rank, world)
 
     import torch
     import rank_biased_window_b200 as rfb
@@ -452,7 +604,7 @@ def main():
     # every step, outside the timed events: a 512 MiB write, then a read of the
     # same buffer so that L2 holds clean lines of other data (a write alone
     # leaves dirty lines whose write-back would be charged to the next step).
-    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    in_bytes = input_bytes(wl, shared, dense)
     flush = None if in_bytes > L2_BYTES else torch.empty(512 * 2**20, dtype=torch.uint8,
                                                         device=dev)
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
@@ -554,7 +706,6 @@ def main():
     f1.record(stream)
     torch.cuda.synchronize(dev)
     ms_e2e_total = f0.elapsed_time(f1)
-
     # ---- max over ranks
     ms_total, ms_e2e_total = max_over_ranks([ms_total, ms_e2e_total], dist, dev)
 
@@ -583,11 +734,15 @@ def main():
                 "peak_kind": f"HBM copy, {peaks['source']}", "traffic": ncu_traffic(dom, wl.name),
                 "avg_launch_ms": per[dom][0]}
     elif dom_flops is not None:
+        # Against the burst bf16 figure (the larger of the two measured peaks,
+        # so the lower fraction); the sustained-peak fraction is given beside it.
         achieved = dom_flops / (per[dom][0] * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"],
-                "peak_kind": f"bf16 sustained, {peaks['source']}",
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_kind": f"bf16 burst, {peaks['source']}",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "sustained_peak": peaks["bf16_tflops_sustained"],
                 "traffic": ncu_traffic(dom, wl.name),
                 "avg_launch_ms": per[dom][0]}
     else:
@@ -597,38 +752,32 @@ def main():
     kernels = {k: {"avg_ms": v[0], "launches": v[1], "share": v[2] / max(sum(w[2] for w in
                per.values()), 1e-9)} for k, v in per.items() if v[1]}
 
+    configs = None
+    if not args.no_configs:
+        configs = run_configs(rfb, torch, dev, stream, dist, world, peaks,
+                              max(3, min(args.steps, 20)), args.warmup)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         flops_c, t_c, R, cores, _ = cpu_sample(wl, args.cpu_seconds)
         cpu = {"value": flops_c / t_c / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"fp64 oracle, head 0 of {wl.B * wl.H}, {R} of {wl.N} query rows "
-                         f"against all keys: forward + query-side backward (dQ, dU), "
-                         f"{t_c:.1f} s"}
+                         f"against all keys: forward"
+                         + (" + query-side backward (dQ, dU)" if wl.backward else "")
+                         + f", {t_c:.1f} s"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) Q,K,V,dO; N(0,1/r) U,W; bf16)",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "r": wl.r,
-                   "global_batch": wl.B * world, "seq_len": wl.N,
-                   "parallelism": (f"data parallel over windows x{world}, dU/dW all-reduced "
-                                   f"(NCCL)" if shared and world > 1 else
-                                   f"replicas x{world}" if world > 1 else "single GPU"),
-                   "bias": ("dense [H, N, N] bf16 = U[h] W[h]^T (materialised-bias "
-                            "comparator, forward only)" if dense else
-                            "U, W [H, N, r] shared by all windows" if shared else
-                            "U, W [B, H, N, r] per window and head"),
-                   "l2": (f"inputs exceed L2 ({in_bytes / 2**20:.0f} MiB > 126 MiB), no flush"
-                          if flush is None else
-                          f"inputs {in_bytes / 2**20:.0f} MiB fit in L2: before each step a "
-                          f"512 MiB write then read flushes L2 (clean lines), outside the "
-                          f"timed events"),
-                   "note": wl.note},
+        "config": workload_config(wl, world, shared=shared, dense=dense),
         "windows_per_s": wl.B * world / (ms_step * 1e-3),
         "pct_of_bf16_peak": value / world / peaks["bf16_tflops"] * 100.0,
+        "peaks": peaks,
         "roofline": roof,
         "kernels": kernels,
+        "configs": configs,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,

@@ -23,7 +23,7 @@
  * rfb_attn_bwd, rfb_attn_bwd_noalloc); variants with one factor pair per head
  * shared by all windows (rfb_attn_*_shared_bias); shifted-window attention on
  * feature maps (rfb_attn_fwd_image_windows, rfb_attn_bwd_image_windows); a dense-bias
- * comparator (rfb_attn_fwd_dense_bias); diagnostics.  Each declaration below
+ * comparator (rfb_attn_fwd_dense_bias); diagnostics and test hooks.  Each declaration below
  * states what differs from these conventions.
  *
  * Conventions for every entry point
@@ -120,17 +120,27 @@ RFB_API int rfb_attn_bwd(const void* q, const void* k, const void* v, const void
  * plugin host that owns the allocator and hands its plugins nothing but their
  * input and output buffers.
  *
- * Limit: a problem whose rfb_attn_bwd_workspace_size() exceeds
- * RFB_NOALLOC_SCRATCH_BYTES (about B*H*N*(d+r) > 8 M elements) is rejected with
- * RFB_ERR_WORKSPACE before anything is enqueued.  The call makes no cudaMalloc,
- * cudaFree or other allocating call.
+ * Limit: the call accepts exactly the problems for which
+ * rfb_attn_bwd_workspace_size(B, H, N, d, r) <= RFB_NOALLOC_SCRATCH_BYTES,
+ * i.e. about 8 + 4 (d + r) + 2 r bytes per row of B*H*N (two fp32 row
+ * statistics, with N rounded up to a multiple of 128; the fp32 dQ | dU
+ * accumulator; bf16 U / s): up to about 73,000 rows for d = 64, r = 32 and
+ * 182,000 rows for d = 32, r = 8.  Larger problems are rejected with
+ * RFB_ERR_WORKSPACE before anything is enqueued.  The call makes no
+ * cudaMalloc, cudaFree or other allocating call.
  *
- * Cost: every GPU on which this library's kernels are loaded keeps the array
- * until the process exits.
- *
- * First call on a device: it looks up the array's device address with that
- * device current (cudaGetSymbolAddress) and caches it; make that first call
- * before any stream capture on the device.
+ * Cost and set-up: the array is device memory that CUDA reserves on a GPU
+ * when this library's kernels are loaded there -- with CUDA's lazy module
+ * loading, at the first library call on that device that launches a kernel
+ * or looks up the array, not when the library is opened -- and keeps until
+ * the process exits.  A caller that reserves the rest of the device's memory
+ * up front must therefore make one library call on the device before it
+ * does.  An empty call of this function (B, H or N == 0, with a supported d
+ * and r and a valid scale) is enough: it loads the kernels, which reserves
+ * the array, and caches the array's device address (cudaGetSymbolAddress,
+ * with that device current), launching nothing.  The first call on a device,
+ * empty or not, does that set-up, so make it before any stream capture on
+ * the device.  An empty call returns RFB_ERR_CUDA if the set-up fails.
  *
  * Sharing: all calls on one device use the same array, which keeps whatever
  * the previous call left; each call clears the parts that must start at zero.
@@ -288,6 +298,25 @@ RFB_API int rfb_last_cuda_error(int* site);
  * the launch status; read the outcome with rfb_last_device_error().
  */
 RFB_API int rfb_selftest_wait_timeout(unsigned int timeout_us, void* stream);
+
+/*
+ * Failure-detection test hook for the attention kernels' own waits (not for
+ * production use).  Every kernel launched after this call gets:
+ *   limit_us  : the limit of each main-loop wait on a copy, an MMA or another
+ *               role of the same CTA, in microseconds (0 restores the default
+ *               of 2 s).  The exit-path waits for copies and MMAs already in
+ *               flight keep 2 s.
+ *   fail_site : a wait site number (the value stored in bits 8..15 of the
+ *               error word) whose wait gives up at once, as if its limit had
+ *               expired, or -1 for none.
+ * A wait that gives up raises its CTA's abort flag and records
+ * RFB_ERR_DEVICE_TIMEOUT | site << 8 in the error word; the CTA's other roles
+ * leave their loops, let in-flight copies and MMAs land, free TMEM and return.
+ * The call's outputs are then incomplete; the context stays usable.  The
+ * setting is process-wide: restore it with rfb_debug_set_wait_limit(0, -1).
+ * Returns RFB_ERR_INVALID_ARG if fail_site is outside [-1, 255].
+ */
+RFB_API int rfb_debug_set_wait_limit(unsigned int limit_us, int fail_site);
 
 /*
  * Optional per-kernel timing.  While enabled, every kernel launch made by

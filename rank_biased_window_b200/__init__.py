@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     attn_bwd,
     attn_bwd_image_windows,
     attn_bwd_noalloc,
+    attn_bwd_noalloc_setup,
     attn_bwd_shared_bias,
     attn_fwd,
     attn_fwd_dense_bias,
@@ -22,6 +23,7 @@ from .binding import (  # noqa: F401
     bwd_image_windows_workspace_size,
     bwd_shared_bias_workspace_size,
     bwd_workspace_size,
+    debug_set_wait_limit,
     last_device_error,
     load_library,
     profile_enable,
@@ -34,10 +36,10 @@ from .binding import (  # noqa: F401
 )
 from .factorize import factorize_bias, relative_position_bias  # noqa: F401
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "bwd_workspace_size", "rfb_attention", "RFBAttention",
+__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_noalloc_setup", "bwd_workspace_size", "rfb_attention", "RFBAttention",
            "attn_fwd_shared_bias", "attn_fwd_dense_bias", "attn_fwd_image_windows", "attn_bwd_image_windows",
            "bwd_image_windows_workspace_size", "attn_bwd_shared_bias", "bwd_shared_bias_workspace_size",
            "rfb_attention_shared_bias", "RFBAttentionSharedBias",
            "rfb_attention_image_windows", "RFBImageWindows", "allreduce_bias_grads",
            "factorize_bias", "relative_position_bias",
-           "last_device_error", "selftest_wait_timeout", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]
+           "last_device_error", "selftest_wait_timeout", "debug_set_wait_limit", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]

@@ -45,6 +45,7 @@ SIGNATURES = {
     "rfb_last_device_error": (_i, []),
     "rfb_last_cuda_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
     "rfb_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
+    "rfb_debug_set_wait_limit": (_i, [ctypes.c_uint, _i]),
     "rfb_selftest_soft_exp2": (_i, [_vp, _vp, _i, _vp]),
     "rfb_profile_enable": (_i, [_i]),
     "rfb_profile_read": (_i, [_fp, ctypes.POINTER(ctypes.c_int)]),
@@ -418,7 +419,23 @@ def allreduce_bias_grads(du, dw, group=None):
     return du, dw
 
 
+# Size of the library's fixed scratch array (RFB_NOALLOC_SCRATCH_BYTES in
+# include/rfb_attn.h; a CPU test checks that the two agree).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def attn_bwd_noalloc_setup(device=None, stream=None):
+    """Loads the library's kernels on `device` (which reserves the fixed
+    scratch array of rfb_attn_bwd_noalloc there) and caches the array's
+    address, by an empty call of that entry point.  Call it before reserving
+    the rest of the device's memory or capturing a stream on it."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else \
+        torch.device(device)
+    with _on_device(dev):
+        rc = load_library().rfb_attn_bwd_noalloc(
+            None, None, None, None, None, None, None, None, None, None, None, None, None,
+            0, 1, 1, 64, 0, 0.125, _stream_ptr(stream, dev))
+    _check(rc, "rfb_attn_bwd_noalloc (set-up)")
 
 
 def attn_bwd_noalloc(q, k, v, u, w, o, lse, dout, scale=None, *, grads=None, stream=None):
@@ -454,6 +471,14 @@ def attn_bwd_noalloc(q, k, v, u, w, o, lse, dout, scale=None, *, grads=None, str
 def last_device_error() -> int:
     """Synchronise the current device, read and clear the kernels' error word."""
     return int(load_library().rfb_last_device_error())
+
+
+def debug_set_wait_limit(limit_us: int = 0, fail_site: int = -1):
+    """Test hook: main-loop wait limit of the kernels launched afterwards (0:
+    the default 2 s) and a wait site that gives up at once (-1: none).
+    Process-wide; debug_set_wait_limit() restores the defaults."""
+    _check(load_library().rfb_debug_set_wait_limit(int(limit_us), int(fail_site)),
+           "rfb_debug_set_wait_limit")
 
 
 def selftest_wait_timeout(timeout_us: int = 1000, stream=None, device=None):

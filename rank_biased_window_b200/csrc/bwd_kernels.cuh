@@ -60,7 +60,8 @@ struct BwdArgs {
   float scale;       // s
   float scale_log2;  // s log2(e)
   float inv_scale;   // 1/s
-  uint64_t timeout_ns;
+  uint64_t timeout_ns;  // limit of each main-loop wait
+  int fail_site;        // test hook: wait site that gives up at once (-1: none)
   // Shifted-window mask of image windows (N = 64, tokens in raster order
   // inside each 8 x 8 window; 0 = no mask): window-head bh is window
   // (bh / mask_heads) of a map of mask_nwy x mask_nwx windows per image.
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const WaitGuard g{abort_flag, args.err, args.timeout_ns};
+  const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -366,9 +367,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bulk_load(st + C::S_L2, l2 + i * kTile, 512, q_full(s));
         bulk_load(st + C::S_DV, dv + i * kTile, 512, q_full(s));
       }
-      wait_drain(kv_full, 0, args.timeout_ns);
+      wait_drain(kv_full, 0);
       for (int j = (i > NS ? i - NS : 0); j < i; ++j)
-        wait_drain(q_full(j % NS), (j / NS) & 1, args.timeout_ns);
+        wait_drain(q_full(j % NS), (j / NS) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------ MMA issue (whole warp)
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     umma_commit(drain_bar);
-    wait_drain(drain_bar, 0, args.timeout_ns);
+    wait_drain(drain_bar, 0);
     __syncwarp();
   } else {
     // ------------------------------------- compute warps (two warpgroups)

@@ -58,7 +58,8 @@ struct FwdArgs {
   int bias_mode;
   float scale_log2;  // s * log2(e)
   float inv_scale;   // 1 / s  (U' = bf16(U / s))
-  uint64_t timeout_ns;
+  uint64_t timeout_ns;  // limit of each main-loop wait
+  int fail_site;        // test hook: wait site that gives up at once (-1: none)
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -67,10 +68,10 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
 
 // Bounded wait that ignores the abort flag: used only on the exit path to let
 // in-flight copies and MMAs land before the CTA frees its resources.
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > timeout_ns) return;
+    if (global_timer_ns() - t0 > kDrainTimeoutNs) return;
   }
 }
 
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const WaitGuard g{abort_flag, args.err, args.timeout_ns};
+  const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
 
   if (warp >= 8) {
    // Control warpgroup: all four warps shrink their budget at this point.
@@ -407,9 +408,9 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         }
       }
       // Let the last copies land before the CTA can exit.
-      if (resident) wait_drain(res_full, 0, args.timeout_ns);
+      if (resident) wait_drain(res_full, 0);
       for (int j = (it > NS ? it - NS : 0); j < it; ++j)
-        wait_drain(in_full(j % NS), (j / NS) & 1, args.timeout_ns);
+        wait_drain(in_full(j % NS), (j / NS) & 1);
     }
    } else if (warp == 9) {
     // --------------------------------------------------- score MMA issue
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     }
     (void)ok;
     umma_commit(drain_bar);
-    wait_drain(drain_bar, 0, args.timeout_ns);
+    wait_drain(drain_bar, 0);
     __syncwarp();
    } else if (warp == 10) {
     // ------------------------------------------------------ PV MMA issue
@@ -451,7 +452,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       umma_commit(in_empty(s));
     }
     umma_commit(drain_bar);
-    wait_drain(drain_bar, 0, args.timeout_ns);
+    wait_drain(drain_bar, 0);
     __syncwarp();
    } else {
     // ------------------------------------------------- U' = U / s in place
@@ -719,7 +720,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const WaitGuard g{abort_flag, args.err, args.timeout_ns};
+  const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
 
   if (warp >= 8) {
    // Control warpgroup: all four warps shrink their budget at this point.
@@ -762,9 +763,9 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         }
       }
       // No copy may still be in flight when the CTA exits.
-      if (uc > 0) wait_drain(q_full, (uc - 1) & 1, args.timeout_ns);
+      if (uc > 0) wait_drain(q_full, (uc - 1) & 1);
       for (int i = (it > NS ? it - NS : 0); i < it; ++i)
-        wait_drain(kv_full(i % NS), (i / NS) & 1, args.timeout_ns);
+        wait_drain(kv_full(i % NS), (i / NS) & 1);
     }
    } else if (warp == 9 || warp == 10) {
     // MMA issue for query tile t = warp - 9 (one converged warp each).
@@ -819,7 +820,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       }
     }
     umma_commit(drain_bar);
-    wait_drain(drain_bar, 0, args.timeout_ns);
+    wait_drain(drain_bar, 0);
     __syncwarp();
    }
   } else {

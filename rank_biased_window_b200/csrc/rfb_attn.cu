@@ -32,7 +32,7 @@ __global__ void selftest_wait_kernel(int* err, uint64_t timeout_ns) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const WaitGuard g{&abort_flag, err, timeout_ns};
+    const WaitGuard g{&abort_flag, err, timeout_ns, -1};
     wait_bounded(smem_u32(&bar), 0, g, 99);  // nothing ever arrives on this barrier
   }
   __syncthreads();
@@ -57,6 +57,11 @@ namespace {
 
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr int kMaxDevices = 64;
+
+// Test hook (rfb_debug_set_wait_limit): the main-loop wait limit and the wait
+// site that gives up at once, passed to every kernel launched afterwards.
+std::atomic<uint64_t> g_wait_limit_ns{kWaitTimeoutNs};
+std::atomic<int> g_fail_site{-1};
 
 // Last failing CUDA call (error code and the site that saw it), for diagnostics.
 std::atomic<int> g_last_cuda_err{0};
@@ -557,7 +562,8 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const void* u, co
   a.bias_mode = shared ? kBiasWindow : kBiasTile;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
-  a.timeout_ns = kWaitTimeoutNs;
+  a.timeout_ns = g_wait_limit_ns.load();
+  a.fail_site = g_fail_site.load();
   return dispatch_fwd_rp(d, rp, m, a, dev.sms, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
@@ -631,7 +637,8 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
-  a.timeout_ns = kWaitTimeoutNs;
+  a.timeout_ns = g_wait_limit_ns.load();
+  a.fail_site = g_fail_site.load();
   // img_mask = {shift, windows per map row, windows per map column, heads}
   a.mask_shift = img_mask ? img_mask[0] : 0;
   a.mask_nwx = img_mask ? img_mask[1] : 1;
@@ -749,7 +756,8 @@ int rfb_attn_fwd_dense_bias(const void* q, const void* k, const void* v, const v
   a.bias_mode = kBiasTile;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
-  a.timeout_ns = kWaitTimeoutNs;
+  a.timeout_ns = g_wait_limit_ns.load();
+  a.fail_site = g_fail_site.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 32 ? launch_long_dense<32>(m, a, dev.sms, st) : launch_long_dense<64>(m, a, dev.sms, st);
 }
@@ -810,7 +818,8 @@ int rfb_attn_fwd_image_windows(const void* q, const void* k, const void* v, cons
   a.shift = shift;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.inv_scale = 1.0f / scale;
-  a.timeout_ns = kWaitTimeoutNs;
+  a.timeout_ns = g_wait_limit_ns.load();
+  a.fail_site = g_fail_site.load();
   return dispatch_window_img(d, rp, m, a, dev.sms, static_cast<cudaStream_t>(stream));
 }
 
@@ -928,14 +937,25 @@ int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int d, int r, float scale, void* stream) {
   bool empty = false;
   if (int rc = check_shape(B, H, N, d, r, scale, &empty)) return rc;
-  if (empty) return RFB_OK;
-  if (ws_layout(B, H, N, d, r).total > RFB_NOALLOC_SCRATCH_BYTES) return RFB_ERR_WORKSPACE;
   void* scratch = nullptr;
+  // An empty call does only the set-up: looking up the array's address loads
+  // the library's kernels on this device, which reserves the array, and caches
+  // the address -- so a caller can do both before it reserves the rest of the
+  // device's memory or captures a stream.
+  if (empty) return noalloc_scratch(&scratch);
+  if (ws_layout(B, H, N, d, r).total > RFB_NOALLOC_SCRATCH_BYTES) return RFB_ERR_WORKSPACE;
   if (int rc = noalloc_scratch(&scratch)) return rc;
   // The backward's first kernel zeroes the accumulator and rewrites the row
   // statistics, so what an earlier call left in the array does not matter.
   return rfb_attn_bwd(q, k, v, u, w, o, lse, dout, dq, dk, dv, du, dw, scratch,
                       RFB_NOALLOC_SCRATCH_BYTES, B, H, N, d, r, scale, stream);
+}
+
+int rfb_debug_set_wait_limit(unsigned int limit_us, int fail_site) {
+  if (fail_site < -1 || fail_site > 255) return RFB_ERR_INVALID_ARG;
+  g_wait_limit_ns.store(limit_us == 0 ? kWaitTimeoutNs : static_cast<uint64_t>(limit_us) * 1000ull);
+  g_fail_site.store(fail_site);
+  return RFB_OK;
 }
 
 const char* rfb_strerror(int status) {

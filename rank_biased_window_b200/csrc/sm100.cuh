@@ -63,14 +63,27 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // CTA's abort flag (shared memory) and the global error word, and returns
 // false; every later bounded wait in the CTA then returns false at once, so
 // all roles leave their loops and reach the common exit, where TMEM is freed.
+// A test hook can name one wait site (fail_site, else -1) whose first wait in
+// each CTA gives up at once, as if its limit had expired, so that the abort
+// path of the real kernels can be exercised without a fault.
 struct WaitGuard {
   volatile int* abort_flag;   // shared memory, one per CTA
   int* err_word;              // global memory
   uint64_t timeout_ns;
+  int fail_site;
 };
+
+// Limit of the exit-path waits (wait_drain): in-flight copies and MMAs always
+// finish, so these keep the full limit whatever the main-loop limit is.
+constexpr uint64_t kDrainTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitGuard& g,
                                              int site) {
+  if (site == g.fail_site) {
+    *g.abort_flag = 1;
+    atomicCAS(g.err_word, 0, kErrDeviceTimeout | (site << 8));
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {

@@ -197,3 +197,32 @@ def test_binding_fails_loudly_without_library(tmp_path):
             binding.load_library(str(tmp_path / "missing.so"))
     finally:
         binding._lib = saved
+
+
+def test_tmem_io_header_is_the_generators_output():
+    """csrc/tmem_io.cuh (the tcgen05.ld / st wrappers) is written by
+    csrc/gen_tmem_io.py; the committed header must be exactly its output."""
+    import subprocess
+    import sys
+    gen = os.path.join(ROOT, "rank_biased_window_b200", "csrc", "gen_tmem_io.py")
+    assert subprocess.run([sys.executable, gen, "--check"]).returncode == 0
+
+
+def test_noalloc_scratch_size_matches_header():
+    """binding.NOALLOC_SCRATCH_BYTES is the header's RFB_NOALLOC_SCRATCH_BYTES."""
+    from rank_biased_window_b200 import binding
+    with open(os.path.join(ROOT, "include", "rfb_attn.h")) as f:
+        m = re.search(r"#define RFB_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", f.read())
+    assert m, "RFB_NOALLOC_SCRATCH_BYTES not found in the header"
+    a, b, c = (int(x) for x in m.groups())
+    assert binding.NOALLOC_SCRATCH_BYTES == a * b * c
+
+
+def test_wait_limit_hook_host_checks(rfb_lib):
+    """The failure-detection hook validates its site on the host and restores
+    the defaults with (0, -1); nothing here touches a GPU."""
+    lib = rfb_lib.load_library()
+    assert lib.rfb_debug_set_wait_limit(0, 256) == 1
+    assert lib.rfb_debug_set_wait_limit(0, -2) == 1
+    assert lib.rfb_debug_set_wait_limit(5, 13) == 0
+    assert lib.rfb_debug_set_wait_limit(0, -1) == 0

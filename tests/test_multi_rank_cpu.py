@@ -129,3 +129,46 @@ def test_shared_bias_gradients_all_reduced_over_two_gloo_ranks():
     for _, du_r, dw_r in got:   # every rank ends with the sum over all windows
         np.testing.assert_allclose(du_r, du.sum(axis=0), rtol=1e-5, atol=1e-6)
         np.testing.assert_allclose(dw_r, dw.sum(axis=0), rtol=1e-5, atol=1e-6)
+
+
+def test_bench_relaunches_itself_for_several_gpus():
+    """`bench.py --gpus 2` outside a torchrun environment starts two local
+    ranks under torch.distributed.run (127.0.0.1); run here with the reference
+    arm (the oracle on the host, no GPU): rank 0 prints one line that counts
+    both ranks, rank 1 exits without work, and the line's config is the one
+    the GPU arm builds for the same workload and rank count."""
+    import json
+    import subprocess
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from rank_biased_window_b200.inputs import WORKLOADS
+    argv = ["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"]
+    cmd = bench.relaunch_argv(argv, 2, 29999)
+    assert cmd[1:5] == ["-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2"]
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-len(argv):] == argv
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", *argv],
+                         capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(s) for s in res.stdout.splitlines() if s.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["config"] == bench.workload_config(WORKLOADS["tiny"], 2)
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_workload_config_is_shared_by_both_arms():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from rank_biased_window_b200.inputs import WORKLOADS
+    c = bench.workload_config(WORKLOADS["train"], 1)
+    assert c["global_batch"] == 2 and c["seq_len"] == 16384 and c["parallelism"] == "single GPU"
+    assert "no flush" in c["l2"]                       # 160 MiB of inputs > L2
+    assert "flush" in bench.workload_config(WORKLOADS["swinir"], 1)["l2"]
+    assert bench.input_bytes(WORKLOADS["train"]) == 4 * 16 * 16384 * 64 * 2 + 2 * 16 * 16384 * 32 * 2
+    assert bench.workload_config(WORKLOADS["train"], 4)["parallelism"] == "replicas x4"
