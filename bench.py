@@ -388,6 +388,8 @@ def run_image_windows(args, rank):
     flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev)
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
     evs = []
+    rfb.profile_read()
+    rfb.profile_enable(True)
     for _ in range(args.steps):
         flush.zero_()
         flush_sum.copy_(flush.view(torch.float32).sum())
@@ -399,6 +401,8 @@ def run_image_windows(args, rank):
         e[2].record()
         evs.append(e)
     torch.cuda.synchronize(dev)
+    rfb.profile_enable(False)
+    prof = rfb.profile_read()
     t_f = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     t_b = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     BH, N = B * (Hs // 8) * (Ws // 8) * nh, 64
@@ -409,6 +413,8 @@ def run_image_windows(args, rank):
             "higher_is_better": True, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t_f + t_b, "fwd_ms": t_f, "bwd_ms": t_b,
             "windows_per_s": B * (Hs // 8) * (Ws // 8) / ((t_f + t_b) * 1e-3),
+            "kernels": {k: {"avg_ms": v[0] / v[1], "launches": v[1]} for k, v in prof.items()
+                        if v[1]},
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) maps, N(0,1/r) factors)",
             "config": {"workload": "image windows", "B": B, "img_h": Hs, "img_w": Ws,
                        "heads": nh, "d": d, "r": r, "win": 8, "shift": shift,

@@ -224,8 +224,8 @@ RFB_API int rfb_attn_fwd_dense_bias(const void* q, const void* k, const void* v,
  *   img_h, img_w : multiples of 8.
  * Errors as rfb_attn_fwd; RFB_ERR_UNSUPPORTED for other win / shift / map
  * sizes, or when the factors of all heads do not fit in shared memory at once
- * ((heads + 1) * 64 * r_pad * 4 bytes beside the input ring; e.g. up to 20
- * heads at r <= 16, 9 at r = 32, 4 at r = 64 for d = 32).
+ * ((heads + 1) * 64 * r_pad * 4 bytes beside the input ring; up to 15 heads
+ * at r <= 16, 7 at r = 32, 3 at r = 64 for d = 32; 11, 5, 2 for d = 64).
  */
 RFB_API int rfb_attn_fwd_image_windows(const void* q, const void* k, const void* v,
                                        const void* u, const void* w, void* o, float* lse, int B,

@@ -31,7 +31,9 @@
 //              MMAs are issued as soon as that half is ready, so one half's
 //              MMAs overlap the other half's softmax.  All MMAs are issued by
 //              one converged warp.
-//   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]).
+//   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]) (with shared
+//              factors dU and dW are instead summed over the windows by
+//              sum_bias_grads_kernel in bwd_window.cuh).
 #pragma once
 #include "fwd_kernels.cuh"
 
@@ -180,40 +182,6 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdArgs a) {
       *reinterpret_cast<uint4*>(a.dq + row * a.D + c) = v;
     else if (a.bias_heads == a.BH)
       *reinterpret_cast<uint4*>(a.du + row * a.r + (c - a.D)) = v;
-  }
-}
-
-// Shared factors: dU[h] = sum_b dU[b H + h] (from the accumulator's dU columns)
-// and dW[h] = sum_b dW[b H + h] (from the fp32 per-window partials), summed in
-// fp32 over b in order, then rounded to bf16.  One thread per 8 values.
-__global__ void __launch_bounds__(256) bwd_post_shared_kernel(const BwdArgs a) {
-  const int H = a.bias_heads, B = a.BH / a.bias_heads;
-  const int DA = a.D + a.r;
-  const int groups = a.r / 8;
-  const long per_mat = static_cast<long>(H) * a.N * groups;
-  for (long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; t < 2 * per_mat;
-       t += static_cast<long>(gridDim.x) * blockDim.x) {
-    const bool is_w = t >= per_mat;
-    const long tt = is_w ? t - per_mat : t;
-    const long hrow = tt / groups;  // h * N + n
-    const int c = static_cast<int>(tt % groups) * 8;
-    float s[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = 0.f;
-    for (int b = 0; b < B; ++b) {
-      const long row = static_cast<long>(b) * H * a.N + hrow;  // (b H + h) N + n
-      const float* src = is_w ? a.dw_part + row * a.r + c : a.acc + row * DA + a.D + c;
-      const float4 x = reinterpret_cast<const float4*>(src)[0];
-      const float4 y = reinterpret_cast<const float4*>(src)[1];
-      s[0] += x.x; s[1] += x.y; s[2] += x.z; s[3] += x.w;
-      s[4] += y.x; s[5] += y.y; s[6] += y.z; s[7] += y.w;
-    }
-    uint4 v;
-    v.x = pack_bf16x2(s[0], s[1]);
-    v.y = pack_bf16x2(s[2], s[3]);
-    v.z = pack_bf16x2(s[4], s[5]);
-    v.w = pack_bf16x2(s[6], s[7]);
-    *reinterpret_cast<uint4*>((is_w ? a.dw : a.du) + hrow * a.r + c) = v;
   }
 }
 

@@ -224,14 +224,19 @@ struct WinCfg {
   static constexpr int QB = kTile * D * 2;    // bytes of a Q / K / V tile
   static constexpr int UB = kTile * RP * 2;   // bytes of a U / W tile
   static constexpr int STAGE = 3 * QB + (IMG ? 0 : 2 * UB);
-  static constexpr int NS_FIT = (224 * 1024) / STAGE;
+  // O of a tile is staged per softmax warpgroup (swizzled like the O tensor
+  // map) and written by TMA stores, one per warp and 32 rows.
+  static constexpr int OB = kTile * D * 2;
+  // Image windows keep every head's factors resident: leave 32 KB for them.
+  static constexpr int NS_FIT = (224 * 1024 - 2 * OB - (IMG ? 32 * 1024 : 0)) / STAGE;
   static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
-  static constexpr int OFF_BAR = NS * STAGE;
+  static constexpr int OFF_OST = NS * STAGE;
+  static constexpr int OFF_BAR = OFF_OST + 2 * OB;
   // TMEM columns: S_a at 128 a, O_a at 256 + D a, P_a (packed bf16) at 384 + 64 a.
   static constexpr int T_O = 256, T_P = 384;
   // in_full[NS] u_ready[NS] in_empty[NS] s_full[2] s_empty[2] p_full[2] o_full[2]
-  // acc_empty[2] drain res_full res_ready
-  static constexpr int NBAR = 3 * NS + 13;
+  // acc_empty[2] drain res_full res_ready exp_turn[2][4]
+  static constexpr int NBAR = 3 * NS + 21;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   // Resident shared factors start after the barriers; one head's U or W rows.
   static constexpr int OFF_RES = (OFF_BAR + NBAR * 8 + 16 + 1023) / 1024 * 1024;
@@ -250,16 +255,18 @@ constexpr uint32_t kWinSoftmaxRegs = 208, kWinControlRegs = 56;
 static_assert(2 * 128 * kWinSoftmaxRegs + 128 * kWinControlRegs <= kWinThreads * 168,
               "register split exceeds the launch budget");
 
-// With IMG the Q / K / V maps are 5-D over the feature maps (D, heads, W, H, B)
-// with a 4 x 4-token box, and U / W 4-D (r, 8, 8, heads) with a 4 x 4 box:
-// each window is copied as four 4 x 4 quadrants, so inside the kernel its
+// With IMG the Q / K / V / O maps are 5-D over the feature maps (D, heads, W,
+// H, B) with a 4 x 4-token box, and U / W 4-D (r, 8, 8, heads) with a 4 x 4
+// box: each window is copied as four 4 x 4 quadrants, so inside the kernel its
 // tokens are in quadrant-major order (row 16 q + 4 (y % 4) + x % 4, q = 2 (y /
 // 4) + x / 4) for Q, K, V, U and W alike; O and LSE go back to map positions.
+// Otherwise mO is the 3-D map of O [BH, N, D] with a 32-row box.
 template <int D, int RP, int NP, bool IMG = false>
 __global__ void __launch_bounds__(kWinThreads, 1)
     fwd_window_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                       const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
-                      const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
+                      const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mO,
+                      const FwdArgs args) {
   using C = WinCfg<D, RP, NP, IMG>;
   constexpr int NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -277,6 +284,9 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (3 * NS + 10);
   const uint32_t res_full = bar0 + 8u * (3 * NS + 11);   // resident factors landed
   const uint32_t res_ready = bar0 + 8u * (3 * NS + 12);  // resident U' scaled
+  // Exponential turns of the two softmax warpgroups, per scheduler (warps w
+  // and w + 4), as in the long kernel.
+  auto exp_turn = [&](int a, int w) { return bar0 + 8u * (3 * NS + 13 + 4 * a + w); };
   const bool resident = RP > 0 && (IMG || args.bias_mode == kBiasResident);
   // Image windows: map coordinates of window-head bh.
   const int nwx = IMG ? args.img_w / 8 : 1, nwy = IMG ? args.img_h / 8 : 1;
@@ -309,6 +319,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       mbar_init(p_full(a), 128);
       mbar_init(o_full(a), 1);
       mbar_init(acc_empty(a), 128);
+      for (int w = 0; w < 4; ++w) mbar_init(exp_turn(a, w), 1);
     }
     mbar_init(drain_bar, 2);
     mbar_init(res_full, 1);
@@ -319,6 +330,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     tma_prefetch(&mQ);
     tma_prefetch(&mK);
     tma_prefetch(&mV);
+    tma_prefetch(&mO);
     if constexpr (RP > 0) {
       tma_prefetch(&mU);
       tma_prefetch(&mW);
@@ -485,6 +497,10 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     const uint32_t p_tm = tmem + lane_base + C::T_P + a * 64;
     const int N = args.N;
     const float sl2 = args.scale_log2;
+    // Warpgroup 0 (even tiles) has the first turn at the exponentials; it has
+    // as many tiles as warpgroup 1 or one more, so the turns always match.
+    const int wq = warp & 3;
+    if (a == 1 && lane == 0) mbar_arrive(exp_turn(0, wq));
     if (resident) {
       // U' = U / s for the resident factors, 16 bytes per thread per step.
       if (wait_warp(res_full, 0, g, 10)) {
@@ -543,9 +559,12 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         }
       }
       const float m = row_max<NP>(sv) * sl2;
+      if (!wait_warp(exp_turn(a, wq), (it >> 1) & 1, g, 22)) break;
       // P_a was last read by PV(it - 2), complete since this warpgroup saw
       // o_full for that tile.
       const float l = exp_row_to_tmem<NP>(sv, sl2, m, p_tm + wl * (NP / 2));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(exp_turn(a ^ 1, wq));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full(a));
@@ -556,11 +575,52 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       tmem_ld_cols<D>(tmem + lane_base + C::T_O + a * D, ov);
       tc_fence_before();
       mbar_arrive(acc_empty(a));
+      // O rows into this warpgroup's staging tile (the TMA store that read the
+      // warp's rows two tiles ago must have finished reading them), then one
+      // TMA store per warp writes its 32 rows.
+      const uint32_t ost = sb + C::OFF_OST + a * C::OB;
+      if (it >= 2) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
+      {
+        const float inv = 1.0f / l;
+#pragma unroll
+        for (int c = 0; c < D; c += 8)
+          st_shared_v4(ost + swz_offset(row, c >> 3, D * 2),
+                       pack_bf16x2(__uint_as_float(ov[c + 0]) * inv, __uint_as_float(ov[c + 1]) * inv),
+                       pack_bf16x2(__uint_as_float(ov[c + 2]) * inv, __uint_as_float(ov[c + 3]) * inv),
+                       pack_bf16x2(__uint_as_float(ov[c + 4]) * inv, __uint_as_float(ov[c + 5]) * inv),
+                       pack_bf16x2(__uint_as_float(ov[c + 6]) * inv, __uint_as_float(ov[c + 7]) * inv));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int r0 = (warp & 3) * 32;           // the warp's first tile row
+        const int wwin = t * C::NW + r0 / NP;     // its window
+        const int n0 = r0 % NP;                   // its first token in the window
+        if (wwin < args.BH && n0 < N) {
+          if constexpr (IMG) {
+            int b, wy, wx, h;
+            window_of(wwin, b, wy, wx, h);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int qd = (n0 >> 4) + k;
+              const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
+              const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+              tma_store_5d(&mO, ost + (r0 + 16 * k) * (D * 2), 0, h, x, y, b);
+            }
+          } else {
+            tma_store_3d(&mO, ost + r0 * (D * 2), 0, n0, wwin);
+          }
+        }
+        bulk_commit();
+      }
       const int win = t * C::NW + wl;
       if (win < args.BH && n < N) {
         size_t r = static_cast<size_t>(win) * N + n;
         if constexpr (IMG) {
-          // back to the token's place in the unrolled map
+          // the token's place in the unrolled map
           int b, wy, wx, h;
           window_of(win, b, wy, wx, h);
           const int qq = n >> 4;
@@ -568,10 +628,11 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           const int x = (wx * 8 + 4 * (qq & 1) + (n & 3) + args.shift) % args.img_w;
           r = ((static_cast<size_t>(b) * args.img_h + y) * args.img_w + x) * args.img_heads + h;
         }
-        store_o_row<D>(args.o + r * D, ov, 1.0f / l);
         args.lse[r] = (m + __log2f(l)) * kLn2;
       }
     }
+    // The O stores must have finished before the CTA exits.
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -612,8 +673,8 @@ struct LongCfg {
   static_assert(T_O + 2 * OD <= T_P, "TMEM budget");
   static_assert(OFF_ONES % 1024 == 0, "ones block alignment");
   // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
-  // q_empty o_empty[2]
-  static constexpr int NBAR = 2 * NS + 13;
+  // q_empty o_empty[2] exp_turn[2][4]
+  static constexpr int NBAR = 2 * NS + 21;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static_assert(NS >= 2, "not enough shared memory for two KV stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
@@ -664,6 +725,10 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   // epilogue has read O (the next unit's first PV may overwrite it).
   const uint32_t q_empty = bar0 + 8u * (10 + 2 * NS);
   auto o_empty = [&](int t) { return bar0 + 8u * (11 + 2 * NS + t); };
+  // Exponential turns: warp w of softmax warpgroup t may start its exponentials
+  // of a tile once exp_turn(t, w) has completed the phase of that tile; the
+  // two warps that share a scheduler (w and w + 4) hand the turn to each other.
+  auto exp_turn = [&](int t, int w) { return bar0 + 8u * (13 + 2 * NS + 4 * t + w); };
   auto q_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB); };
   auto u_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB) + C::QB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
@@ -693,6 +758,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       mbar_init(p_full(t), 128);
       mbar_init(pv_done(t), 1);
       mbar_init(o_empty(t), 128);
+      for (int w = 0; w < 4; ++w) mbar_init(exp_turn(t, w), 1);
     }
     mbar_init(drain_bar, 2);
     fence_mbar_init();
@@ -834,6 +900,13 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     // Scores are accumulator * sl2 in log2 units; the comparator adds its bias
     // to the scaled scores first and then uses a unit factor.
     const float sl2 = DENSE ? 1.0f : args.scale_log2;
+    // The two warpgroups take turns at the exponentials, warp by warp on each
+    // scheduler (warps w and w + 4): warpgroup 0 has the first turn.  While one
+    // runs its exponentials (the MUFU-bound phase) the other loads scores,
+    // takes row maxima and waits for its MMAs, so the phases overlap instead
+    // of both warpgroups contending for the exponential unit at once.
+    const int wq = warp & 3;
+    if (t == 1 && lane == 0) mbar_arrive(exp_turn(0, wq));
     int jt = 0;  // S tiles of this query tile so far (= K/V tiles of the CTA)
     bool ok = true;
     for (int u = first; ok && u < nunits; u += stride) {
@@ -882,9 +955,12 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
         // The P buffer of this tile and O: the previous PV must have finished.
         if (jt >= 1 && !wait_warp(pv_done(t), (jt - 1) & 1, g, 17)) { ok = false; break; }
+        if (!wait_warp(exp_turn(t, wq), jt & 1, g, 21)) { ok = false; break; }
         tc_fence_after();
         if constexpr (C::LCOL) exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
         else l += exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(exp_turn(t ^ 1, wq));
         if (fix_o) {
           uint32_t ov[D];
           tmem_ld_cols<D>(o_tm, ov);

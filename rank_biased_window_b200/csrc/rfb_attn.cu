@@ -15,6 +15,7 @@
 
 #include "rfb_attn.h"
 #include "bwd_kernels.cuh"
+#include "bwd_window.cuh"
 #include "fwd_kernels.cuh"
 
 namespace rfb {
@@ -344,7 +345,7 @@ struct LaunchTimer {
 };
 
 struct Maps {
-  CUtensorMap q, k, v, u, w, g, acc;
+  CUtensorMap q, k, v, u, w, g, acc, o;
 };
 
 // ---------------------------------------------------------------- forward
@@ -369,7 +370,8 @@ int launch_window(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
     }
   }
   LaunchTimer timer(kIdFwd, st);
-  fwd_window_kernel<D, RP, NP><<<grid, kWinThreads, smem, st>>>(m.q, m.k, m.v, m.u, m.w, args);
+  fwd_window_kernel<D, RP, NP><<<grid, kWinThreads, smem, st>>>(m.q, m.k, m.v, m.u, m.w, m.o,
+                                                                 args);
   return launch_status();
 }
 
@@ -400,7 +402,7 @@ int launch_window_img(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st)
   const int grid = tiles < sms ? tiles : sms;
   LaunchTimer timer(kIdFwd, st);
   fwd_window_kernel<D, RP, 64, true><<<grid, kWinThreads, static_cast<int>(need), st>>>(
-      m.q, m.k, m.v, m.u, m.w, a);
+      m.q, m.k, m.v, m.u, m.w, m.o, a);
   return launch_status();
 }
 
@@ -489,6 +491,38 @@ int dispatch_bwd_main(int d, int rp, const Maps& m, const BwdArgs& a, cudaStream
   return RFB_ERR_UNSUPPORTED;
 }
 
+// Window backward (d = 32, r_pad <= 16, N <= 128): one persistent kernel.
+struct WinBwdMaps {
+  CUtensorMap q, k, v, g, o, u, w, dq, dk, dv;
+};
+
+template <int RP, int NP, bool IMG>
+int launch_bwd_window(const WinBwdMaps& m, const BwdWinArgs& a, int sms, cudaStream_t st) {
+  using C = BwdWinCfg<RP, NP, IMG>;
+  static std::atomic<uint64_t> done{0};
+  if (int rc = ensure_smem(bwd_window_kernel<RP, NP, IMG>, C::SMEM, done)) return rc;
+  const int tiles = (a.BH + C::NW - 1) / C::NW;
+  const int grid = tiles < sms ? tiles : sms;
+  LaunchTimer timer(kIdBwdMain, st);
+  bwd_window_kernel<RP, NP, IMG><<<grid, kBwdWinThreads, C::SMEM, st>>>(
+      m.q, m.k, m.v, m.g, m.o, m.u, m.w, m.dq, m.dk, m.dv, a);
+  return launch_status();
+}
+
+int dispatch_bwd_window(int rp, int N, bool img, const WinBwdMaps& m, const BwdWinArgs& a, int sms,
+                        cudaStream_t st) {
+  if (img) return rp == 0 ? launch_bwd_window<0, 64, true>(m, a, sms, st)
+                          : launch_bwd_window<16, 64, true>(m, a, sms, st);
+  if (N <= 64)
+    return rp == 0 ? launch_bwd_window<0, 64, false>(m, a, sms, st)
+                   : launch_bwd_window<16, 64, false>(m, a, sms, st);
+  return rp == 0 ? launch_bwd_window<0, 128, false>(m, a, sms, st)
+                 : launch_bwd_window<16, 128, false>(m, a, sms, st);
+}
+
+// Whether the window backward takes these sizes.
+bool window_bwd_ok(int N, int d, int rp) { return d == 32 && rp <= 16 && N <= kTile; }
+
 int grid_for(long long work, int per_block, int sms) {
   long long g = (work + per_block - 1) / per_block;
   const long long cap = static_cast<long long>(sms) * 8;
@@ -546,6 +580,8 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, const void* u, co
   int rc = encode_3d(&m.q, q, d, N, BH, d, rows, heads);
   if (!rc) rc = encode_3d(&m.k, k, d, N, BH, d, rows, heads);
   if (!rc) rc = encode_3d(&m.v, v, d, N, BH, d, rows, heads);
+  // The window kernel writes O by TMA stores of 32 rows.
+  if (!rc && N <= kTile) rc = encode_3d(&m.o, o, d, N, BH, d, 32, 1);
   // Shared factors: [H, N, r], one window's rows per copy.
   const int bias_heads = shared ? H : BH;
   const int bias_box = shared ? 1 : heads;
@@ -597,6 +633,54 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
   const int BH = B * H;
   const int bias_heads = shared ? H : BH;
   const int rp = pad_rank(r);
+  if (!img_mask && window_bwd_ok(N, d, rp)) {
+    // Whole windows per tile: one kernel, plus the sum over the windows of the
+    // shared factors' gradients.
+    const int np = N <= 64 ? 64 : kTile, nw = kTile / np;
+    WinBwdMaps wm;
+    std::memset(&wm, 0, sizeof(wm));
+    int rc = encode_3d(&wm.q, q, d, N, BH, d, np, nw);
+    if (!rc) rc = encode_3d(&wm.k, k, d, N, BH, d, np, nw);
+    if (!rc) rc = encode_3d(&wm.v, v, d, N, BH, d, np, nw);
+    if (!rc) rc = encode_3d(&wm.g, dout, d, N, BH, d, np, nw);
+    if (!rc) rc = encode_3d(&wm.o, o, d, N, BH, d, np, nw);
+    if (!rc && r > 0) rc = encode_3d(&wm.u, u, r, N, bias_heads, d, np, shared ? 1 : nw);
+    if (!rc && r > 0) rc = encode_3d(&wm.w, w, r, N, bias_heads, d, np, shared ? 1 : nw);
+    if (!rc) rc = encode_3d(&wm.dq, dq, d, N, BH, d, 32, 1);
+    if (!rc) rc = encode_3d(&wm.dk, dk, d, N, BH, d, 32, 1);
+    if (!rc) rc = encode_3d(&wm.dv, dv, d, N, BH, d, 32, 1);
+    if (rc) return rc;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    BwdWinArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.lse = lse;
+    a.du = static_cast<__nv_bfloat16*>(du);
+    a.dw = static_cast<__nv_bfloat16*>(dw);
+    if (shared && r > 0) {  // fp32 rows per window-head in the workspace
+      a.du_part = reinterpret_cast<float*>(ws + L.acc);
+      a.dw_part = reinterpret_cast<float*>(ws + L.dw_part);
+    }
+    a.err = dev.err_word;
+    a.BH = BH;
+    a.N = N;
+    a.r = r;
+    a.bias_heads = bias_heads;
+    a.shared = shared ? 1 : 0;
+    a.img_heads = 1;
+    a.scale = scale;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.inv_scale = 1.0f / scale;
+    a.timeout_ns = g_wait_limit_ns.load();
+    a.fail_site = g_fail_site.load();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = dispatch_bwd_window(rp, N, false, wm, a, dev.sms, st))) return rc;
+    if (shared && r > 0) {
+      LaunchTimer timer(kIdBwdPost, st);
+      sum_bias_grads_kernel<<<H * N, 256, 0, st>>>(a.du_part, r, a.dw_part, r, a.du, a.dw, B, H,
+                                                   N, r);
+    }
+    return launch_status();
+  }
   Maps m;
   std::memset(&m, 0, sizeof(m));
   int rc = encode_3d(&m.q, q, d, N, BH, d, kTile, 1);
@@ -658,8 +742,9 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
     bwd_post_kernel<<<grid_for(groups, 256, dev.sms), 256, 0, st>>>(a);
     if (shared && r > 0) {
       if ((rc = launch_status())) return rc;
-      const long long sgroups = 2LL * H * N * (r / 8);
-      bwd_post_shared_kernel<<<grid_for(sgroups, 256, dev.sms), 256, 0, st>>>(a);
+      // dU from the accumulator's dU columns, dW from the per-window fp32 rows
+      sum_bias_grads_kernel<<<H * N, 256, 0, st>>>(a.acc + d, d + r, a.dw_part, r, a.du, a.dw, B,
+                                                   H, N, r);
     }
   }
   return launch_status();
@@ -794,6 +879,7 @@ int rfb_attn_fwd_image_windows(const void* q, const void* k, const void* v, cons
   int rc = encode_nd(&m.q, q, 5, dims, strides, box);
   if (!rc) rc = encode_nd(&m.k, k, 5, dims, strides, box);
   if (!rc) rc = encode_nd(&m.v, v, 5, dims, strides, box);
+  if (!rc) rc = encode_nd(&m.o, o, 5, dims, strides, box);
   if (!rc && r > 0) {
     // U, W [heads, 64, r] as (r, 8, 8, heads), a 4 x 4 box.
     const cuuint64_t udims[4] = {static_cast<cuuint64_t>(r), 8, 8, static_cast<cuuint64_t>(heads)};
@@ -881,6 +967,75 @@ int rfb_attn_bwd_image_windows(const void* q, const void* k, const void* v, cons
   DeviceInfo dev;
   if (int rc = device_info(&dev)) return rc;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int rp = pad_rank(r);
+  if (window_bwd_ok(64, d, rp)) {
+    // One kernel gathers the rolled windows from the maps and scatters dQ, dK,
+    // dV back in its TMA addressing; the factors' fp32 rows per window-head go
+    // to the workspace and are summed over the windows afterwards.
+    WinBwdMaps wm;
+    std::memset(&wm, 0, sizeof(wm));
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(img_w), static_cast<cuuint64_t>(img_h),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t rowb = static_cast<cuuint64_t>(d) * 2;
+    const cuuint64_t strides[4] = {rowb, rowb * heads, rowb * heads * img_w,
+                                   rowb * heads * img_w * img_h};
+    const cuuint32_t box[5] = {static_cast<cuuint32_t>(d), 1, 4, 4, 1};
+    int rc = encode_nd(&wm.q, q, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.k, k, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.v, v, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.g, dout, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.o, o, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.dq, dq, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.dk, dk, 5, dims, strides, box);
+    if (!rc) rc = encode_nd(&wm.dv, dv, 5, dims, strides, box);
+    if (!rc && r > 0) {
+      // U, W [heads, 64, r] as (r, 8, 8, heads), a 4 x 4 box 32 columns wide
+      // (zero filled beyond r)
+      const cuuint64_t udims[4] = {static_cast<cuuint64_t>(r), 8, 8,
+                                   static_cast<cuuint64_t>(heads)};
+      const cuuint64_t urow = static_cast<cuuint64_t>(r) * 2;
+      const cuuint64_t ustr[3] = {urow, urow * 8, urow * 64};
+      const cuuint32_t ubox[4] = {static_cast<cuuint32_t>(d), 4, 4, 1};
+      rc = encode_nd(&wm.u, u, 4, udims, ustr, ubox);
+      if (!rc) rc = encode_nd(&wm.w, w, 4, udims, ustr, ubox);
+    }
+    if (rc) return rc;
+    const int nwin = static_cast<int>(bh / heads);
+    const WsLayout inner = ws_layout(nwin, heads, 64, d, r, true);
+    BwdWinArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.lse = lse;
+    a.du = static_cast<__nv_bfloat16*>(du);
+    a.dw = static_cast<__nv_bfloat16*>(dw);
+    if (r > 0) {
+      a.du_part = reinterpret_cast<float*>(ws + L.inner + inner.acc);
+      a.dw_part = reinterpret_cast<float*>(ws + L.inner + inner.dw_part);
+    }
+    a.err = dev.err_word;
+    a.BH = static_cast<int>(bh);
+    a.N = 64;
+    a.r = r;
+    a.bias_heads = heads;
+    a.shared = 1;
+    a.img_h = img_h;
+    a.img_w = img_w;
+    a.img_heads = heads;
+    a.shift = shift;
+    a.scale = scale;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.inv_scale = 1.0f / scale;
+    a.timeout_ns = g_wait_limit_ns.load();
+    a.fail_site = g_fail_site.load();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = dispatch_bwd_window(rp, 64, true, wm, a, dev.sms, st))) return rc;
+    if (r > 0) {
+      LaunchTimer timer(kIdBwdPost, st);
+      sum_bias_grads_kernel<<<heads * 64, 256, 0, st>>>(a.du_part, r, a.dw_part, r, a.du, a.dw,
+                                                        nwin, heads, 64, r);
+    }
+    return launch_status();
+  }
   auto wt = [&](int i) { return reinterpret_cast<__nv_bfloat16*>(ws + L.win[i]); };
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long pieces = bh * 64 * (d / 8);

@@ -165,6 +165,25 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32
       "r"(src), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// Bulk tensor stores shared -> global (tile mode), tracked with the bulk
+// async-group mechanism of the issuing thread.  Elements outside the tensor
+// are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -295,6 +314,16 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows) {
   const int chunk = (col & 63) >> 3;
   return static_cast<uint32_t>(blk * rows * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) +
                                ((col & 7) << 1));
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile of rows
+// `row_bytes` wide (32, 64 or 128), stored with the matching TMA swizzle
+// (the tile starts on a 1024-byte boundary): the chunk index is XORed with
+// address bits 7 and up.
+__device__ __forceinline__ uint32_t swz_offset(int row, int chunk, int row_bytes) {
+  const int line = (row * row_bytes) >> 7;  // 128-byte line of the row
+  const int x = row_bytes == 128 ? (line & 7) : row_bytes == 64 ? (line & 3) : (line & 1);
+  return static_cast<uint32_t>(row * row_bytes + ((chunk ^ x) << 4));
 }
 
 // -------------------------------------------------------------- numerics

@@ -36,6 +36,11 @@ CASES = [
     (1, 1, 200, 64, 64),   # dQ|dU share the S^T columns (no room for their own)
     (1, 2, 130, 64, 16),
     (3, 1, 64, 32, 0),
+    # windows of <= 128 tokens with d = 32, r <= 16 (the window backward)
+    (2, 3, 100, 32, 16),
+    (5, 1, 33, 32, 8),
+    (4, 6, 64, 32, 16),
+    (2, 2, 128, 32, 0),
 ]
 
 
@@ -111,3 +116,16 @@ def test_autograd_function(rfb_lib, oracle_mod, cuda_dev):
     ref = oracle_mod.bwd(f["q"], f["k"], f["v"], f["u"], f["w"], f["dout"], 1 / math.sqrt(d))
     for name, t, want in zip("qkvuw", (g["q"], g["k"], g["v"], g["u"], g["w"]), ref):
         assert_close("d" + name, t.grad, want)
+
+
+def test_swinir_shaped_window_backward(rfb_lib, oracle_mod, cuda_dev):
+    """64 SwinIR-style 8 x 8 windows, 6 heads, d = 32, r = 8 (the window
+    backward, two windows per tile): every gradient against the oracle."""
+    B, H, N, d, r = 64, 6, 64, 32, 8
+    x = make_inputs(B, H, N, d, r, seed=2600, with_dout=True)
+    s = 1.0 / math.sqrt(d)
+    _, _, grads = _gpu_fwd_bwd(rfb_lib, x, cuda_dev, s, r)
+    f = {k: to_f64(v) for k, v in x.items()}
+    ref = oracle_mod.bwd(f["q"], f["k"], f["v"], f["u"], f["w"], f["dout"], s)
+    for name, got, want in zip(("dQ", "dK", "dV", "dU", "dW"), grads, ref):
+        assert_close(name, got, want)

@@ -83,6 +83,8 @@ BWD_CASES = [
     (1, 24, 16, 6, 32, 8, 4),    # SwinIR-like heads
     (2, 16, 16, 1, 64, 0, 4),    # no bias
     (1, 16, 16, 2, 64, 32, 4),
+    (2, 32, 32, 6, 32, 8, 4),    # 32 windows x 6 heads, SwinIR-sized windows
+    (1, 16, 24, 2, 32, 0, 4),    # d = 32 without bias
 ]
 
 

@@ -42,6 +42,8 @@ CASES = [
     (2, 3, 130, 32, 16),
     (4, 1, 128, 64, 64),
     (1, 2, 64, 32, 0),    # no bias: same as the per-window path
+    (4, 6, 64, 32, 8),    # window backward, two windows per tile, heads wrapping
+    (3, 2, 100, 32, 16),  # window backward, one window per tile
 ]
 
 
