@@ -284,11 +284,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(sdp_full(h), 1);
-      mbar_init(ds_full(h), 128);
+      mbar_init(ds_full(h), 4);   // one arrival per warp of the half's warpgroup
       mbar_init(a_done(h), 1);
     }
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 256);
+    mbar_init(dq_free, 8);        // one arrival per compute warp
     mbar_init(drain_bar, 1);
     fence_mbar_init();
   }
@@ -551,7 +551,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(ds_full(wg));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full(wg));
       return true;
     };
     // Partial dQ | dU of tile j (TMEM lane = query row): this warpgroup reads its
@@ -572,7 +573,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (ch < C::NCH) tmem_ld32(tmem + lane_base + C::T_DQ + ch * 32, z[m]);
       }
       tc_fence_before();
-      mbar_arrive(dq_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
 #pragma unroll
       for (int m = 0; m < MY_MAX; ++m) {
         const int ch = wg + 2 * m;

@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
     mbar_init(sdp_full, 1);
     mbar_init(ds_full, 4);      // one arrival per compute warp
     mbar_init(grad_full, 1);
-    mbar_init(grad_free, 128);
+    mbar_init(grad_free, 4);    // one arrival per compute warp
     mbar_init(vec_full(0), 4);
     mbar_init(vec_full(1), 4);
     mbar_init(drain_bar, 1);
@@ -441,7 +441,8 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       tmem_ld_any<D + RP>(tmem + lane_base + C::T_DK, gk);
       tmem_ld_any<D + RP>(tmem + lane_base + C::T_DQ, gq);
       tc_fence_before();
-      mbar_arrive(grad_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(grad_free);
       // dQ = s dS K (query rows), dK = s dS^T Q, dV = P^T dO (key rows): staged
       // in this warp's rows of the dS tile, which the gradient MMAs have read.
       stage_row32(stg_q, lane, gq, args.scale);

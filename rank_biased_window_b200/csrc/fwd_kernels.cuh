@@ -235,8 +235,8 @@ struct WinCfg {
   // TMEM columns: S_a at 128 a, O_a at 256 + D a, P_a (packed bf16) at 384 + 64 a.
   static constexpr int T_O = 256, T_P = 384;
   // in_full[NS] u_ready[NS] in_empty[NS] s_full[2] s_empty[2] p_full[2] o_full[2]
-  // acc_empty[2] drain res_full res_ready exp_turn[2][4]
-  static constexpr int NBAR = 3 * NS + 21;
+  // acc_empty[2] drain res_full res_ready
+  static constexpr int NBAR = 3 * NS + 13;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   // Resident shared factors start after the barriers; one head's U or W rows.
   static constexpr int OFF_RES = (OFF_BAR + NBAR * 8 + 16 + 1023) / 1024 * 1024;
@@ -284,9 +284,6 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (3 * NS + 10);
   const uint32_t res_full = bar0 + 8u * (3 * NS + 11);   // resident factors landed
   const uint32_t res_ready = bar0 + 8u * (3 * NS + 12);  // resident U' scaled
-  // Exponential turns of the two softmax warpgroups, per scheduler (warps w
-  // and w + 4), as in the long kernel.
-  auto exp_turn = [&](int a, int w) { return bar0 + 8u * (3 * NS + 13 + 4 * a + w); };
   const bool resident = RP > 0 && (IMG || args.bias_mode == kBiasResident);
   // Image windows: map coordinates of window-head bh.
   const int nwx = IMG ? args.img_w / 8 : 1, nwy = IMG ? args.img_h / 8 : 1;
@@ -315,11 +312,10 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(s_full(a), 1);
-      mbar_init(s_empty(a), 128);
-      mbar_init(p_full(a), 128);
+      mbar_init(s_empty(a), 4);   // one arrival per softmax warp
+      mbar_init(p_full(a), 4);
       mbar_init(o_full(a), 1);
-      mbar_init(acc_empty(a), 128);
-      for (int w = 0; w < 4; ++w) mbar_init(exp_turn(a, w), 1);
+      mbar_init(acc_empty(a), 4);
     }
     mbar_init(drain_bar, 2);
     mbar_init(res_full, 1);
@@ -497,10 +493,6 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     const uint32_t p_tm = tmem + lane_base + C::T_P + a * 64;
     const int N = args.N;
     const float sl2 = args.scale_log2;
-    // Warpgroup 0 (even tiles) has the first turn at the exponentials; it has
-    // as many tiles as warpgroup 1 or one more, so the turns always match.
-    const int wq = warp & 3;
-    if (a == 1 && lane == 0) mbar_arrive(exp_turn(0, wq));
     if (resident) {
       // U' = U / s for the resident factors, 16 bytes per thread per step.
       if (wait_warp(res_full, 0, g, 10)) {
@@ -536,7 +528,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       uint32_t sv[NP];
       tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
       tc_fence_before();
-      mbar_arrive(s_empty(a));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty(a));
       if (N < NP) mask_tail<NP>(sv, N);
       if constexpr (IMG) {
         // Shifted-window mask: in the last window row (column) of the rolled
@@ -559,22 +552,21 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         }
       }
       const float m = row_max<NP>(sv) * sl2;
-      if (!wait_warp(exp_turn(a, wq), (it >> 1) & 1, g, 22)) break;
       // P_a was last read by PV(it - 2), complete since this warpgroup saw
       // o_full for that tile.
       const float l = exp_row_to_tmem<NP>(sv, sl2, m, p_tm + wl * (NP / 2));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(exp_turn(a ^ 1, wq));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full(a));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full(a));
       // Epilogue of this tile once its PV has landed.
       if (!wait_warp(o_full(a), (it >> 1) & 1, g, 6)) break;
       tc_fence_after();
       uint32_t ov[D];
       tmem_ld_cols<D>(tmem + lane_base + C::T_O + a * D, ov);
       tc_fence_before();
-      mbar_arrive(acc_empty(a));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(a));
       // O rows into this warpgroup's staging tile (the TMA store that read the
       // warp's rows two tiles ago must have finished reading them), then one
       // TMA store per warp writes its 32 rows.
@@ -655,53 +647,64 @@ struct LongCfg {
   static constexpr int BT = DENSE ? kTile * kTile * 2 : 0;  // one query tile's bias tile
   static constexpr int OFF_BIAS = 2 * QB + UB;                // within a stage
   static constexpr int STAGE = 2 * QB + UB + 2 * BT;        // K, V, W, bias tiles
-  // Two query tiles per CTA: Q0 U0 Q1 U1, then the KV stages.  P lives in TMEM.
-  static constexpr int OFF_Q = 0;            // Q tile t at OFF_Q + t * (QB + UB), U right after
-  static constexpr int OFF_STAGE = 2 * (QB + UB);
+  // Two query tiles per unit: Q0 U0 Q1 U1, in QSETS sets so that the next
+  // unit's tiles load while the current unit runs -- for d = 32, where the
+  // K/V ring keeps its six stages; with d = 64 a second set would cost a K/V
+  // stage, which measured slower.  Then the K/V stages.  P lives in TMEM.
+  static constexpr int QSETS = (D == 32 && !DENSE) ? 2 : 1;
+  static constexpr int OFF_Q = 0;  // set b, tile t at OFF_Q + (2 b + t) (QB + UB), U right after Q
+  static constexpr int OFF_STAGE = QSETS * 2 * (QB + UB);
   // With d = 32 the row sums come out of the PV MMA: B is [V | 1] (a constant
   // 128 x 32 block of ones as a second MN block, N = d + 16), so column d of
   // the O accumulator collects sum_j bf16(p_j) and the softmax adds nothing.
   static constexpr bool LCOL = (D == 32);
   static constexpr int OD = LCOL ? D + 16 : D;  // O accumulator columns per query tile
   static constexpr int ONES = LCOL ? kTile * 64 : 0;
-  static constexpr int NS_FIT = (226 * 1024 - OFF_STAGE - ONES) / STAGE;
+  // Shared-memory exchange between the two key-half warpgroups of a query
+  // tile: half-row maxima [t][h][128] (and, at the end of a unit, key half
+  // 1's row sums in the [t][0] slots).
+  static constexpr int XCH = 2 * 2 * kTile * 4;
+  static constexpr int NS_FIT = (232448 - 256 - OFF_STAGE - ONES - XCH) / STAGE;
   static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
   static constexpr int OFF_ONES = OFF_STAGE + NS * STAGE;  // 1024-byte aligned
-  static constexpr int OFF_BAR = OFF_ONES + ONES;
+  static constexpr int OFF_MAX = OFF_ONES + ONES;
+  static constexpr int OFF_BAR = OFF_MAX + XCH;
   // TMEM columns: S_t at 128 t, O_t at 256 + OD t, P_t (packed bf16) at 384 + 64 t.
   static constexpr int T_O = 256, T_P = 384;
   static_assert(T_O + 2 * OD <= T_P, "TMEM budget");
   static_assert(OFF_ONES % 1024 == 0, "ones block alignment");
-  // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] drain
-  // q_empty o_empty[2] exp_turn[2][4]
-  static constexpr int NBAR = 2 * NS + 21;
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  // q_full kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] mx_full[2] p_full[2]
+  // pv_done[2] drain q_empty o_empty[2] sum_full[2] q_full' q_empty' (second set)
+  static constexpr int NBAR = 2 * NS + 19;
+  // The dynamic shared memory is declared 1024-byte aligned and used without
+  // slack (checked on entry).
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
   static_assert(NS >= 2, "not enough shared memory for two KV stages");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
 };
 
-// Warpgroups 0 / 1: softmax of query tile 0 / 1; warpgroup 2: warp 8 TMA, warps
-// 9 / 10 MMA issue for tile 0 / 1, warp 11 idle.  Registers: launched with 168
-// per thread (384 x 168 = 64512); warpgroup 2 gives its share down to 56 and
-// the softmax warpgroups take 208 (2 x 128 x 208 + 128 x 56 = 60416 <= 64512).
-constexpr int kLongThreads = 384;
-constexpr uint32_t kLongSoftmaxRegs = 208, kLongControlRegs = 56;
-static_assert(2 * 128 * kLongSoftmaxRegs + 128 * kLongControlRegs <= kLongThreads * 168,
-              "register split exceeds the launch budget");
+// Warps 0-15: four softmax warpgroups, warpgroup g = 2 t + h takes query tile t
+// and key half h (keys 64 h .. 64 h + 63 of every 128-key tile); warp 16 TMA
+// producer; warps 17 / 18 MMA issue for query tiles 0 / 1.  A query tile's
+// exponentials are shared by two warps on every scheduler, which keeps the
+// exponential unit busier than one warp can; the other query tile's
+// warpgroups meanwhile load scores, take maxima and wait for their MMAs.
+constexpr int kLongThreads = 608;
 // Pairs of every 4 softmax exponentials computed in software in the long
-// forward (the MUFU unit is its limit): one, measured best for d = 32 and 64.
+// forward (the MUFU unit is its limit).
 constexpr int kLongSoftPairs = 1;
 
 // Long regime: a persistent CTA per SM works through units (head, pair of
-// 128-query tiles), each a loop over 128-key tiles.  Each query tile of a unit
-// has its own softmax warpgroup, MMA-issuing warp, S buffer (TMEM columns
-// t*128), O accumulator (TMEM 256 + t*OD) and P buffer (TMEM 384 + 64 t); the two
-// pipelines run independently and out of phase, so one's exponentials overlap
-// the other's loads, maxima and waits, and each K/V tile serves 256 query rows.
-// Barrier phases run on across units, so the K/V loads and the scores of the
-// next unit start while the current unit's last tiles and epilogue finish.
-// With DENSE (the comparator) mU is the map of the dense bias [bias heads, N,
-// N] (box 64 x 128) and mW is unused.
+// 128-query tiles), each a loop over 128-key tiles.  Each query tile t has an
+// MMA-issuing warp, an S buffer (TMEM columns 128 t), an O accumulator, a P
+// buffer and two softmax warpgroups, one per key half of every tile; the two
+// exchange their half-row maxima through shared memory so that both apply the
+// same running maximum (online softmax with a lazy rescale of O, done by the
+// key-half-0 warpgroup), and each keeps the row sums of its half.  The next
+// tile's scores are issued as soon as both halves have loaded S, so they
+// overlap the exponentials; each K/V tile serves 256 query rows.  Barrier
+// phases run on across units.  With DENSE (the comparator) mU is the map of the
+// dense bias [bias heads, N, N] (box 64 x 128) and mW is unused.
 template <int D, int RP, bool DENSE = false>
 __global__ void __launch_bounds__(kLongThreads, 1)
     fwd_long_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
@@ -709,28 +712,32 @@ __global__ void __launch_bounds__(kLongThreads, 1)
                     const __grid_constant__ CUtensorMap mW, const FwdArgs args) {
   using C = LongCfg<D, RP, DENSE>;
   constexpr int NS = C::NS;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align_1024(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sb = smem_u32(smem);
+  if (sb & 1023u) {  // the swizzled operand tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(args.err, 0, kErrAlignment | (97 << 8));
+    return;
+  }
   const uint32_t bar0 = sb + C::OFF_BAR;
-  const uint32_t q_full = bar0;
+  // Q / U' set b loaded, and read by the unit's last score MMAs.
+  auto q_full = [&](int b) { return b == 0 ? bar0 : bar0 + 8u * (17 + 2 * NS); };
   auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto kv_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
   auto s_full = [&](int t) { return bar0 + 8u * (1 + 2 * NS + t); };
   auto s_empty = [&](int t) { return bar0 + 8u * (3 + 2 * NS + t); };
-  auto p_full = [&](int t) { return bar0 + 8u * (5 + 2 * NS + t); };
-  auto pv_done = [&](int t) { return bar0 + 8u * (7 + 2 * NS + t); };
-  const uint32_t drain_bar = bar0 + 8u * (9 + 2 * NS);
-  // The unit's last score MMAs are done (Q / U' may be replaced), and tile t's
-  // epilogue has read O (the next unit's first PV may overwrite it).
-  const uint32_t q_empty = bar0 + 8u * (10 + 2 * NS);
-  auto o_empty = [&](int t) { return bar0 + 8u * (11 + 2 * NS + t); };
-  // Exponential turns: warp w of softmax warpgroup t may start its exponentials
-  // of a tile once exp_turn(t, w) has completed the phase of that tile; the
-  // two warps that share a scheduler (w and w + 4) hand the turn to each other.
-  auto exp_turn = [&](int t, int w) { return bar0 + 8u * (13 + 2 * NS + 4 * t + w); };
-  auto q_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB); };
-  auto u_addr = [&](int t) { return sb + C::OFF_Q + t * (C::QB + C::UB) + C::QB; };
+  auto mx_full = [&](int t) { return bar0 + 8u * (5 + 2 * NS + t); };
+  auto p_full = [&](int t) { return bar0 + 8u * (7 + 2 * NS + t); };
+  auto pv_done = [&](int t) { return bar0 + 8u * (9 + 2 * NS + t); };
+  const uint32_t drain_bar = bar0 + 8u * (11 + 2 * NS);
+  // The unit's last score MMAs are done (Q / U' may be replaced); tile t's
+  // epilogue has read O (the next unit's first PV may overwrite it); the key
+  // half-1 row sums of tile t are in shared memory.
+  auto q_empty = [&](int b) { return bar0 + 8u * (b == 0 ? 12 + 2 * NS : 18 + 2 * NS); };
+  auto o_empty = [&](int t) { return bar0 + 8u * (13 + 2 * NS + t); };
+  auto sum_full = [&](int t) { return bar0 + 8u * (15 + 2 * NS + t); };
+  auto q_addr = [&](int b, int t) { return sb + C::OFF_Q + (2 * b + t) * (C::QB + C::UB); };
+  auto u_addr = [&](int b, int t) { return q_addr(b, t) + C::QB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -746,19 +753,23 @@ __global__ void __launch_bounds__(kLongThreads, 1)
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 2);  // one commit per query tile's MMA warp
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full(b), 1);
+      mbar_init(q_empty(b), 2);  // one commit per query tile's MMA warp
+    }
     for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 2);  // one arrival per query tile's MMA warp
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full(t), 1);
-      mbar_init(s_empty(t), 128);
-      mbar_init(p_full(t), 128);
+      // one arrival per warp (lane 0, after __syncwarp), both key halves
+      mbar_init(s_empty(t), 8);
+      mbar_init(mx_full(t), 8);
+      mbar_init(p_full(t), 8);
       mbar_init(pv_done(t), 1);
-      mbar_init(o_empty(t), 128);
-      for (int w = 0; w < 4; ++w) mbar_init(exp_turn(t, w), 1);
+      mbar_init(o_empty(t), 4);
+      mbar_init(sum_full(t), 4);
     }
     mbar_init(drain_bar, 2);
     fence_mbar_init();
@@ -771,14 +782,14 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_async_smem();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 16 && lane == 0) {
     tma_prefetch(&mQ);
     tma_prefetch(&mK);
     tma_prefetch(&mV);
     if constexpr (RP > 0 || DENSE) tma_prefetch(&mU);
     if constexpr (RP > 0) tma_prefetch(&mW);
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -788,21 +799,22 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
 
-  if (warp >= 8) {
-   // Control warpgroup: all four warps shrink their budget at this point.
-   warpgroup_reg_dealloc<kLongControlRegs>();
-   if (warp == 8) {
+  if (warp == 16) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       int it = 0, uc = 0;  // K/V tiles and units loaded so far
       bool ok = true;
       for (int u = first; ok && u < nunits; u += stride, ++uc) {
         const int bh = u / npairs, q0 = (u % npairs) * 2 * kTile;
-        if (uc > 0 && !wait_bounded(q_empty, (uc - 1) & 1, g, 10)) break;
-        mbar_expect_tx(q_full, 2 * (C::QB + C::UB));
+        const int qb = uc % C::QSETS;
+        if (uc >= C::QSETS &&
+            !wait_bounded(q_empty(qb), ((uc / C::QSETS) - 1) & 1, g, 10))
+          break;
+        mbar_expect_tx(q_full(qb), 2 * (C::QB + C::UB));
         for (int t = 0; t < 2; ++t) {
-          tma_load_3d(q_addr(t), &mQ, q_full, 0, q0 + t * kTile, bh);
+          tma_load_3d(q_addr(qb, t), &mQ, q_full(qb), 0, q0 + t * kTile, bh);
           if constexpr (RP > 0)
-            tma_load_3d(u_addr(t), &mU, q_full, 0, q0 + t * kTile, bh % args.bias_heads);
+            tma_load_3d(u_addr(qb, t), &mU, q_full(qb), 0, q0 + t * kTile, bh % args.bias_heads);
         }
         for (int j = 0; j < nkv; ++j, ++it) {
           const int s = it % NS;
@@ -829,24 +841,25 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         }
       }
       // No copy may still be in flight when the CTA exits.
-      if (uc > 0) wait_drain(q_full, (uc - 1) & 1);
-      for (int i = (it > NS ? it - NS : 0); i < it; ++i)
-        wait_drain(kv_full(i % NS), (i / NS) & 1);
+      for (int k = (uc > C::QSETS ? uc - C::QSETS : 0); k < uc; ++k)
+        wait_drain(q_full(k % C::QSETS), (k / C::QSETS) & 1);
+      for (int i = (it > NS ? it - NS : 0); i < it; ++i) wait_drain(kv_full(i % NS), (i / NS) & 1);
     }
-   } else if (warp == 9 || warp == 10) {
-    // MMA issue for query tile t = warp - 9 (one converged warp each).
-    const int t = warp - 9;
+  } else if (warp == 17 || warp == 18) {
+    // ---------------------------- MMA issue for query tile t (whole warp)
+    const int t = warp - 17;
     int it = 0, jt = 0, uc = 0;  // K/V tiles, S tiles of this query tile, units
     bool ok = true;
-    // S_t = Q_t K^T + U'_t W^T for K/V tile `it` into tile t's S columns, once
-    // its warpgroup has loaded the previous scores (s_empty).
+    // S_t = Q_t K^T + U'_t W^T for K/V tile `itj`, once both halves have loaded
+    // the previous scores (s_empty).
+    int qb = 0;  // Q / U' set of the current unit
     auto do_s = [&](int itj, int jtj) -> bool {
       const int s = itj % NS;
       if (!wait_warp(kv_full(s), (itj / NS) & 1, g, 13)) return false;
       if (jtj >= 1 && !wait_warp(s_empty(t), (jtj - 1) & 1, g, 14)) return false;
       tc_fence_after();
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-      issue_scores<D, RP>(tmem + t * 128, q_addr(t), st, u_addr(t), st + 2 * C::QB);
+      issue_scores<D, RP>(tmem + t * 128, q_addr(qb, t), st, u_addr(qb, t), st + 2 * C::QB);
       umma_commit(s_full(t));
       return true;
     };
@@ -865,9 +878,10 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       return true;
     };
     for (int u = first; ok && u < nunits; u += stride, ++uc) {
-      if (!wait_warp(q_full, uc & 1, g, 12)) break;
+      qb = uc % C::QSETS;
+      if (!wait_warp(q_full(qb), (uc / C::QSETS) & 1, g, 12)) break;
       if constexpr (RP > 0) {
-        scale_tile_bf16(u_addr(t), C::UB, args.inv_scale);
+        scale_tile_bf16(u_addr(qb, t), C::UB, args.inv_scale);
         fence_async_smem();
       }
       __syncwarp();
@@ -876,7 +890,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         if (j + 1 < nkv) {
           if (!do_s(it + 1, jt + 1)) { ok = false; break; }
         } else {
-          umma_commit(q_empty);  // the unit's last scores read Q_t / U'_t
+          umma_commit(q_empty(qb));  // the unit's last scores read Q_t / U'_t
         }
         // The previous unit's epilogue must have read O before it is overwritten.
         if (j == 0 && uc > 0 && !wait_warp(o_empty(t), (uc - 1) & 1, g, 18)) { ok = false; break; }
@@ -888,48 +902,45 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0);
     __syncwarp();
-   }
-  } else {
-    warpgroup_reg_alloc<kLongSoftmaxRegs>();
-    const int t = warp >> 2;             // query tile of this warpgroup
+  } else if (warp < 16) {
+    // ---------------------------------------- softmax, query tile t, key half h
+    const int wg = warp >> 2;
+    const int t = wg >> 1, h = wg & 1;
     const int row = threadIdx.x & 127;   // TMEM lane == query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_tm = tmem + lane_base + t * 128;
+    const uint32_t s_tm = tmem + lane_base + t * 128 + 64 * h;      // this half's scores
     const uint32_t o_tm = tmem + lane_base + C::T_O + t * C::OD;
-    const uint32_t p_tm = tmem + lane_base + C::T_P + t * 64;
+    const uint32_t p_tm = tmem + lane_base + C::T_P + t * 64 + 32 * h;  // this half's P
+    // half-row maxima [t][h][row]; key half 1's row sums go to the [t][0] slot
+    // at the end of a unit (half 0 no longer writes it until its epilogue is
+    // done, and half 1 has read half 0's last maximum).
+    auto max_addr = [&](int hh) { return sb + C::OFF_MAX + (t * 2 + hh) * (kTile * 4) + row * 4; };
+    const uint32_t sum_addr = max_addr(0);
     // Scores are accumulator * sl2 in log2 units; the comparator adds its bias
     // to the scaled scores first and then uses a unit factor.
     const float sl2 = DENSE ? 1.0f : args.scale_log2;
-    // The two warpgroups take turns at the exponentials, warp by warp on each
-    // scheduler (warps w and w + 4): warpgroup 0 has the first turn.  While one
-    // runs its exponentials (the MUFU-bound phase) the other loads scores,
-    // takes row maxima and waits for its MMAs, so the phases overlap instead
-    // of both warpgroups contending for the exponential unit at once.
-    const int wq = warp & 3;
-    if (t == 1 && lane == 0) mbar_arrive(exp_turn(0, wq));
-    int jt = 0;  // S tiles of this query tile so far (= K/V tiles of the CTA)
+    int jt = 0, uc = 0;  // S tiles of this query tile so far, units
     bool ok = true;
-    for (int u = first; ok && u < nunits; u += stride) {
+    for (int u = first; ok && u < nunits; u += stride, ++uc) {
       const int bh = u / npairs, q0 = (u % npairs) * 2 * kTile;
-      float m_run = -INFINITY, l = 0.f;
+      float m_run = -INFINITY, l = 0.f;  // l: this half's row sum (d = 64)
       for (int j = 0; j < nkv; ++j, ++jt) {
         if (!wait_warp(s_full(t), jt & 1, g, 16)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sv[128];
-        tmem_ld_cols<128>(s_tm, sv);
+        uint32_t sv[64];
+        tmem_ld_cols<64>(s_tm, sv);
         tc_fence_before();
-        mbar_arrive(s_empty(t));
         if constexpr (DENSE) {
           // s_j = acc_j s log2(e) + bias_j log2(e), the bias row from this K/V
           // tile's stage (its copy is awaited here too; it landed with K / V).
           const int s = jt % NS;
           if (!wait_warp(kv_full(s), (jt / NS) & 1, g, 20)) { ok = false; break; }
-          const uint32_t bt = sb + C::OFF_STAGE + s * C::STAGE + C::OFF_BIAS + t * C::BT;
+          const uint32_t bt = sb + C::OFF_STAGE + s * C::STAGE + C::OFF_BIAS + t * C::BT +
+                              h * (C::BT / 2);
           const float sl = args.scale_log2;
 #pragma unroll
-          for (int c = 0; c < 128; c += 8) {
-            const uint4 bv = ld_shared_v4(bt + (c >> 6) * (C::BT / 2) + row * 128 +
-                                          ((((c & 63) >> 3) ^ (row & 7)) << 4));
+          for (int c = 0; c < 64; c += 8) {
+            const uint4 bv = ld_shared_v4(bt + row * 128 + (((c >> 3) ^ (row & 7)) << 4));
             const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -941,10 +952,23 @@ __global__ void __launch_bounds__(kLongThreads, 1)
             }
           }
         }
-        const int kvalid = N - j * kTile;  // >= 1; >= 128 except on the last tile
-        if (kvalid < kTile) mask_tail<128>(sv, kvalid);
-        const float m_new = fmaxf(m_run, row_max<128>(sv) * sl2);
-        // Lazy rescale: keep the running max unless it grew by more than 2^8.
+        const int kvalid = N - j * kTile - 64 * h;  // keys of this half that exist
+        if (kvalid < 64) mask_tail<64>(sv, kvalid);
+        // Row maximum over both halves: publish this half's, read the other's.
+        // The next scores (and with them the next maxima) wait for s_empty,
+        // which both halves signal only after reading, so one slot suffices.
+        const float mh = row_max<64>(sv) * sl2;
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(max_addr(h)), "f"(mh) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mx_full(t));
+        if (!wait_warp(mx_full(t), jt & 1, g, 21)) { ok = false; break; }
+        float mo;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mo) : "r"(max_addr(h ^ 1)) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty(t));
+        const float m_new = fmax3(m_run, mh, mo);
+        // Lazy rescale: keep the running max unless it grew by more than 2^8
+        // (both halves take the same decision from the same values).
         const bool need = m_new > m_run + 8.0f;
         float alpha = 1.f;
         if (need) {
@@ -952,15 +976,12 @@ __global__ void __launch_bounds__(kLongThreads, 1)
           l *= alpha;
           m_run = m_new;
         }
-        const bool fix_o = __any_sync(0xffffffffu, need && j > 0);
-        // The P buffer of this tile and O: the previous PV must have finished.
+        const bool fix_o = h == 0 && __any_sync(0xffffffffu, need && j > 0);
+        // P_t and O_t: the previous PV must have finished.
         if (jt >= 1 && !wait_warp(pv_done(t), (jt - 1) & 1, g, 17)) { ok = false; break; }
-        if (!wait_warp(exp_turn(t, wq), jt & 1, g, 21)) { ok = false; break; }
         tc_fence_after();
-        if constexpr (C::LCOL) exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
-        else l += exp_row_to_tmem<128, kLongSoftPairs>(sv, sl2, m_run, p_tm);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(exp_turn(t ^ 1, wq));
+        if constexpr (C::LCOL) exp_row_to_tmem<64, kLongSoftPairs>(sv, sl2, m_run, p_tm);
+        else l += exp_row_to_tmem<64, kLongSoftPairs>(sv, sl2, m_run, p_tm);
         if (fix_o) {
           uint32_t ov[D];
           tmem_ld_cols<D>(o_tm, ov);
@@ -977,11 +998,30 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full(t));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(t));
       }
       if (!ok || nkv == 0) break;
+      if constexpr (!C::LCOL) {
+        if (h == 1) {
+          // Key half 1 hands its row sums to half 0, which writes the output.
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(sum_addr), "f"(l) : "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sum_full(t));
+          continue;
+        }
+      } else {
+        if (h == 1) continue;
+      }
       if (!wait_warp(pv_done(t), (jt - 1) & 1, g, 19)) break;
+      if constexpr (!C::LCOL) {
+        if (!wait_warp(sum_full(t), uc & 1, g, 22)) break;
+        float l1;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l1) : "r"(sum_addr) : "memory");
+        l += l1;
+      }
       tc_fence_after();
+      const int q = q0 + t * kTile + row;
       uint32_t ov[D];
       tmem_ld_cols<D>(o_tm, ov);
       if constexpr (C::LCOL) {
@@ -990,8 +1030,8 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         l = __uint_as_float(lv[0]);
       }
       tc_fence_before();
-      mbar_arrive(o_empty(t));
-      const int q = q0 + t * kTile + row;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty(t));
       if (q < N) {
         const size_t r = static_cast<size_t>(bh) * N + q;
         store_o_row<D>(args.o + r * D, ov, 1.0f / l);
@@ -1002,7 +1042,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
