@@ -23,7 +23,8 @@
  * rfb_attn_bwd, rfb_attn_bwd_noalloc); variants with one factor pair per head
  * shared by all windows (rfb_attn_*_shared_bias); shifted-window attention on
  * feature maps (rfb_attn_fwd_image_windows, rfb_attn_bwd_image_windows); a dense-bias
- * comparator (rfb_attn_fwd_dense_bias); diagnostics and test hooks.  Each declaration below
+ * comparator (rfb_attn_fwd_dense_bias); the factoriser's products
+ * (rfb_bias_project); diagnostics and test hooks.  Each declaration below
  * states what differs from these conventions.
  *
  * Conventions for every entry point
@@ -268,6 +269,23 @@ RFB_API int rfb_attn_bwd_image_windows(const void* q, const void* k, const void*
                                        size_t workspace_bytes, int B, int img_h, int img_w,
                                        int heads, int d, int r, int win, int shift, float scale,
                                        void* stream);
+
+/*
+ * The N x N products of the low-rank factoriser of a materialised bias (the
+ * step before the attention path that turns a dense per-head bias into the
+ * factors U, W; "FlashBias: Fast Computation of Attention with Bias",
+ * Abstract: low-rank bias approximation):
+ *     transpose == 0:  out[h] = bias[h] . x[h]
+ *     transpose != 0:  out[h] = bias[h]^T . x[h]
+ *   bias : [H, N, N] fp32 device pointer (row i, column j = bias[h][i][j]).
+ *   x    : [H, N, k] fp32 device pointer, 1 <= k <= 80.
+ *   out  : [H, N, k] fp32 device pointer, written (must not alias bias or x).
+ * Accumulation in fp32; pointers 16-byte aligned.  Asynchronous on stream.
+ * Errors: RFB_ERR_INVALID_ARG (negative sizes, k < 1, NULL pointers),
+ * RFB_ERR_UNSUPPORTED (k > 80), RFB_ERR_ALIGNMENT.  H or N == 0 is a no-op.
+ */
+RFB_API int rfb_bias_project(const float* bias, const float* x, float* out, int H, int N, int k,
+                             int transpose, void* stream);
 
 /* Human-readable text for a status code (static storage). */
 RFB_API const char* rfb_strerror(int status);

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     attn_fwd_dense_bias,
     attn_fwd_image_windows,
     attn_fwd_shared_bias,
+    bias_project,
     bwd_image_windows_workspace_size,
     bwd_shared_bias_workspace_size,
     bwd_workspace_size,
@@ -41,5 +42,5 @@ __all__ = ["attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_noalloc_setup",
            "bwd_image_windows_workspace_size", "attn_bwd_shared_bias", "bwd_shared_bias_workspace_size",
            "rfb_attention_shared_bias", "RFBAttentionSharedBias",
            "rfb_attention_image_windows", "RFBImageWindows", "allreduce_bias_grads",
-           "factorize_bias", "relative_position_bias",
+           "factorize_bias", "relative_position_bias", "bias_project",
            "last_device_error", "selftest_wait_timeout", "debug_set_wait_limit", "load_library", "strerror", "LIB_PATH", "profile_enable", "profile_read"]

@@ -46,6 +46,7 @@ SIGNATURES = {
     "rfb_last_cuda_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
     "rfb_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "rfb_debug_set_wait_limit": (_i, [ctypes.c_uint, _i]),
+    "rfb_bias_project": (_i, [_vp, _vp, _vp] + [_i] * 4 + [_vp]),
     "rfb_selftest_soft_exp2": (_i, [_vp, _vp, _i, _vp]),
     "rfb_profile_enable": (_i, [_i]),
     "rfb_profile_read": (_i, [_fp, ctypes.POINTER(ctypes.c_int)]),
@@ -471,6 +472,30 @@ def attn_bwd_noalloc(q, k, v, u, w, o, lse, dout, scale=None, *, grads=None, str
 def last_device_error() -> int:
     """Synchronise the current device, read and clear the kernels' error word."""
     return int(load_library().rfb_last_device_error())
+
+
+def bias_project(bias, x, transpose=False, *, out=None, stream=None):
+    """out[h] = bias[h] @ x[h] (or bias[h]^T @ x[h]) on the GPU, fp32:
+    bias [H, N, N], x [H, N, k] with k <= 80 (the factoriser's products)."""
+    if bias.dim() != 3 or bias.shape[1] != bias.shape[2]:
+        raise ValueError("bias must be [H, N, N]")
+    H, N, _ = (int(v) for v in bias.shape)
+    if x.dim() != 3 or tuple(x.shape[:2]) != (H, N):
+        raise ValueError(f"x must be [{H}, {N}, k]")
+    k = int(x.shape[2])
+    dev = bias.device
+    for name, t in (("bias", bias), ("x", x)):
+        if t.dtype != torch.float32 or not t.is_cuda or t.device != dev or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
+    o = torch.empty((H, N, k), dtype=torch.float32, device=dev) if out is None else out
+    if (o.dtype != torch.float32 or o.device != dev or tuple(o.shape) != (H, N, k)
+            or not o.is_contiguous()):
+        raise ValueError(f"out must be a contiguous float32 [{H}, {N}, {k}] tensor on {dev}")
+    with _on_device(dev):
+        rc = load_library().rfb_bias_project(_ptr(bias), _ptr(x), _ptr(o), H, N, k,
+                                            1 if transpose else 0, _stream_ptr(stream, dev))
+    _check(rc, "rfb_bias_project")
+    return o
 
 
 def debug_set_wait_limit(limit_us: int = 0, fail_site: int = -1):

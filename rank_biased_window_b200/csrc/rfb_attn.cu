@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "rfb_attn.h"
+#include "bias_project.cuh"
 #include "bwd_kernels.cuh"
 #include "bwd_window.cuh"
 #include "fwd_kernels.cuh"
@@ -1104,6 +1105,25 @@ int rfb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
   // statistics, so what an earlier call left in the array does not matter.
   return rfb_attn_bwd(q, k, v, u, w, o, lse, dout, dq, dk, dv, du, dw, scratch,
                       RFB_NOALLOC_SCRATCH_BYTES, B, H, N, d, r, scale, stream);
+}
+
+int rfb_bias_project(const float* bias, const float* x, float* out, int H, int N, int k,
+                     int transpose, void* stream) {
+  if (H < 0 || N < 0 || k < 1 || k > kProjMaxK) return k > kProjMaxK ? RFB_ERR_UNSUPPORTED
+                                                                    : RFB_ERR_INVALID_ARG;
+  if (H == 0 || N == 0) return RFB_OK;
+  if (!bias || !x || !out) return RFB_ERR_INVALID_ARG;
+  if (!aligned16(bias) || !aligned16(x) || !aligned16(out)) return RFB_ERR_ALIGNMENT;
+  if (static_cast<long long>(N) > 65535LL * kProjRows || H > 65535) return RFB_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (int rc = device_info(&dev)) return rc;
+  const dim3 grid((N + kProjRows - 1) / kProjRows, H);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (transpose)
+    bias_project_kernel<true><<<grid, kProjThreads, 0, st>>>(bias, x, out, N, k);
+  else
+    bias_project_kernel<false><<<grid, kProjThreads, 0, st>>>(bias, x, out, N, k);
+  return launch_status();
 }
 
 int rfb_debug_set_wait_limit(unsigned int limit_us, int fail_site) {

@@ -9,48 +9,60 @@ with randomness", 2011: range finder with power iterations, then an SVD of the
 small projected matrix):
 
     Y = B G  (G Gaussian N x (r + p));  repeat q times: Y = B (B^T Y), orthonormalised
-    Q = orth(Y);  C = Q^T B  ((r + p) x N);  C = X S Z^T  (small SVD)
+    Q = orth(Y);  C^T = B^T Q  (N x (r + p));  C = X S Z^T  (small SVD)
     U = Q X[:, :r] sqrt(S[:r]),  W = Z[:, :r] sqrt(S[:r])
 
-The N x N products are plain library GEMMs and the QR / small SVD library
-routines (torch on the bias's device); this runs once per model, off the
-attention path.
+Every product with the N x N bias runs in the library's kernel
+(rfb_bias_project, fp32); the QR and SVD of the thin N x (r + p) matrices and
+the small products with them are library routines (torch on the bias's
+device).  This runs once per model, off the attention path.
 """
 from __future__ import annotations
 
 import torch
 
 
-def factorize_bias(bias: torch.Tensor, r: int, *, oversample: int = 8, power_iters: int = 2,
-                   seed: int = 0, out_dtype=torch.bfloat16):
-    """bias ``[H, N, N]`` (any float dtype, any device).  Returns ``(U, W,
-    rel_err)``: U, W ``[H, N, r]`` in ``out_dtype`` and the relative Frobenius
-    error ``||B - U W^T|| / ||B||`` per head, measured in fp32 on the rounded
-    factors."""
+def _factorize(bias: torch.Tensor, r: int, project, *, oversample: int = 8, power_iters: int = 2,
+               seed: int = 0, out_dtype=torch.bfloat16):
+    """The algorithm, with project(B, X, transpose) computing B X or B^T X for
+    B [H, N, N] and X [H, N, k] (fp32)."""
     if bias.dim() != 3 or bias.shape[1] != bias.shape[2]:
         raise ValueError("bias must be [H, N, N]")
     H, N, _ = bias.shape
     if not (0 < r <= N):
         raise ValueError("need 0 < r <= N")
     k = min(N, r + oversample)
-    B = bias.float()
+    B = bias.float().contiguous()
     g = torch.Generator(device=B.device)
     g.manual_seed(int(seed))
     G = torch.randn((H, N, k), generator=g, device=B.device, dtype=torch.float32)
-    Y = torch.bmm(B, G)
-    Q, _ = torch.linalg.qr(Y)
+    Q, _ = torch.linalg.qr(project(B, G, False))
     for _ in range(power_iters):
-        Z, _ = torch.linalg.qr(torch.bmm(B.transpose(1, 2), Q))
-        Q, _ = torch.linalg.qr(torch.bmm(B, Z))
-    C = torch.bmm(Q.transpose(1, 2), B)                      # [H, k, N]
-    X, S, Zt = torch.linalg.svd(C, full_matrices=False)     # C = X diag(S) Zt
+        Z, _ = torch.linalg.qr(project(B, Q.contiguous(), True))
+        Q, _ = torch.linalg.qr(project(B, Z.contiguous(), False))
+    Ct = project(B, Q.contiguous(), True)                    # [H, N, k] = (Q^T B)^T
+    X, S, Zt = torch.linalg.svd(Ct.transpose(1, 2), full_matrices=False)   # C = X diag(S) Zt
     root = S[:, :r].clamp_min(0).sqrt()
     U = torch.bmm(Q, X[:, :, :r]) * root[:, None, :]
     W = Zt[:, :r, :].transpose(1, 2) * root[:, None, :]
     U, W = U.to(out_dtype).contiguous(), W.to(out_dtype).contiguous()
+    # reported error of the rounded factors (a library product: diagnostics only)
     R = B - torch.bmm(U.float(), W.float().transpose(1, 2))
     rel = torch.linalg.matrix_norm(R) / torch.linalg.matrix_norm(B).clamp_min(1e-30)
     return U, W, rel
+
+
+def factorize_bias(bias: torch.Tensor, r: int, *, oversample: int = 8, power_iters: int = 2,
+                   seed: int = 0, out_dtype=torch.bfloat16):
+    """bias ``[H, N, N]`` on a CUDA device (any float dtype).  Returns
+    ``(U, W, rel_err)``: U, W ``[H, N, r]`` in ``out_dtype`` and the relative
+    Frobenius error ``||B - U W^T|| / ||B||`` per head, measured in fp32 on the
+    rounded factors.  r + oversample (capped at N) must be at most 80."""
+    from .binding import bias_project
+    if not bias.is_cuda:
+        raise ValueError("factorize_bias runs its products on the GPU: bias must be a CUDA tensor")
+    return _factorize(bias, r, lambda B, X, t: bias_project(B, X, t), oversample=oversample,
+                      power_iters=power_iters, seed=seed, out_dtype=out_dtype)
 
 
 def relative_position_bias(H: int, wh: int, ww: int, *, seed: int = 0, device="cpu"):

@@ -226,3 +226,15 @@ def test_wait_limit_hook_host_checks(rfb_lib):
     assert lib.rfb_debug_set_wait_limit(0, -2) == 1
     assert lib.rfb_debug_set_wait_limit(5, 13) == 0
     assert lib.rfb_debug_set_wait_limit(0, -1) == 0
+
+
+def test_bias_project_host_checks(rfb_lib):
+    """Argument checks of the factoriser's product entry point happen on the
+    host (nothing is launched)."""
+    lib = rfb_lib.load_library()
+    n = None
+    assert lib.rfb_bias_project(n, n, n, 0, 64, 8, 0, n) == 0     # empty
+    assert lib.rfb_bias_project(n, n, n, 2, 64, 0, 0, n) == 1     # k < 1
+    assert lib.rfb_bias_project(n, n, n, 2, 64, 81, 0, n) == 2    # k > 80
+    assert lib.rfb_bias_project(n, n, n, -1, 64, 8, 0, n) == 1    # negative size
+    assert lib.rfb_bias_project(n, n, n, 2, 64, 8, 1, n) == 1     # null pointers

@@ -1,13 +1,24 @@
 """Low-rank factoriser of a materialised bias: the oracle's truncated SVD is
 pinned by the Eckart-Young closed form, exact recovery of rank-r input and a
-diagonal case; the randomised factoriser (torch, any device) is checked
-against the oracle's optimal error."""
+diagonal case; the randomised factoriser's algorithm is checked against the
+oracle's optimal error on the CPU (with torch's product standing in for the
+library's), and on the GPU with the library's product kernel."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from rank_biased_window_b200.factorize import factorize_bias, relative_position_bias
+from rank_biased_window_b200.factorize import _factorize, factorize_bias, relative_position_bias
+
+
+def _torch_project(B, X, transpose):
+    """B X or B^T X with torch: the host-side stand-in for rfb_bias_project,
+    so that the factoriser's algorithm can be checked without a GPU."""
+    return torch.bmm(B.transpose(1, 2) if transpose else B, X)
+
+
+def _factorize_cpu(B, r, **kw):
+    return _factorize(B, r, _torch_project, **kw)
 
 
 def test_oracle_error_is_eckart_young():
@@ -74,7 +85,7 @@ def test_oracle_pins_catch_planted_mistake(name, old, new, monkeypatch):
 @pytest.mark.parametrize("r", [4, 8, 16])
 def test_randomised_factoriser_near_optimal_cpu(r):
     B = relative_position_bias(3, 8, 8, seed=11)
-    U, W, err = factorize_bias(B, r, out_dtype=torch.float32)
+    U, W, err = _factorize_cpu(B, r, out_dtype=torch.float32)
     assert U.shape == (3, 64, r) and W.shape == (3, 64, r)
     _, _, opt = oracle.factorize_bias(B.double().numpy(), r)
     # within 2 % of the best possible rank-r error (power iterations converge fast)
@@ -89,18 +100,50 @@ def test_randomised_factoriser_exact_rank_and_bf16_output():
     g = torch.Generator().manual_seed(3)
     U0, W0 = torch.randn((2, 48, 8), generator=g), torch.randn((2, 48, 8), generator=g)
     B = torch.bmm(U0, W0.transpose(1, 2))
-    U, W, err = factorize_bias(B, 8)                       # bf16 factors
+    U, W, err = _factorize_cpu(B, 8)                       # bf16 factors
     assert U.dtype == torch.bfloat16
     assert err.max().item() < 1e-2                          # bf16 rounding of the factors
-    _, _, err32 = factorize_bias(B, 8, out_dtype=torch.float32)
+    _, _, err32 = _factorize_cpu(B, 8, out_dtype=torch.float32)
     assert err32.max().item() < 1e-5
 
 
 def test_factoriser_argument_checks():
     with pytest.raises(ValueError):
-        factorize_bias(torch.zeros(2, 4, 5), 2)
+        _factorize_cpu(torch.zeros(2, 4, 5), 2)
     with pytest.raises(ValueError):
-        factorize_bias(torch.zeros(2, 4, 4), 0)
+        _factorize_cpu(torch.zeros(2, 4, 4), 0)
+    with pytest.raises(ValueError, match="GPU"):      # no CPU path for the public call
+        factorize_bias(torch.zeros(2, 4, 4), 2)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("shape", [(2, 100, 24), (3, 256, 40), (1, 1000, 80), (2, 64, 1)],
+                         ids=lambda s: "H{}N{}k{}".format(*s))
+def test_bias_project_matches_fp64(rfb_lib, cuda_dev, shape):
+    """rfb_bias_project (both orientations) against an fp64 product on the
+    host, ragged N included."""
+    H, N, k = shape
+    g = torch.Generator().manual_seed(N + k)
+    B = torch.randn((H, N, N), generator=g)
+    X = torch.randn((H, N, k), generator=g)
+    for t in (False, True):
+        got = rfb_lib.bias_project(B.to(cuda_dev), X.to(cuda_dev), t).double().cpu()
+        want = torch.bmm(B.double().transpose(1, 2) if t else B.double(), X.double())
+        rel = ((got - want).norm() / want.norm()).item()
+        assert rel < 1e-6, (t, rel)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("r", [8, 16, 32])
+def test_gpu_factoriser_near_optimal(rfb_lib, cuda_dev, r):
+    """The factoriser with the library's products on a 16 x 16-window bias:
+    within 2 % of the best possible rank-r error (fp32 factors)."""
+    B = relative_position_bias(4, 16, 16, seed=13, device=cuda_dev)
+    U, W, err = factorize_bias(B, r, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert rfb_lib.last_device_error() == 0
+    _, _, opt = oracle.factorize_bias(B.double().cpu().numpy(), r)
+    assert (err.cpu().numpy() <= opt * 1.02 + 1e-5).all(), (err, opt)
 
 
 @pytest.mark.gpu
