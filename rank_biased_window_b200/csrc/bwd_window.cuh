@@ -189,61 +189,62 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int it = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-        const int s = it % NS;
-        if (it >= NS && !wait_bounded(in_empty(s), ((it / NS) + 1) & 1, g, 51)) break;
-        const uint32_t st = sb + s * C::STAGE;
-        mbar_expect_tx(in_full(s), C::STAGE);
-        const int w0 = t * NW;
-        if constexpr (IMG) {
-          // Four 4 x 4 quadrants per window of the rolled map; a missing last
-          // window repeats the previous one (nothing of it is stored).
-#pragma unroll
-          for (int i = 0; i < NW; ++i) {
-            int b, wy, wx, h;
-            window_of(min(w0 + i, args.BH - 1), b, wy, wx, h);
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-              const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
-              const uint32_t off = i * (NP * D * 2) + qd * (16 * D * 2);
-              tma_load_5d(st + C::S_Q + off, &mQ, in_full(s), 0, h, x, y, b);
-              tma_load_5d(st + C::S_K + off, &mK, in_full(s), 0, h, x, y, b);
-              tma_load_5d(st + C::S_V + off, &mV, in_full(s), 0, h, x, y, b);
-              tma_load_5d(st + C::S_DO + off, &mDO, in_full(s), 0, h, x, y, b);
-              tma_load_5d(st + C::S_O + off, &mO, in_full(s), 0, h, x, y, b);
-              if constexpr (RP > 0) {
-                tma_load_4d(st + C::S_U + off, &mU, in_full(s), 0, 4 * (qd & 1), 4 * (qd >> 1), h);
-                tma_load_4d(st + C::S_W + off, &mW, in_full(s), 0, 4 * (qd & 1), 4 * (qd >> 1), h);
-              }
-            }
+    // The whole warp runs the loop: lane 0 waits for the stage and posts the
+    // expected bytes, then the lanes share the tile's copies (with image
+    // windows a tile takes 4 quadrant copies per tensor and window).
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int s = it % NS;
+      if (it >= NS && !wait_warp(in_empty(s), ((it / NS) + 1) & 1, g, 51)) break;
+      const uint32_t st = sb + s * C::STAGE;
+      if (lane == 0) mbar_expect_tx(in_full(s), C::STAGE);
+      __syncwarp();
+      const int w0 = t * NW;
+      if constexpr (IMG) {
+        // Four 4 x 4 quadrants per window of the rolled map; a missing last
+        // window repeats the previous one (nothing of it is stored).  Copy
+        // j = (window i, quadrant qd, tensor c) goes to lane j % 32.
+        constexpr int NT = RP > 0 ? 7 : 5;
+        for (int j = lane; j < NW * 4 * NT; j += 32) {
+          const int i = j / (4 * NT), qd = (j / NT) % 4, c = j % NT;
+          int b, wy, wx, h;
+          window_of(min(w0 + i, args.BH - 1), b, wy, wx, h);
+          const uint32_t off = i * (NP * D * 2) + qd * (16 * D * 2);
+          if (c >= 5) {
+            tma_load_4d(st + (c == 5 ? C::S_U : C::S_W) + off, c == 5 ? &mU : &mW, in_full(s), 0,
+                        4 * (qd & 1), 4 * (qd >> 1), h);
+          } else {
+            const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
+            const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+            const CUtensorMap* mp = c == 0 ? &mQ : c == 1 ? &mK : c == 2 ? &mV : c == 3 ? &mDO : &mO;
+            const uint32_t so = c == 0 ? C::S_Q : c == 1 ? C::S_K : c == 2 ? C::S_V : c == 3 ? C::S_DO : C::S_O;
+            tma_load_5d(st + so + off, mp, in_full(s), 0, h, x, y, b);
           }
-        } else {
-          tma_load_3d(st + C::S_Q, &mQ, in_full(s), 0, 0, w0);
-          tma_load_3d(st + C::S_K, &mK, in_full(s), 0, 0, w0);
-          tma_load_3d(st + C::S_V, &mV, in_full(s), 0, 0, w0);
-          tma_load_3d(st + C::S_DO, &mDO, in_full(s), 0, 0, w0);
-          tma_load_3d(st + C::S_O, &mO, in_full(s), 0, 0, w0);
-          if constexpr (RP > 0) {
-            if (!args.shared) {
-              tma_load_3d(st + C::S_U, &mU, in_full(s), 0, 0, w0);
-              tma_load_3d(st + C::S_W, &mW, in_full(s), 0, 0, w0);
-            } else {
-              // Shared factors: one copy per window (its bias head).
+        }
+      } else if (lane == 0) {
+        tma_load_3d(st + C::S_Q, &mQ, in_full(s), 0, 0, w0);
+        tma_load_3d(st + C::S_K, &mK, in_full(s), 0, 0, w0);
+        tma_load_3d(st + C::S_V, &mV, in_full(s), 0, 0, w0);
+        tma_load_3d(st + C::S_DO, &mDO, in_full(s), 0, 0, w0);
+        tma_load_3d(st + C::S_O, &mO, in_full(s), 0, 0, w0);
+        if constexpr (RP > 0) {
+          if (!args.shared) {
+            tma_load_3d(st + C::S_U, &mU, in_full(s), 0, 0, w0);
+            tma_load_3d(st + C::S_W, &mW, in_full(s), 0, 0, w0);
+          } else {
+            // Shared factors: one copy per window (its bias head).
 #pragma unroll
-              for (int i = 0; i < NW; ++i) {
-                const int z = (w0 + i) % args.bias_heads;
-                tma_load_3d(st + C::S_U + i * (NP * D * 2), &mU, in_full(s), 0, 0, z);
-                tma_load_3d(st + C::S_W + i * (NP * D * 2), &mW, in_full(s), 0, 0, z);
-              }
+            for (int i = 0; i < NW; ++i) {
+              const int z = (w0 + i) % args.bias_heads;
+              tma_load_3d(st + C::S_U + i * (NP * D * 2), &mU, in_full(s), 0, 0, z);
+              tma_load_3d(st + C::S_W + i * (NP * D * 2), &mW, in_full(s), 0, 0, z);
             }
           }
         }
       }
-      for (int j = (it > NS ? it - NS : 0); j < it; ++j) wait_drain(in_full(j % NS), (j / NS) & 1);
     }
+    if (lane == 0)
+      for (int j = (it > NS ? it - NS : 0); j < it; ++j) wait_drain(in_full(j % NS), (j / NS) & 1);
   } else if (warp == 5) {
     // --------------------------------------------------------- MMA issue
     constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
@@ -319,6 +320,25 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
     // this warp's rows of the dS tile double as its output staging: dQ, dK in
     // block 0, dV in block 1 (32 rows x 64 bytes each)
     const uint32_t stg_q = dsb + warp * 4096, stg_k = stg_q + 2048, stg_v = dsb + 16384 + warp * 4096;
+    // lanes issuing this warp's output stores (each waits for its own copies)
+    constexpr int kStoreLanes = IMG ? 6 : 3;
+    // LSE of this thread's query row of tile tt (0 for padding rows); loaded
+    // one tile ahead so that its global-memory latency overlaps a whole tile.
+    auto load_lse = [&](int tt) -> float {
+      const int wn = tt * NW + wl;
+      if (tt >= num_tiles || wn >= args.BH || n >= N) return 0.f;
+      size_t r = static_cast<size_t>(wn) * N + n;
+      if constexpr (IMG) {
+        int b, wy, wx, h;
+        window_of(wn, b, wy, wx, h);
+        const int qq = n >> 4;
+        const int y = (wy * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift) % args.img_h;
+        const int x = (wx * 8 + 4 * (qq & 1) + (n & 3) + args.shift) % args.img_w;
+        r = ((static_cast<size_t>(b) * args.img_h + y) * args.img_w + x) * args.img_heads + h;
+      }
+      return args.lse[r];
+    };
+    float lse_next = load_lse(blockIdx.x);
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int s = it % NS;
@@ -327,18 +347,13 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       const bool valid = win < args.BH && n < N;
       int b = 0, wy = 0, wx = 0, h = 0;
       if constexpr (IMG) window_of(min(win, args.BH - 1), b, wy, wx, h);
+      const float lse_cur = lse_next;
+      lse_next = load_lse(t + gridDim.x);
       // ---- -LSE log2(e) and -D of this query row
       if (!wait_warp(in_full(s), (it / NS) & 1, g, 56)) break;
       float nl2 = 0.f, nd = 0.f;
       if (valid) {
-        size_t r = static_cast<size_t>(win) * N + n;
-        if constexpr (IMG) {
-          const int qq = n >> 4;
-          const int y = (wy * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift) % args.img_h;
-          const int x = (wx * 8 + 4 * (qq & 1) + (n & 3) + args.shift) % args.img_w;
-          r = ((static_cast<size_t>(b) * args.img_h + y) * args.img_w + x) * args.img_heads + h;
-        }
-        nl2 = -args.lse[r] * kLog2e;
+        nl2 = -lse_cur * kLog2e;
         float acc = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -364,7 +379,7 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       if (!wait_warp(vec_full(it & 1), (it >> 1) & 1, g, 58)) break;
       if (it > 0) {
         // this warp's TMA stores of the previous tile read the rows written next
-        if (lane == 0) bulk_wait_read<0>();
+        if (lane < kStoreLanes) bulk_wait_read<0>();
         __syncwarp();
       }
       tc_fence_after();
@@ -450,26 +465,25 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       stage_row32(stg_v, lane, gv, 1.0f);
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) {
+      if (lane < kStoreLanes) {
+        // lane L stores tensor L % 3 (dQ, dK, dV) (with image windows, the
+        // quadrant L / 3 of the warp's two)
         const int r0 = warp * 32;
         const int wwin = t * NW + r0 / NP, n0 = r0 % NP;
+        const int c = lane % 3;
+        const CUtensorMap* mp = c == 0 ? &mDQ : c == 1 ? &mDK : &mDV;
+        const uint32_t src = c == 0 ? stg_q : c == 1 ? stg_k : stg_v;
         if (wwin < args.BH && n0 < N) {
           if constexpr (IMG) {
             int b2, wy2, wx2, h2;
             window_of(wwin, b2, wy2, wx2, h2);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int qd = (n0 >> 4) + k;
-              const int y = (wy2 * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-              const int x = (wx2 * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
-              tma_store_5d(&mDQ, stg_q + k * 1024, 0, h2, x, y, b2);
-              tma_store_5d(&mDK, stg_k + k * 1024, 0, h2, x, y, b2);
-              tma_store_5d(&mDV, stg_v + k * 1024, 0, h2, x, y, b2);
-            }
+            const int k = lane / 3;
+            const int qd = (n0 >> 4) + k;
+            const int y = (wy2 * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
+            const int x = (wx2 * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+            tma_store_5d(mp, src + k * 1024, 0, h2, x, y, b2);
           } else {
-            tma_store_3d(&mDQ, stg_q, 0, n0, wwin);
-            tma_store_3d(&mDK, stg_k, 0, n0, wwin);
-            tma_store_3d(&mDV, stg_v, 0, n0, wwin);
+            tma_store_3d(mp, src, 0, n0, wwin);
           }
         }
         bulk_commit();
@@ -521,7 +535,7 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       }
     }
     // The TMA stores must have finished before the CTA exits.
-    if (lane == 0) bulk_wait_all();
+    if (lane < kStoreLanes) bulk_wait_all();
   }
 
   tc_fence_before();

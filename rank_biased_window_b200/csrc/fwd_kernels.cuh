@@ -347,56 +347,55 @@ __global__ void __launch_bounds__(kWinThreads, 1)
    warpgroup_reg_dealloc<kWinControlRegs>();
    if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      if (resident) {
-        // Every bias head once (head hh % H at slot hh), for the whole kernel.
-        mbar_expect_tx(res_full, C::res_bytes(args.bias_heads));
-        for (int hh = 0; hh < res_heads; ++hh) {
-          const int z = hh % args.bias_heads;
-          if constexpr (IMG) {
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              const uint32_t off = hh * C::HB + qd * (16 * RP * 2);
-              tma_load_4d(res_u + off, &mU, res_full, 0, 4 * (qd & 1), 4 * (qd >> 1), z);
-              tma_load_4d(res_w + off, &mW, res_full, 0, 4 * (qd & 1), 4 * (qd >> 1), z);
-            }
-          } else {
-            tma_load_3d(res_u + hh * C::HB, &mU, res_full, 0, 0, z);
-            tma_load_3d(res_w + hh * C::HB, &mW, res_full, 0, 0, z);
-          }
-        }
-      }
-      const uint32_t stage_tx = resident ? 3 * C::QB : C::STAGE;
-      int it = 0;
-      for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-        const int s = it % NS;
-        if (it >= NS && !wait_bounded(in_empty(s), ((it / NS) + 1) & 1, g, 1)) break;
-        const uint32_t st = sb + s * C::STAGE;
-        mbar_expect_tx(in_full(s), stage_tx);
-        const int w0 = t * C::NW;
+    // The whole warp runs the loop: lane 0 posts the expected bytes and issues
+    // the resident factors' copies; the lanes share a tile's copies (with
+    // image windows 4 quadrant copies per tensor and window).
+    if (resident && lane == 0) {
+      // Every bias head once (head hh % H at slot hh), for the whole kernel.
+      mbar_expect_tx(res_full, C::res_bytes(args.bias_heads));
+      for (int hh = 0; hh < res_heads; ++hh) {
+        const int z = hh % args.bias_heads;
         if constexpr (IMG) {
-          // Each window as four 4 x 4 quadrants of the rolled map, taken from
-          // the unrolled map at (row + shift, column + shift) mod size.  A
-          // missing last window repeats the previous one (not stored).
 #pragma unroll
-          for (int i = 0; i < C::NW; ++i) {
-            int b, wy, wx, h;
-            window_of(min(w0 + i, args.BH - 1), b, wy, wx, h);
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-              const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
-              const uint32_t off = i * (NP * D * 2) + qd * (16 * D * 2);
-              tma_load_5d(st + off, &mQ, in_full(s), 0, h, x, y, b);
-              tma_load_5d(st + C::QB + off, &mK, in_full(s), 0, h, x, y, b);
-              tma_load_5d(st + 2 * C::QB + off, &mV, in_full(s), 0, h, x, y, b);
-            }
+          for (int qd = 0; qd < 4; ++qd) {
+            const uint32_t off = hh * C::HB + qd * (16 * RP * 2);
+            tma_load_4d(res_u + off, &mU, res_full, 0, 4 * (qd & 1), 4 * (qd >> 1), z);
+            tma_load_4d(res_w + off, &mW, res_full, 0, 4 * (qd & 1), 4 * (qd >> 1), z);
           }
         } else {
-          tma_load_3d(st, &mQ, in_full(s), 0, 0, w0);
-          tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
-          tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
+          tma_load_3d(res_u + hh * C::HB, &mU, res_full, 0, 0, z);
+          tma_load_3d(res_w + hh * C::HB, &mW, res_full, 0, 0, z);
         }
+      }
+    }
+    const uint32_t stage_tx = resident ? 3 * C::QB : C::STAGE;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int s = it % NS;
+      if (it >= NS && !wait_warp(in_empty(s), ((it / NS) + 1) & 1, g, 1)) break;
+      const uint32_t st = sb + s * C::STAGE;
+      if (lane == 0) mbar_expect_tx(in_full(s), stage_tx);
+      __syncwarp();
+      const int w0 = t * C::NW;
+      if constexpr (IMG) {
+        // Each window as four 4 x 4 quadrants of the rolled map, taken from
+        // the unrolled map at (row + shift, column + shift) mod size.  A
+        // missing last window repeats the previous one (not stored).  Copy
+        // j = (window i, quadrant qd, tensor c) goes to lane j % 32.
+        for (int jj = lane; jj < C::NW * 4 * 3; jj += 32) {
+          const int i = jj / 12, qd = (jj / 3) % 4, c = jj % 3;
+          int b, wy, wx, h;
+          window_of(min(w0 + i, args.BH - 1), b, wy, wx, h);
+          const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
+          const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+          const uint32_t off = i * (NP * D * 2) + qd * (16 * D * 2);
+          tma_load_5d(st + c * C::QB + off, c == 0 ? &mQ : c == 1 ? &mK : &mV, in_full(s), 0, h, x,
+                      y, b);
+        }
+      } else if (lane == 0) {
+        tma_load_3d(st, &mQ, in_full(s), 0, 0, w0);
+        tma_load_3d(st + C::QB, &mK, in_full(s), 0, 0, w0);
+        tma_load_3d(st + 2 * C::QB, &mV, in_full(s), 0, 0, w0);
         if constexpr (RP > 0 && !IMG) {
           if (resident) {
             // factors already resident
@@ -415,7 +414,9 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           }
         }
       }
-      // Let the last copies land before the CTA can exit.
+    }
+    // Let the last copies land before the CTA can exit.
+    if (lane == 0) {
       if (resident) wait_drain(res_full, 0);
       for (int j = (it > NS ? it - NS : 0); j < it; ++j)
         wait_drain(in_full(j % NS), (j / NS) & 1);
@@ -493,6 +494,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     const uint32_t p_tm = tmem + lane_base + C::T_P + a * 64;
     const int N = args.N;
     const float sl2 = args.scale_log2;
+    constexpr int kStoreLanes = IMG ? 2 : 1;  // lanes issuing the warp's O stores
     if (resident) {
       // U' = U / s for the resident factors, 16 bytes per thread per step.
       if (wait_warp(res_full, 0, g, 10)) {
@@ -572,7 +574,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       // TMA store per warp writes its 32 rows.
       const uint32_t ost = sb + C::OFF_OST + a * C::OB;
       if (it >= 2) {
-        if (lane == 0) bulk_wait_read<0>();
+        if (lane < kStoreLanes) bulk_wait_read<0>();
         __syncwarp();
       }
       {
@@ -587,21 +589,19 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) {
+      if (lane < kStoreLanes) {
         const int r0 = (warp & 3) * 32;           // the warp's first tile row
         const int wwin = t * C::NW + r0 / NP;     // its window
         const int n0 = r0 % NP;                   // its first token in the window
         if (wwin < args.BH && n0 < N) {
           if constexpr (IMG) {
+            // lane k stores quadrant k of the warp's two
             int b, wy, wx, h;
             window_of(wwin, b, wy, wx, h);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int qd = (n0 >> 4) + k;
-              const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-              const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
-              tma_store_5d(&mO, ost + (r0 + 16 * k) * (D * 2), 0, h, x, y, b);
-            }
+            const int qd = (n0 >> 4) + lane;
+            const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
+            const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+            tma_store_5d(&mO, ost + (r0 + 16 * lane) * (D * 2), 0, h, x, y, b);
           } else {
             tma_store_3d(&mO, ost + r0 * (D * 2), 0, n0, wwin);
           }
@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       }
     }
     // The O stores must have finished before the CTA exits.
-    if (lane == 0) bulk_wait_all();
+    if (lane < kStoreLanes) bulk_wait_all();
   }
 
   tc_fence_before();
