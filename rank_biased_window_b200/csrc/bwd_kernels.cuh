@@ -17,20 +17,22 @@
 //   bwd_main : one CTA per (head, 128-key tile); K, W, V stay in shared memory,
 //              dV, dK, dW accumulate in TMEM across all 128-query tiles.  Per
 //              query tile: S^T and dP^T by tcgen05 into TMEM; two compute
-//              warpgroups (64 query columns each) form P^T and dS^T and write
-//              them back into TMEM in place (bf16), dS^T also into swizzled
-//              shared memory; dV, dK, dW (+=) read their A operand from TMEM;
+//              warpgroups (64 query columns each) form P^T and dS^T, write P^T
+//              back into TMEM in place (bf16) and dS^T into swizzled shared
+//              memory; dV (+=) reads its A operand P^T from TMEM, dK and dW
+//              (+=) read dS^T from shared memory, so that the next tile's
+//              dP^T can be issued as soon as the softmax has read dP^T and
+//              its S^T as soon as dV is done (the tensor pipe stays fed);
 //              the partial dQ|dU tile goes to TMEM columns of its own (when
-//              they fit), which the compute warps stage in 128-byte-swizzled
-//              shared memory and add into the fp32 accumulator with TMA bulk
-//              tensor reductions, each warp its own 32 query rows (no barrier
-//              spans a warpgroup).  The reduction of tile i runs after the
-//              softmax of tile i + 1, overlapping tile i + 1's MMAs.  Each
-//              query half (one warpgroup's 64 columns) has barriers of its
-//              own: S^T / dP^T of a half (N = 64 MMAs) and its dV / dK / dW
-//              MMAs are issued as soon as that half is ready, so one half's
-//              MMAs overlap the other half's softmax.  All MMAs are issued by
-//              one converged warp.
+//              they fit), which four reduction warps of their own stage in
+//              128-byte-swizzled shared memory and add into the fp32
+//              accumulator with TMA bulk tensor reductions, each warp its own
+//              32 query rows, while the softmax warps go on with the next
+//              tile.  Each query half (one warpgroup's 64 columns) has
+//              barriers of its own: S^T / dP^T of a half (N = 64 MMAs) and its
+//              dV / dK / dW MMAs are issued as soon as that half is ready, so
+//              one half's MMAs overlap the other half's softmax.  All MMAs are
+//              issued by one converged warp.
 //   bwd_post : dQ = bf16(acc[:, :d]), dU = bf16(acc[:, d:d+r]) (with shared
 //              factors dU and dW are instead summed over the windows by
 //              sum_bias_grads_kernel in bwd_window.cuh).
@@ -47,8 +49,11 @@ struct BwdArgs {
   const __nv_bfloat16* dout;  // [BH, N, D]
   const __nv_bfloat16* u;     // [BH, N, r]   bias factor U
   __nv_bfloat16* uprime;      // [BH, N, r]   U' = bf16(U / s), written by bwd_pre
-  float* dvec;                // [BH, Npad]   -D_i
-  float* lse2;                // [BH, Npad]   -LSE_i * log2(e)
+  // [BH, Npad, 16] bf16 per query row: -LSE_i / s and -D_i, each as three
+  // bf16 parts (columns 0-2 and 3-5; hi + mid + lo carries fp32 precision),
+  // zeros elsewhere.  The score MMAs add them to S^T / s and dP^T through a
+  // constant operand of ones, so the softmax needs no per-query loads.
+  __nv_bfloat16* aug;
   float* acc;                 // [BH, N, D + r] fp32 dQ | dU accumulator
   __nv_bfloat16* dq;          // [BH, N, D]
   __nv_bfloat16* dk;          // [BH, N, D]
@@ -110,6 +115,16 @@ __global__ void __launch_bounds__(256) img_move_kernel(const ImgMoveArgs a) {
   }
 }
 
+// x as the sum of three bf16 values (each returned as the float it rounds to):
+// hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid); the remainder is
+// below 2^-24 |x|, as for fp32.
+__device__ __forceinline__ void split3_bf16(float x, float (&p)[3]) {
+  p[0] = __bfloat162float(__float2bfloat16_rn(x));
+  const float r1 = x - p[0];
+  p[1] = __bfloat162float(__float2bfloat16_rn(r1));
+  p[2] = __bfloat162float(__float2bfloat16_rn(r1 - p[1]));
+}
+
 // ------------------------------------------------------------------ bwd_pre
 // Thread group of G = D/8 lanes per row (16-byte loads); rows grid-strided.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
@@ -121,7 +136,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
        row += static_cast<long>(gridDim.x) * rows_per_block) {
     const int bh = static_cast<int>(row / a.Npad);
     const int i = static_cast<int>(row % a.Npad);
-    float dsum = 0.f, l2 = 0.f;  // stored negated: -D_i and -LSE_i log2(e)
+    float dsum = 0.f, lse = 0.f;
     if (i < a.N) {
       const size_t base = (static_cast<size_t>(bh) * a.N + i) * a.D + sub * 8;
       const uint4 ov = *reinterpret_cast<const uint4*>(a.o + base);
@@ -133,12 +148,23 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
         dsum = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(gw[e] << 16), dsum);
         dsum = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(gw[e] & 0xFFFF0000u), dsum);
       }
-      l2 = a.lse[static_cast<size_t>(bh) * a.N + i] * kLog2e;
+      lse = a.lse[static_cast<size_t>(bh) * a.N + i];
     }
     for (int off = G / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off, G);
     if (sub == 0) {
-      a.dvec[row] = -dsum;
-      a.lse2[row] = -l2;
+      // Padding rows (i >= N) get zeros; their scores are masked anyway.
+      uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (i < a.N) {
+        float c[3], dd[3];
+        split3_bf16(-lse * a.inv_scale, c);
+        split3_bf16(-dsum, dd);
+        w[0] = pack_bf16x2(c[0], c[1]);
+        w[1] = pack_bf16x2(c[2], dd[0]);
+        w[2] = pack_bf16x2(dd[1], dd[2]);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(a.aug + static_cast<size_t>(row) * 16);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
   // Zero the dQ | dU accumulator.
@@ -200,11 +226,15 @@ struct BwdCfg {
   static constexpr int OFF_V = QB;
   static constexpr int OFF_W = 2 * QB;
   static constexpr int KVB = 2 * QB + UQB;
-  // stage: Q, dO, U', -LSE log2(e) [128], -D [128]
-  static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_L2 = 2 * QB + UQB, S_DV = S_L2 + 512;
-  static constexpr int STAGE = 2 * QB + UQB + 1024;
+  // Two constant K-major A tiles [128 x 16] bf16 (32-byte rows and swizzle):
+  // ones in columns 0-2 (they add the -LSE / s parts of the query rows' aug
+  // rows to S^T / s) and in columns 3-5 (the -D parts, to dP^T).
+  static constexpr int OFF_ONES = KVB;
+  static constexpr int ONEB = kTile * 32;
+  // stage: Q, dO, U', the 128 query rows' aug rows (32 bytes each)
+  static constexpr int S_Q = 0, S_DO = QB, S_U = 2 * QB, S_AUG = 2 * QB + UQB;
+  static constexpr int STAGE = 2 * QB + UQB + kTile * 32;
   static constexpr int PB = kTile * kTile * 2;  // one dS tile (bf16)
-  static constexpr int STG = kTile * 32 * 4;    // one 128 x 32 fp32 staging buffer
   static constexpr int NCH = (D + RP + 31) / 32;  // dQ | dU chunks of 32 columns
   // TMEM columns.  When dQ | dU fit in columns of their own, the dQ reduction
   // of tile i is deferred until after the softmax of tile i + 1 (DEFER): the
@@ -215,33 +245,37 @@ struct BwdCfg {
   static constexpr bool DEFER = (256 + 2 * D + RP + NCH * 32) <= 512;
   static constexpr int T_DQ = DEFER ? 256 + 2 * D + RP : 0;
   static constexpr int NDS = DEFER ? 2 : 1;
-  // Staging buffers: with DEFER each warpgroup's first chunk is staged in its
-  // block of the dS buffer, so only warpgroup 0's further chunks need one.
-  static constexpr int NSTG = DEFER ? 1 : 2;
+  // The dQ | dU chunks are staged for their TMA reductions in the two 64-query
+  // blocks (16 KB each) of the tile's dS buffer, free once dQ's MMAs have
+  // read it: chunk c in block c & 1, chunks 2 and 3 once the copies of
+  // chunks 0 and 1 have read theirs.
   // The dynamic shared memory is declared 1024-byte aligned (no slack); 256
   // bytes are kept for the barriers.
-  static constexpr int NS_FIT = (232448 - 256 - KVB - NDS * PB - NSTG * STG) / STAGE;
+  static constexpr int NS_FIT = (232448 - 256 - KVB - 2 * ONEB - NDS * PB) / STAGE;
   static constexpr int NS = NS_FIT > 3 ? 3 : NS_FIT;
-  static constexpr int OFF_STAGE = KVB;
+  static constexpr int OFF_STAGE = KVB + 2 * ONEB;
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_STG = OFF_DS + NDS * PB;
-  static constexpr int OFF_BAR = OFF_STG + NSTG * STG;
+  static constexpr int OFF_BAR = OFF_DS + NDS * PB;
   // kv_full q_full[NS] q_empty[NS] sdp_full[2] ds_full[2] dq_full dq_free drain a_done[2]
-  static constexpr int NBAR = 2 * NS + 10;
+  // ds_free[2][2]
+  static constexpr int NBAR = 2 * NS + 14;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
-  static_assert(NS >= 1, "shared memory budget");
+  static_assert(NS >= 2, "shared memory budget");
+  static_assert(OFF_STAGE % 1024 == 0 && STAGE % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 232448, "shared memory budget exceeded");
   static_assert(T_DW + RP <= 512 && NCH * 32 <= 128, "TMEM budget");
 };
 
-constexpr int kBwdThreads = 320;  // warps 0-7 compute (two warpgroups), 8 TMA, 9 MMA
+// warps 0-7 softmax (two warpgroups), 8 TMA, 9 MMA, 10-13 dQ | dU reduction
+constexpr int kBwdThreads = 448;
 
 template <int D, int RP>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                     const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mU,
                     const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mDO,
-                    const __grid_constant__ CUtensorMap mAcc, const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap mAcc,
+                    const __grid_constant__ CUtensorMap mAug, const BwdArgs args) {
   using C = BwdCfg<D, RP>;
   constexpr int NS = C::NS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -256,14 +290,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto q_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
   // Query half h (columns 64h .. 64h + 63 of a tile, warpgroup h): its S^T and
-  // dP^T are in TMEM, its P^T / dS^T are written, its dV / dK / dW MMAs (which
-  // read P^T / dS^T from TMEM) are done.
+  // dP^T are in TMEM, its P^T / dS^T are written, its dV MMAs (which read P^T
+  // from TMEM) are done.
   auto sdp_full = [&](int h) { return bar0 + 8u * (1 + 2 * NS + h); };
   auto ds_full = [&](int h) { return bar0 + 8u * (3 + 2 * NS + h); };
   const uint32_t dq_full = bar0 + 8u * (5 + 2 * NS);
   const uint32_t dq_free = bar0 + 8u * (6 + 2 * NS);
   const uint32_t drain_bar = bar0 + 8u * (7 + 2 * NS);
   auto a_done = [&](int h) { return bar0 + 8u * (8 + 2 * NS + h); };
+  // Block k (queries 64k .. 64k + 63) of dS buffer b: the reductions staged
+  // in it have been read, so warpgroup k may write the next dS^T there.
+  auto ds_free = [&](int b, int k) { return bar0 + 8u * (10 + 2 * NS + 2 * b + k); };
   auto ds_buf = [&](int i) { return sb + C::OFF_DS + (C::NDS == 2 ? (i & 1) : 0) * C::PB; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -288,9 +325,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(a_done(h), 1);
     }
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 8);        // one arrival per compute warp
+    mbar_init(dq_free, 4);        // one arrival per reduction warp
+    for (int b = 0; b < 2; ++b)
+      for (int k = 0; k < 2; ++k) mbar_init(ds_free(b, k), 4);
     mbar_init(drain_bar, 1);
     fence_mbar_init();
+  }
+  {
+    // The ones tiles: row r of tile t holds bf16 1.0 in columns 3t .. 3t + 2
+    // (first 16-byte chunk of the row, stored at its 32-byte-swizzle place).
+    const uint4 one_l = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+    const uint4 one_d = make_uint4(0u, 0x3F800000u, 0x3F803F80u, 0u);
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int idx = threadIdx.x; idx < 2 * kTile * 2; idx += kBwdThreads) {
+      const int t = idx / (2 * kTile), r = (idx / 2) % kTile, c = idx & 1;
+      uint4* dst = reinterpret_cast<uint4*>(smem + C::OFF_ONES + t * C::ONEB + swz_offset(r, c, 32));
+      *dst = c != 0 ? zero : (t == 0 ? one_l : one_d);
+    }
+    fence_async_smem();
   }
   if (warp == 8 && lane == 0) {
     tma_prefetch(&mQ);
@@ -298,6 +350,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch(&mV);
     tma_prefetch(&mDO);
     tma_prefetch(&mAcc);
+    tma_prefetch(&mAug);
     if constexpr (RP > 0) {
       tma_prefetch(&mU);
       tma_prefetch(&mW);
@@ -320,8 +373,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_load_3d(sb + C::OFF_K, &mK, kv_full, 0, k0, bh);
       tma_load_3d(sb + C::OFF_V, &mV, kv_full, 0, k0, bh);
       if constexpr (RP > 0) tma_load_3d(sb + C::OFF_W, &mW, kv_full, 0, k0, bh % args.bias_heads);
-      const float* l2 = args.lse2 + static_cast<size_t>(bh) * args.Npad;
-      const float* dv = args.dvec + static_cast<size_t>(bh) * args.Npad;
       int i = 0;
       for (; i < nq; ++i) {
         const int s = i % NS;
@@ -332,8 +383,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(st + C::S_DO, &mDO, q_full(s), 0, i * kTile, bh);
         if constexpr (RP > 0)
           tma_load_3d(st + C::S_U, &mU, q_full(s), 0, i * kTile, bh % args.bias_heads);
-        bulk_load(st + C::S_L2, l2 + i * kTile, 512, q_full(s));
-        bulk_load(st + C::S_DV, dv + i * kTile, 512, q_full(s));
+        tma_load_3d(st + C::S_AUG, &mAug, q_full(s), 0, i * kTile, bh);
       }
       wait_drain(kv_full, 0);
       for (int j = (i > NS ? i - NS : 0); j < i; ++j)
@@ -349,31 +399,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
       if (!wait_warp(q_full(s), (i / NS) & 1, g, 33)) return false;
       if (!C::DEFER && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
-      // P^T / dS^T of the previous tile live in these columns: the MMAs reading
-      // them must be done before this tile's S^T / dP^T overwrite them.
-      if (i > 0 && !wait_warp(a_done(h), (i - 1) & 1, g, 41)) return false;
       tc_fence_after();
       const uint32_t tS = tmem + C::T_S + h * 64, tP = tmem + C::T_DP + h * 64;
       const uint32_t q = st + C::S_Q + h * 64 * (D * 2), o = st + C::S_DO + h * 64 * (D * 2);
-      // S^T and dP^T K-steps alternate between the two accumulators.
+      // dP^T first: the softmax has read the previous dP^T of this half (its
+      // dS^T goes to shared memory only), so these columns are free.
+      // The query rows' aug rows: + (-D) through the second ones tile.
+      const uint64_t aug = desc_kmajor(st + C::S_AUG + h * 64 * 32, 32);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        umma_bf16(tS, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2), desc_kmajor(q + kk * 32, D * 2),
-                  idS, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < D / 16; ++kk)
         umma_bf16(tP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2), desc_kmajor(o + kk * 32, D * 2),
                   idS, kk > 0 ? 1u : 0u);
-      }
+      umma_bf16(tP, desc_kmajor(sb + C::OFF_ONES + C::ONEB, 32), aug, idS, 1u);
+      // P^T of the previous tile lives in the S^T columns: the dV MMAs reading
+      // it must be done before S^T is overwritten (dK / dW and the dP^T above
+      // are still queued behind them, so the tensor pipe does not run dry).
+      if (i > 0 && !wait_warp(a_done(h), (i - 1) & 1, g, 41)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_bf16(tS, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2), desc_kmajor(q + kk * 32, D * 2),
+                  idS, kk > 0 ? 1u : 0u);
       const uint32_t u = st + C::S_U + h * 64 * (C::UW * 2);
 #pragma unroll
       for (int kk = 0; kk < RP / 16; ++kk)
         umma_bf16(tS, desc_kmajor(sb + C::OFF_W + kk * 32, C::UW * 2),
                   desc_kmajor(u + kk * 32, C::UW * 2), idS, 1u);
+      umma_bf16(tS, desc_kmajor(sb + C::OFF_ONES, 32), aug, idS, 1u);  // + (-LSE / s)
       umma_commit(sdp_full(h));
       return true;
     };
-    // dV += P^T dO, dK += dS^T Q, dW += dS^T U' over the 64 queries of half h,
-    // with A read from TMEM (P^T over the S^T columns, dS^T over the dP^T
-    // columns, packed bf16 in columns 64h .. 64h + 31), K-steps round-robin.
+    // dV += P^T dO over the 64 queries of half h with A = P^T read from TMEM
+    // (packed bf16 over the S^T columns 64h .. 64h + 31), then a_done(h); then
+    // dK += dS^T Q, dW += dS^T U' with A = dS^T from its swizzled shared-memory
+    // block h (K-major: 128 key rows of 64 queries).
     auto issue_grad_kv = [&](int i, int h) {
       const uint32_t st = sb + C::OFF_STAGE + (i % NS) * C::STAGE;
       constexpr uint32_t idD = idesc_bf16_f32(128, D, false, true);
@@ -381,25 +440,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        const uint32_t aoff = (kk >> 2) * 64 + (kk & 3) * 8;
-        umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + aoff,
+        umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + h * 64 + (kk & 3) * 8,
                      desc_mnmajor(st + C::S_DO + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+      }
+      umma_commit(a_done(h));
+      const uint32_t dsa = ds_buf(i) + h * (kTile * 128);
+#pragma unroll
+      for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        const uint64_t ad = desc_kmajor(dsa + (kk & 3) * 32, 128);
         if constexpr (C::MERGE_KW) {
           // [dK | dW] += dS^T [Q | U']: one B operand, atoms Q (64 cols) and U'
           // (C::S_U - C::S_Q bytes further), N = D + RP.
           constexpr uint32_t idKW = idesc_bf16_f32(128, D + RP, false, true);
-          umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
-                       desc_mnmajor(st + C::S_Q + kk * 16 * 128, 128, C::S_U - C::S_Q), idKW, acc);
+          umma_bf16(tmem + C::T_DK, ad, desc_mnmajor(st + C::S_Q + kk * 16 * 128, 128, C::S_U - C::S_Q),
+                    idKW, acc);
         } else {
-          umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + aoff,
-                       desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+          umma_bf16(tmem + C::T_DK, ad,
+                    desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
           if constexpr (RP > 0)
-            umma_bf16_ts(tmem + C::T_DW, tmem + C::T_DP + aoff,
-                         desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
-                         acc);
+            umma_bf16(tmem + C::T_DW, ad,
+                      desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR, acc);
         }
       }
-      umma_commit(a_done(h));
     };
     // dQ = dS K and dU = dS W (A = the dS^T tile read transposed): one chain
     // over [K | W] (N = D + RP) when W is staged beside K, else interleaved.
@@ -461,14 +524,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     umma_commit(drain_bar);
     wait_drain(drain_bar, 0);
     __syncwarp();
-  } else {
-    // ------------------------------------- compute warps (two warpgroups)
+  } else if (warp < 8) {
+    // ------------------------------------- softmax warps (two warpgroups)
     const int wg = warp >> 2;                  // 0: queries 0-63, 1: queries 64-127
     const int row = threadIdx.x & 127;         // TMEM lane == key row (S^T) == query row (dQ)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const bool key_ok = (k0 + row) < N;
     const uint64_t sl2x2 = f2_pack(args.scale_log2, args.scale_log2);
-    const uint32_t stg = sb + C::OFF_STG + (C::NSTG == 2 ? wg : 0) * C::STG;
     // Shifted-window mask: in the last window row (column) of a shifted map the
     // top and bottom (left and right) 4-token halves are different regions, so
     // key k and query q interact only if ((k ^ q) & mask_bits) == 0 (bit 5 of
@@ -479,30 +541,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int wx = bw % args.mask_nwx, wy = (bw / args.mask_nwx) % args.mask_nwy;
       mask_bits = (wy == args.mask_nwy - 1 ? 32 : 0) | (wx == args.mask_nwx - 1 ? 4 : 0);
     }
-    const int my_chunks = (C::NCH - wg + 1) / 2;   // chunks wg, wg + 2, ...
-    // P^T = 2^(S^T s log2e - LSE log2e), dS^T = P^T o (dP^T - D) for this
-    // warpgroup's 64 query columns of tile i; P^T and dS^T go back into TMEM in
-    // place (packed bf16, columns wg*64 + [0, 32)), dS^T also into shared memory.
+    // P^T = 2^((S^T / s - LSE / s) s log2e), dS^T = P^T o (dP^T - D) for
+    // this warpgroup's 64 query columns of tile i (the MMAs have subtracted
+    // LSE / s and D already); P^T goes back into TMEM in place (packed bf16,
+    // columns wg*64 + [0, 32)), dS^T into shared memory.
     auto softmax = [&](int i) -> bool {
-      const int s = i % NS;
-      const uint32_t st = sb + C::OFF_STAGE + s * C::STAGE;
-      if (!wait_warp(q_full(s), (i / NS) & 1, g, 37)) return false;
       if (!wait_warp(sdp_full(wg), i & 1, g, 38)) return false;
       tc_fence_after();
-      if constexpr (C::DEFER) {
-        // Block wg of this dS buffer staged this warpgroup's first dQ | dU chunk
-        // of tile i - 2; the last reductions issued are reduce_dq(i - 2)'s, so
-        // only its later chunks (from the staging buffer) may still be read.
-        // A warp writes the same 32 rows of the block that it staged and
-        // reduced, so it waits on its own copies only.
-        if (i >= 2) {
-          if (lane == 0) {
-            if (my_chunks >= 2) bulk_wait_read<1>();
-            else bulk_wait_read<0>();
-          }
-          __syncwarp();
-        }
-      }
       const int qvalid = N - i * kTile;
       const uint32_t dsb = ds_buf(i);
 #pragma unroll 1
@@ -522,27 +567,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const uint4 nl = ld_shared_v4(st + C::S_L2 + (c + e) * 4);  // -LSE log2e
-          const uint4 nd = ld_shared_v4(st + C::S_DV + (c + e) * 4);  // -D
+        // S^T / s already holds - LSE / s and dP^T already holds - D.
 #pragma unroll
-          for (int t = 0; t < 4; t += 2) {
-            const uint64_t nl2 = (t == 0) ? (static_cast<uint64_t>(nl.y) << 32 | nl.x)
-                                          : (static_cast<uint64_t>(nl.w) << 32 | nl.z);
-            const uint64_t nd2 = (t == 0) ? (static_cast<uint64_t>(nd.y) << 32 | nd.x)
-                                          : (static_cast<uint64_t>(nd.w) << 32 | nd.z);
-            const uint64_t x2 = static_cast<uint64_t>(xy[e + t + 1]) << 32 | xy[e + t];
-            const uint64_t y2 = static_cast<uint64_t>(xy[32 + e + t + 1]) << 32 | xy[32 + e + t];
-            const float2 arg = f2_unpack(f2_fma(x2, sl2x2, nl2));
-            const float p0 = fast_exp2(arg.x), p1 = fast_exp2(arg.y);
-            const float2 ds = f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(y2, nd2)));
-            pk[(e + t) >> 1] = pack_bf16x2(p0, p1);
-            dk[(e + t) >> 1] = pack_bf16x2(ds.x, ds.y);
-          }
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t x2 = static_cast<uint64_t>(xy[e + 1]) << 32 | xy[e];
+          const uint64_t y2 = static_cast<uint64_t>(xy[32 + e + 1]) << 32 | xy[32 + e];
+          const float2 arg = f2_unpack(f2_mul(x2, sl2x2));
+          const float p0 = fast_exp2(arg.x), p1 = fast_exp2(arg.y);
+          const float2 ds = f2_unpack(f2_mul(f2_pack(p0, p1), y2));
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+          dk[e >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         const int pcol = wg * 64 + (c - wg * 64) / 2;
         tmem_st16_nowait(tmem + lane_base + C::T_S + pcol, pk);
-        tmem_st16_nowait(tmem + lane_base + C::T_DP + pcol, dk);
+        // This dS buffer last staged the reductions of tile i - NDS: they must
+        // have been read before dS^T overwrites them.
+        if (c == wg * 64 && i >= C::NDS &&
+            !wait_warp(ds_free(i % C::NDS, wg), ((i / C::NDS) + 1) & 1, g, 43))
+          return false;
 #pragma unroll
         for (int e = 0; e < 32; e += 8)
           st_shared_v4(dsb + sw128_offset(row, c + e, 128), dk[e / 2], dk[e / 2 + 1],
@@ -555,78 +597,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) mbar_arrive(ds_full(wg));
       return true;
     };
-    // Partial dQ | dU of tile j (TMEM lane = query row): this warpgroup reads its
-    // chunks (wg, wg + 2, ... of 32 columns), frees the TMEM columns, then
-    // stages each chunk in its 128-byte-swizzled buffer; each warp adds its 32
-    // rows into the fp32 accumulator with a TMA bulk tensor reduction of its
-    // own (32 x 32 box) issued by its lane 0, whose bulk groups are the only
-    // ones that warp ever waits for.  Rows entirely past N issue no copy but
-    // still commit a (empty) group, so the wait counts hold.
-    auto reduce_dq = [&](int j) -> bool {
-      if (!wait_warp(dq_full, j & 1, g, 39)) return false;
-      tc_fence_after();
-      constexpr int MY_MAX = (C::NCH + 1) / 2;
-      uint32_t z[MY_MAX][32];
-#pragma unroll
-      for (int m = 0; m < MY_MAX; ++m) {
-        const int ch = wg + 2 * m;
-        if (ch < C::NCH) tmem_ld32(tmem + lane_base + C::T_DQ + ch * 32, z[m]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
-#pragma unroll
-      for (int m = 0; m < MY_MAX; ++m) {
-        const int ch = wg + 2 * m;
-        if (ch >= C::NCH) break;
-        uint32_t buf = stg;
-        if (C::DEFER && m == 0) {
-          // This warpgroup's first chunk goes into its own 64-query block of the
-          // dS buffer of tile j, free now that dQ_j's MMAs have read it (dq_full)
-          // and the reduction staged there earlier was awaited by softmax(j).
-          buf = ds_buf(j) + wg * (kTile * 128);
-        } else {
-          if (lane == 0) {
-            if (C::DEFER) bulk_wait_read<1>();  // only this tile's first chunk may still read
-            else bulk_wait_read_all();
-          }
-          __syncwarp();
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float v4[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int col = ch * 32 + q * 4 + t;
-            v4[t] = __uint_as_float(z[m][q * 4 + t]) * (col < D ? args.scale : 1.0f);
-          }
-          st_shared_v4(buf + row * 128 + ((q ^ (row & 7)) << 4), __float_as_uint(v4[0]),
-                       __float_as_uint(v4[1]), __float_as_uint(v4[2]), __float_as_uint(v4[3]));
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const int wq = (warp & 3) * 32;  // this warp's 32 query rows
-          if (j * kTile + wq < N)
-            tma_reduce_add_3d(&mAcc, buf + wq * 128, ch * 32, j * kTile + wq, bh);
-          bulk_commit();
-        }
-      }
-      return true;
-    };
     bool ok = true;
-    for (int i = 0; ok && i < nq; ++i) {
-      ok = softmax(i);
-      if (!ok) break;
-      if constexpr (C::DEFER) {
-        if (i > 0) ok = reduce_dq(i - 1);
-      } else {
-        ok = reduce_dq(i);
-      }
-    }
-    if (C::DEFER && ok && nq > 0) ok = reduce_dq(nq - 1);
+    for (int i = 0; ok && i < nq; ++i) ok = softmax(i);
+    // The MMA warp's final commit: every dV, dK, dW MMA has completed.
+    if (ok && nq > 0) ok = wait_warp(drain_bar, 0, g, 44);
     if (ok && nq > 0) {
-      // The last dq_full implies all dV, dK, dW MMAs have completed.
+      tc_fence_after();
       const size_t r0 = static_cast<size_t>(bh) * N + k0 + row;
       if (wg == 0) {
         uint32_t gv[D];
@@ -666,6 +642,90 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t gk[D];
         tmem_ld_cols<D>(tmem + lane_base + C::T_DK, gk);
         if (key_ok) store_o_row<D>(args.dk + r0 * D, gk, args.scale);
+      }
+    }
+  } else {
+    // --------------------------------- dQ | dU reduction warps (10 - 13)
+    // Partial dQ | dU of tile j (TMEM lane = query row): each warp takes its 32
+    // query rows of every 32-column chunk, scales the dQ columns by s, stages
+    // the chunk 128-byte swizzled and adds it into the fp32 accumulator with a
+    // TMA bulk tensor reduction (32 x 32 box) issued by its lane 0.  The
+    // chunks are staged in the two 64-query blocks of the tile's dS buffer
+    // (read by dQ's MMAs already, dq_full): with three chunks, chunk 0 in block
+    // 0 and chunks 1, 2 in block 1 (block 0 is released after one copy);
+    // otherwise chunk c in block c & 1.  Warpgroup k overwrites block k NDS
+    // tiles later, once that block's copies have read it (ds_free).  Rows
+    // entirely past N issue no copy.
+    const int rw = warp & 3;                     // TMEM lane quarter
+    const uint32_t lane_base = static_cast<uint32_t>(rw * 32) << 16;
+    const int row = rw * 32 + lane;              // query row within the tile
+    const int wq = rw * 32;
+    for (int j = 0; j < nq; ++j) {
+      if (!wait_warp(dq_full, j & 1, g, 39)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < C::NCH; ++ch) {
+        uint32_t z[32];
+        tmem_ld32(tmem + lane_base + C::T_DQ + ch * 32, z);
+        if (ch == C::NCH - 1) {
+          // dQ | dU of this tile are in registers: the next dQ MMAs may start.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dq_free);
+        }
+        const int blk = C::NCH == 3 ? (ch > 0 ? 1 : 0) : (ch & 1);
+        const uint32_t buf = ds_buf(j) + blk * (kTile * 128);
+        if (ch >= 2) {
+          // The block's previous copy must have read it: with three chunks
+          // that is chunk 1's, the last committed (and then block 0 is free
+          // too), with four chunk ch - 2's, the one before the last.
+          if (lane == 0) {
+            if (C::NCH == 3) bulk_wait_read<0>();
+            else bulk_wait_read<1>();
+          }
+          __syncwarp();
+          if (C::NCH == 3 && lane == 0) mbar_arrive(ds_free(j % C::NDS, 0));
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float v4[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int col = ch * 32 + q * 4 + t;
+            v4[t] = __uint_as_float(z[q * 4 + t]) * (col < D ? args.scale : 1.0f);
+          }
+          st_shared_v4(buf + row * 128 + ((q ^ (row & 7)) << 4), __float_as_uint(v4[0]),
+                       __float_as_uint(v4[1]), __float_as_uint(v4[2]), __float_as_uint(v4[3]));
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (j * kTile + wq < N)
+            tma_reduce_add_3d(&mAcc, buf + wq * 128, ch * 32, j * kTile + wq, bh);
+          bulk_commit();
+        }
+      }
+      // Release each block once the copies out of it have read it.
+      const int b = j % C::NDS;
+      if constexpr (C::NCH == 3) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_free(b, 1));
+      } else if constexpr (C::NCH == 1) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(ds_free(b, 0));
+          mbar_arrive(ds_free(b, 1));
+        }
+      } else {
+        // the last two copies came from blocks 0 and 1, in that order
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_free(b, 0));
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_free(b, 1));
       }
     }
     if (lane == 0) bulk_wait_all();  // reductions complete before the CTA exits

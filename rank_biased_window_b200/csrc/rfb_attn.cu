@@ -346,7 +346,7 @@ struct LaunchTimer {
 };
 
 struct Maps {
-  CUtensorMap q, k, v, u, w, g, acc, o;
+  CUtensorMap q, k, v, u, w, g, acc, o, aug;
 };
 
 // ---------------------------------------------------------------- forward
@@ -447,24 +447,22 @@ int dispatch_fwd_rp(int d, int rp, const Maps& m, const FwdArgs& a, int sms, cud
 
 // --------------------------------------------------------------- backward
 struct WsLayout {
-  size_t dvec, lse2, acc, uprime, dw_part, total;
+  size_t aug, acc, uprime, dw_part, total;
   int npad;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Backward workspace: -D and -LSE log2(e) [BH, Npad] fp32, the fp32 dQ | dU
-// accumulator [BH, N, d + r], U' [bias heads, N, r] bf16 and, for shared
-// factors, the fp32 per-window dW [BH, N, r].
+// Backward workspace: the query rows' -LSE / s and -D as bf16 parts
+// [BH, Npad, 16], the fp32 dQ | dU accumulator [BH, N, d + r], U' [bias heads,
+// N, r] bf16 and, for shared factors, the fp32 per-window dW [BH, N, r].
 WsLayout ws_layout(int B, int H, int N, int d, int r, bool shared = false) {
   WsLayout L{};
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t bias_heads = shared ? static_cast<size_t>(H) : bh;
   L.npad = (N + kTile - 1) / kTile * kTile;
-  const size_t vec = align256(bh * L.npad * sizeof(float));
-  L.dvec = 0;
-  L.lse2 = vec;
-  L.acc = 2 * vec;
+  L.aug = 0;
+  L.acc = align256(bh * L.npad * 16 * 2);
   L.uprime = L.acc + align256(bh * N * static_cast<size_t>(d + r) * sizeof(float));
   L.dw_part = L.uprime + align256(bias_heads * N * static_cast<size_t>(r) * 2);
   L.total = L.dw_part + (shared ? align256(bh * N * static_cast<size_t>(r) * sizeof(float)) : 0);
@@ -479,7 +477,7 @@ int launch_bwd_main(const Maps& m, const BwdArgs& a, cudaStream_t st) {
   const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
   LaunchTimer timer(kIdBwdMain, st);
   bwd_main_kernel<D, RP><<<grid, kBwdThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, m.g, m.acc,
-                                                              a);
+                                                              m.aug, a);
   return launch_status();
 }
 
@@ -696,6 +694,7 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
     rc = encode_3d(&m.u, ws + L.uprime, r, N, bias_heads, d == 64 ? 64 : rp, kTile, 1);
   if (!rc && r > 0) rc = encode_3d(&m.w, w, r, N, bias_heads, d == 64 ? 64 : rp, kTile, 1);
   if (!rc) rc = encode_acc_3d(&m.acc, ws + L.acc, d + r, N, BH);
+  if (!rc) rc = encode_3d(&m.aug, ws + L.aug, 16, L.npad, BH, 16, kTile, 1);
   if (rc) return rc;
   BwdArgs a;
   a.o = static_cast<const __nv_bfloat16*>(o);
@@ -703,8 +702,7 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
   a.dout = static_cast<const __nv_bfloat16*>(dout);
   a.u = static_cast<const __nv_bfloat16*>(u);
   a.uprime = reinterpret_cast<__nv_bfloat16*>(ws + L.uprime);
-  a.dvec = reinterpret_cast<float*>(ws + L.dvec);
-  a.lse2 = reinterpret_cast<float*>(ws + L.lse2);
+  a.aug = reinterpret_cast<__nv_bfloat16*>(ws + L.aug);
   a.acc = reinterpret_cast<float*>(ws + L.acc);
   a.dq = static_cast<__nv_bfloat16*>(dq);
   a.dk = static_cast<__nv_bfloat16*>(dk);
