@@ -123,10 +123,11 @@ RFB_API int rfb_attn_bwd(const void* q, const void* k, const void* v, const void
  *
  * Limit: the call accepts exactly the problems for which
  * rfb_attn_bwd_workspace_size(B, H, N, d, r) <= RFB_NOALLOC_SCRATCH_BYTES,
- * i.e. about 8 + 4 (d + r) + 2 r bytes per row of B*H*N (two fp32 row
- * statistics, with N rounded up to a multiple of 128; the fp32 dQ | dU
- * accumulator; bf16 U / s): up to about 73,000 rows for d = 64, r = 32 and
- * 182,000 rows for d = 32, r = 8.  Larger problems are rejected with
+ * i.e. about 32 + 4 (d + r) + 2 r bytes per row of B*H*N (the row
+ * statistics -LSE / s and -D as six bf16 parts in a 32-byte row, with N
+ * rounded up to a multiple of 128; the fp32 dQ | dU accumulator; bf16 U / s):
+ * up to about 69,900 rows for d = 64, r = 32 and 161,000 rows for d = 32,
+ * r = 8.  Larger problems are rejected with
  * RFB_ERR_WORKSPACE before anything is enqueued.  The call makes no
  * cudaMalloc, cudaFree or other allocating call.
  *

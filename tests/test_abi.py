@@ -68,10 +68,10 @@ def test_workspace_size(rfb_lib):
     assert lib.rfb_attn_bwd_workspace_size(1, 1, 64, 48, 8) == 0
     B, H, N, d, r = 2, 8, 16384, 64, 32
     ws = lib.rfb_attn_bwd_workspace_size(B, H, N, d, r)
-    # two fp32 row vectors (padded to 128 rows), the fp32 dQ|dU accumulator and
-    # the bf16 copy U' = U / s
-    need = B * H * N * (d + r) * 4 + 2 * B * H * N * 4 + B * H * N * r * 2
-    assert need <= ws < need + 2 * B * H * 128 * 4 + 1024
+    # the 32-byte rows of bf16 parts of -LSE / s and -D (padded to 128 rows),
+    # the fp32 dQ|dU accumulator and the bf16 copy U' = U / s
+    need = B * H * N * (d + r) * 4 + B * H * N * 32 + B * H * N * r * 2
+    assert need <= ws < need + B * H * 128 * 32 + 1024
 
 
 def test_shared_bias_host_checks_and_workspace(rfb_lib):
@@ -87,9 +87,9 @@ def test_shared_bias_host_checks_and_workspace(rfb_lib):
     ws = lib.rfb_attn_bwd_shared_bias_workspace_size(B, H, N, d, r)
     # as the per-window layout, but U' holds one copy per head (H, not B H)
     # and the per-window fp32 dW is added
-    need = (B * H * N * (d + r) * 4 + 2 * B * H * N * 4 + H * N * r * 2
+    need = (B * H * N * (d + r) * 4 + B * H * N * 32 + H * N * r * 2
             + B * H * N * r * 4)
-    assert need <= ws < need + 2 * B * H * 128 * 4 + 2048
+    assert need <= ws < need + B * H * 128 * 32 + 2048
 
 
 def test_dense_bias_host_checks(rfb_lib):
