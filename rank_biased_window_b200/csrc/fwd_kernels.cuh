@@ -885,7 +885,9 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         fence_async_smem();
       }
       __syncwarp();
-      ok = do_s(it, jt);
+      // Query tile 1 starts each unit once tile 0's first P is written, so
+      // that the two tiles' exponentials alternate instead of coinciding.
+      ok = (t == 0 || wait_warp(p_full(0), jt & 1, g, 15)) && do_s(it, jt);
       for (int j = 0; ok && j < nkv; ++j) {
         if (j + 1 < nkv) {
           if (!do_s(it + 1, jt + 1)) { ok = false; break; }
