@@ -523,55 +523,18 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       for (int c = 0; c < 64; c += 16) tmem_st16_nowait(p_tm + c, zero);
       tmem_st_wait();
     }
-    int it = a;
-    for (int t = blockIdx.x + a * gridDim.x; t < num_tiles; t += 2 * gridDim.x, it += 2) {
-      if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) break;
-      tc_fence_after();
-      uint32_t sv[NP];
-      tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty(a));
-      if (N < NP) mask_tail<NP>(sv, N);
-      if constexpr (IMG) {
-        // Shifted-window mask: in the last window row (column) of the rolled
-        // map the two quadrant rows (columns) come from opposite edges of the
-        // unrolled map; keys of another region are excluded.
-        if (args.shift > 0) {
-          int b, wy, wx, h;
-          window_of(min(t * C::NW + wl, args.BH - 1), b, wy, wx, h);
-          const int qq = n >> 4;
-          const bool split_y = wy == nwy - 1, split_x = wx == nwx - 1;
-#pragma unroll
-          for (int kq = 0; kq < 4; ++kq) {
-            const bool ok_key = (!split_y || (kq >> 1) == (qq >> 1)) &&
-                                (!split_x || (kq & 1) == (qq & 1));
-            if (!ok_key) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) sv[kq * 16 + e] = 0xFF800000u;
-            }
-          }
-        }
-      }
-      const float m = row_max<NP>(sv) * sl2;
-      // P_a was last read by PV(it - 2), complete since this warpgroup saw
-      // o_full for that tile.
-      const float l = exp_row_to_tmem<NP>(sv, sl2, m, p_tm + wl * (NP / 2));
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(a));
-      // Epilogue of this tile once its PV has landed.
-      if (!wait_warp(o_full(a), (it >> 1) & 1, g, 6)) break;
+    // Epilogue of tile t (iteration it of the CTA), whose PV has landed
+    // (o_full awaited): O_a is read (acc_empty frees it for the next PV), the
+    // O rows go into this warpgroup's staging tile (the TMA store that read
+    // the warp's rows two tiles ago must have finished reading them), one TMA
+    // store per warp writes its 32 rows, and LSE is written directly.
+    auto epilogue = [&](int t, int it, float m, float l) {
       tc_fence_after();
       uint32_t ov[D];
       tmem_ld_cols<D>(tmem + lane_base + C::T_O + a * D, ov);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(a));
-      // O rows into this warpgroup's staging tile (the TMA store that read the
-      // warp's rows two tiles ago must have finished reading them), then one
-      // TMA store per warp writes its 32 rows.
       const uint32_t ost = sb + C::OFF_OST + a * C::OB;
       if (it >= 2) {
         if (lane < kStoreLanes) bulk_wait_read<0>();
@@ -622,7 +585,60 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         }
         args.lse[r] = (m + __log2f(l)) * kLn2;
       }
+    };
+    // Each tile's epilogue runs after the next tile's exponentials (of this
+    // warpgroup), so the tile's PV overlaps them instead of being waited for.
+    bool ok = true, pending = false;
+    int pt = 0, pit = 0;       // the tile whose epilogue is pending
+    float pm = 0.f, pl = 1.f;  // its row maximum and row sum
+    int it = a;
+    for (int t = blockIdx.x + a * gridDim.x; t < num_tiles; t += 2 * gridDim.x, it += 2) {
+      if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[NP];
+      tmem_ld_cols<NP>(tmem + lane_base + a * 128 + wl * NP, sv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty(a));
+      if (N < NP) mask_tail<NP>(sv, N);
+      if constexpr (IMG) {
+        // Shifted-window mask: in the last window row (column) of the rolled
+        // map the two quadrant rows (columns) come from opposite edges of the
+        // unrolled map; keys of another region are excluded.
+        if (args.shift > 0) {
+          int b, wy, wx, h;
+          window_of(min(t * C::NW + wl, args.BH - 1), b, wy, wx, h);
+          const int qq = n >> 4;
+          const bool split_y = wy == nwy - 1, split_x = wx == nwx - 1;
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            const bool ok_key = (!split_y || (kq >> 1) == (qq >> 1)) &&
+                                (!split_x || (kq & 1) == (qq & 1));
+            if (!ok_key) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sv[kq * 16 + e] = 0xFF800000u;
+            }
+          }
+        }
+      }
+      const float m = row_max<NP>(sv) * sl2;
+      // P_a and O_a: the pending tile's PV must have read P_a and written O_a.
+      if (pending && !wait_warp(o_full(a), (pit >> 1) & 1, g, 6)) { ok = false; break; }
+      tc_fence_after();
+      const float l = exp_row_to_tmem<NP>(sv, sl2, m, p_tm + wl * (NP / 2));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full(a));
+      // The pending tile's O is read now, so this tile's PV may start.
+      if (pending) epilogue(pt, pit, pm, pl);
+      pending = true;
+      pt = t;
+      pit = it;
+      pm = m;
+      pl = l;
     }
+    if (ok && pending && wait_warp(o_full(a), (pit >> 1) & 1, g, 6)) epilogue(pt, pit, pm, pl);
     // The O stores must have finished before the CTA exits.
     if (lane < kStoreLanes) bulk_wait_all();
   }
