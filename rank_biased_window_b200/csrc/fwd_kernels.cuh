@@ -864,12 +864,23 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   } else if (warp == 17 || warp == 18) {
     // ---------------------------- MMA issue for query tile t (whole warp)
     const int t = warp - 17;
-    int it = 0, jt = 0, uc = 0;  // K/V tiles, S tiles of this query tile, units
+    int it = 0, jt = 0;  // K/V tiles, S tiles of this query tile
     bool ok = true;
-    // S_t = Q_t K^T + U'_t W^T for K/V tile `itj`, once both halves have loaded
-    // the previous scores (s_empty).
-    int qb = 0;  // Q / U' set of the current unit
-    auto do_s = [&](int itj, int jtj) -> bool {
+    // Q_t / U'_t of this CTA's unit number ucn: loaded, and U' = U / s scaled
+    // in place by this warp.
+    auto prep_unit = [&](int ucn) -> bool {
+      const int b = ucn % C::QSETS;
+      if (!wait_warp(q_full(b), (ucn / C::QSETS) & 1, g, 12)) return false;
+      if constexpr (RP > 0) {
+        scale_tile_bf16(u_addr(b, t), C::UB, args.inv_scale);
+        fence_async_smem();
+      }
+      __syncwarp();
+      return true;
+    };
+    // S_t = Q_t K^T + U'_t W^T for K/V tile `itj` with Q / U' set qb, once
+    // both halves have loaded the previous scores (s_empty).
+    auto do_s = [&](int itj, int jtj, int qb) -> bool {
       const int s = itj % NS;
       if (!wait_warp(kv_full(s), (itj / NS) & 1, g, 13)) return false;
       if (jtj >= 1 && !wait_warp(s_empty(t), (jtj - 1) & 1, g, 14)) return false;
@@ -893,28 +904,61 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       umma_commit(kv_empty(s));
       return true;
     };
-    for (int u = first; ok && u < nunits; u += stride, ++uc) {
-      qb = uc % C::QSETS;
-      if (!wait_warp(q_full(qb), (uc / C::QSETS) & 1, g, 12)) break;
-      if constexpr (RP > 0) {
-        scale_tile_bf16(u_addr(qb, t), C::UB, args.inv_scale);
-        fence_async_smem();
-      }
-      __syncwarp();
-      // Query tile 1 starts each unit once tile 0's first P is written, so
-      // that the two tiles' exponentials alternate instead of coinciding.
-      ok = (t == 0 || wait_warp(p_full(0), jt & 1, g, 15)) && do_s(it, jt);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv) {
-          if (!do_s(it + 1, jt + 1)) { ok = false; break; }
-        } else {
-          umma_commit(q_empty(qb));  // the unit's last scores read Q_t / U'_t
+    if constexpr (C::QSETS == 2) {
+      // One sequence over this CTA's tiles (unit uc, key tile j): the next
+      // tile's scores are issued as soon as the softmax has loaded the
+      // current ones, across unit boundaries too -- the next unit's Q / U'
+      // are in the other set, its U' scaled halfway through this unit -- so a
+      // unit's first scores are ready when its softmax starts.
+      const int nu = first < nunits ? (nunits - first + stride - 1) / stride : 0;
+      if (nu > 0 && nkv > 0) {
+        // Query tile 1 starts once tile 0's first P is written, so that the
+        // two tiles' exponentials start offset.
+        ok = prep_unit(0) && (t == 0 || wait_warp(p_full(0), 0, g, 15)) && do_s(0, 0, 0);
+        int prepared = 1;  // units whose Q / U' are ready
+        for (int uc = 0, j = 0; ok;) {
+          const bool last_j = j + 1 == nkv;
+          const bool has_next = !last_j || uc + 1 < nu;
+          if (uc + 1 < nu && prepared == uc + 1 && j == nkv / 2) {
+            if (!(ok = prep_unit(uc + 1))) break;
+            ++prepared;
+          }
+          if (has_next && !(ok = do_s(it + 1, jt + 1, (last_j ? uc + 1 : uc) % 2))) break;
+          if (last_j) umma_commit(q_empty(uc % 2));  // the unit's scores are all issued
+          // The previous unit's epilogue must have read O before it is overwritten.
+          if (j == 0 && uc > 0 && !(ok = wait_warp(o_empty(t), (uc - 1) & 1, g, 18))) break;
+          if (!(ok = do_pv(it, jt, j == 0))) break;
+          ++it;
+          ++jt;
+          if (!has_next) break;
+          if (last_j) {
+            ++uc;
+            j = 0;
+          } else {
+            ++j;
+          }
         }
-        // The previous unit's epilogue must have read O before it is overwritten.
-        if (j == 0 && uc > 0 && !wait_warp(o_empty(t), (uc - 1) & 1, g, 18)) { ok = false; break; }
-        if (!do_pv(it, jt, j == 0)) { ok = false; break; }
-        ++it;
-        ++jt;
+      }
+    } else {
+      int uc = 0;
+      for (int u = first; ok && u < nunits; u += stride, ++uc) {
+        const int qb = uc % C::QSETS;
+        if (!prep_unit(uc)) break;
+        // Query tile 1 starts each unit once tile 0's first P is written, so
+        // that the two tiles' exponentials start offset.
+        ok = (t == 0 || wait_warp(p_full(0), jt & 1, g, 15)) && do_s(it, jt, qb);
+        for (int j = 0; ok && j < nkv; ++j) {
+          if (j + 1 < nkv) {
+            if (!do_s(it + 1, jt + 1, qb)) { ok = false; break; }
+          } else {
+            umma_commit(q_empty(qb));  // the unit's last scores read Q_t / U'_t
+          }
+          // The previous unit's epilogue must have read O before it is overwritten.
+          if (j == 0 && uc > 0 && !wait_warp(o_empty(t), (uc - 1) & 1, g, 18)) { ok = false; break; }
+          if (!do_pv(it, jt, j == 0)) { ok = false; break; }
+          ++it;
+          ++jt;
+        }
       }
     }
     umma_commit(drain_bar);
