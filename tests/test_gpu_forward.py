@@ -45,6 +45,11 @@ CASES = [
     (1, 1, 1000, 64, 0),
     (1, 1, 1024, 32, 16),
     (1, 1, 777, 64, 64),
+    # d = 32 with several units (head, query-tile pair) per CTA: the next
+    # unit's first scores are issued before the current unit ends
+    (8, 50, 300, 32, 16),  # 3 key tiles, ragged
+    (4, 100, 200, 32, 8),  # 2 key tiles: the next unit prepared at the last tile
+    (2, 100, 257, 32, 0),  # a last query pair of one row
 ]
 
 
