@@ -908,9 +908,14 @@ __global__ void __launch_bounds__(kLongThreads, 1)
       // One sequence over this CTA's tiles (unit uc, key tile j): the next
       // tile's scores are issued as soon as the softmax has loaded the
       // current ones, across unit boundaries too -- the next unit's Q / U'
-      // are in the other set, its U' scaled halfway through this unit -- so a
-      // unit's first scores are ready when its softmax starts.
+      // are in the other set -- so a unit's first scores are ready when its
+      // softmax starts.  The next unit's Q / U' are awaited (and U' scaled)
+      // at key tile prep_j: the producer loads them after the current unit's
+      // last K / V tile, whose stage the PV of tile nkv - 1 - NS releases, so
+      // prep_j must come after that PV is issued (j >= nkv - NS), else the two
+      // warps would wait for each other.
       const int nu = first < nunits ? (nunits - first + stride - 1) / stride : 0;
+      const int prep_j = nkv / 2 > nkv - NS ? nkv / 2 : nkv - NS;
       if (nu > 0 && nkv > 0) {
         // Query tile 1 starts once tile 0's first P is written, so that the
         // two tiles' exponentials start offset.
@@ -919,7 +924,7 @@ __global__ void __launch_bounds__(kLongThreads, 1)
         for (int uc = 0, j = 0; ok;) {
           const bool last_j = j + 1 == nkv;
           const bool has_next = !last_j || uc + 1 < nu;
-          if (uc + 1 < nu && prepared == uc + 1 && j == nkv / 2) {
+          if (uc + 1 < nu && prepared == uc + 1 && j == prep_j) {
             if (!(ok = prep_unit(uc + 1))) break;
             ++prepared;
           }

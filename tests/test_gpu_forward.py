@@ -50,6 +50,7 @@ CASES = [
     (8, 50, 300, 32, 16),  # 3 key tiles, ragged
     (4, 100, 200, 32, 8),  # 2 key tiles: the next unit prepared at the last tile
     (2, 100, 257, 32, 0),  # a last query pair of one row
+    (1, 40, 1664, 32, 8),  # 13 key tiles per unit (more than twice the K / V stages)
 ]
 
 
