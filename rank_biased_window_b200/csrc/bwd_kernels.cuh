@@ -236,11 +236,11 @@ struct BwdCfg {
   static constexpr int STAGE = 2 * QB + UQB + kTile * 32;
   static constexpr int PB = kTile * kTile * 2;  // one dS tile (bf16)
   static constexpr int NCH = (D + RP + 31) / 32;  // dQ | dU chunks of 32 columns
-  // TMEM columns.  When dQ | dU fit in columns of their own, the dQ reduction
-  // of tile i is deferred until after the softmax of tile i + 1 (DEFER): the
-  // next tile's S^T / dP^T MMAs are issued before tile i's dQ | dU MMAs, so
-  // the dS tile in shared memory is double buffered.  Otherwise dQ | dU reuse
-  // the S^T columns and each tile runs its phases in order.
+  // TMEM columns.  When dQ | dU fit in columns of their own (DEFER), the next
+  // tile's S^T / dP^T MMAs are issued before tile i's dQ | dU MMAs and the
+  // reduction of tile i overlaps the next tile's softmax, so the dS tile in
+  // shared memory is double buffered.  Otherwise dQ | dU reuse the S^T
+  // columns and each tile runs its phases in order.
   static constexpr int T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D, T_DW = 256 + 2 * D;
   static constexpr bool DEFER = (256 + 2 * D + RP + NCH * 32) <= 512;
   static constexpr int T_DQ = DEFER ? 256 + 2 * D + RP : 0;

@@ -12,7 +12,8 @@
 // One persistent CTA per SM walks through tiles:
 //   warp 4      TMA producer: Q, K, V, dO, O and the factors U, W of a tile
 //               (U, W staged 32 columns wide, zero padded, so that [Q | U'] and
-//               [K | W] are single MMA operands), a ring of input stages;
+//               [K | W] are single MMA operands), a ring of input stages; the
+//               tile's copies are spread over the warp's lanes;
 //   warp 5      MMA issue: S^T/s = K Q^T + W U'^T and dP^T = V dO^T into TMEM,
 //               then dV = P^T dO, [dK | dW] = dS^T [Q | U'] (A operands read
 //               from TMEM) and [dQ | dU] = dS [K | W] (A = the dS^T tile in

@@ -16,15 +16,18 @@
 //     128/NP whole windows (NP = 64 or 128 rows per window).  One S tile per
 //     tile, single-pass softmax, block-diagonal P (off-window blocks stay 0).
 //     Warps 0-3 and 4-7 softmax + epilogue of even and odd tiles (thread = row
-//     = TMEM lane), warp 8 TMA producer, warp 9 score MMAs, warp 10 PV MMAs,
+//     = TMEM lane; a tile's epilogue runs after the warpgroup's next
+//     exponentials, O leaves by TMA stores), warp 8 TMA producer (a tile's
+//     copies spread over its lanes), warp 9 score MMAs, warp 10 PV MMAs,
 //     warp 11 U' scaling; P goes back into TMEM (packed bf16) for the PV MMA.
 //   * fwd_long_kernel    (N > 128): persistent CTAs over units (head, two
 //     128-query tiles); each unit loops over 128-key tiles with an online
-//     softmax (lazy rescale of O in TMEM).  Warpgroups 0 / 1 softmax of query
-//     tile 0 / 1 (running out of phase), warp 8 TMA, warps 9 / 10 MMA issue
-//     for tile 0 / 1; P goes back into TMEM as packed bf16 and the PV MMA
-//     reads it from there.  The softmax warpgroups take registers from the
-//     control warpgroup (setmaxnreg).  With d = 32 the row sums of P come
+//     softmax (lazy rescale of O in TMEM).  Warps 0-15 are four softmax
+//     warpgroups, one per (query tile, 64-key half), exchanging half-row
+//     maxima through shared memory; warp 16 TMA; warps 17 / 18 MMA issue for
+//     query tile 0 / 1 (with d = 32 the next unit's first scores are issued
+//     before the current unit ends); P goes back into TMEM as packed bf16
+//     and the PV MMA reads it from there.  With d = 32 the row sums of P come
 //     out of the PV MMA (a block of ones beside V), not from the softmax.
 // Operands are staged by TMA with the swizzle that matches their row width.
 #pragma once
