@@ -392,6 +392,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------ MMA issue (whole warp)
     constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+    // Operand descriptors are built once (resident operands) or once per tile
+    // (stage operands) and stepped through the K-steps with constant adds.
+    const uint64_t dK = desc_kmajor(sb + C::OFF_K, D * 2);
+    const uint64_t dV = desc_kmajor(sb + C::OFF_V, D * 2);
+    const uint64_t dW = desc_kmajor(sb + C::OFF_W, C::UW * 2);
+    const uint64_t dOnesL = desc_kmajor(sb + C::OFF_ONES, 32);
+    const uint64_t dOnesD = desc_kmajor(sb + C::OFF_ONES + C::ONEB, 32);
+    // [K | W] as the MN-major B operand of dQ | dU (W beside K for d = 64).
+    const uint64_t dKWmn = C::MERGE_KW ? desc_mnmajor(sb + C::OFF_K, 128, C::OFF_W - C::OFF_K)
+                                       : desc_mnmajor(sb + C::OFF_K, D * 2, 128 * D * 2);
+    const uint64_t dWmn = desc_mnmajor(sb + C::OFF_W, RP > 0 ? RP * 2 : 32, 128 * (RP > 0 ? RP : 16) * 2);
     // Query half h of tile i:  S^T / s = K Q_h^T + W U'_h^T  and  dP^T = V dO_h^T
     // into TMEM columns 64h .. 64h + 63 of the S^T / dP^T accumulators.
     auto issue_sdp = [&](int i, int h) -> bool {
@@ -401,16 +412,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!C::DEFER && i > 0 && !wait_warp(dq_free, (i - 1) & 1, g, 34)) return false;
       tc_fence_after();
       const uint32_t tS = tmem + C::T_S + h * 64, tP = tmem + C::T_DP + h * 64;
-      const uint32_t q = st + C::S_Q + h * 64 * (D * 2), o = st + C::S_DO + h * 64 * (D * 2);
+      const uint64_t dQ = desc_kmajor(st + C::S_Q + h * 64 * (D * 2), D * 2);
+      const uint64_t dO = desc_kmajor(st + C::S_DO + h * 64 * (D * 2), D * 2);
+      const uint64_t dU = desc_kmajor(st + C::S_U + h * 64 * (C::UW * 2), C::UW * 2);
       // dP^T first: the softmax has read the previous dP^T of this half (its
       // dS^T goes to shared memory only), so these columns are free.
       // The query rows' aug rows: + (-D) through the second ones tile.
       const uint64_t aug = desc_kmajor(st + C::S_AUG + h * 64 * 32, 32);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_bf16(tP, desc_kmajor(sb + C::OFF_V + kk * 32, D * 2), desc_kmajor(o + kk * 32, D * 2),
-                  idS, kk > 0 ? 1u : 0u);
-      umma_bf16(tP, desc_kmajor(sb + C::OFF_ONES + C::ONEB, 32), aug, idS, 1u);
+        umma_bf16(tP, desc_add(dV, kk * 32), desc_add(dO, kk * 32), idS, kk > 0 ? 1u : 0u);
+      umma_bf16(tP, dOnesD, aug, idS, 1u);
       // P^T of the previous tile lives in the S^T columns: the dV MMAs reading
       // it must be done before S^T is overwritten (dK / dW and the dP^T above
       // are still queued behind them, so the tensor pipe does not run dry).
@@ -418,14 +430,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_bf16(tS, desc_kmajor(sb + C::OFF_K + kk * 32, D * 2), desc_kmajor(q + kk * 32, D * 2),
-                  idS, kk > 0 ? 1u : 0u);
-      const uint32_t u = st + C::S_U + h * 64 * (C::UW * 2);
+        umma_bf16(tS, desc_add(dK, kk * 32), desc_add(dQ, kk * 32), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
       for (int kk = 0; kk < RP / 16; ++kk)
-        umma_bf16(tS, desc_kmajor(sb + C::OFF_W + kk * 32, C::UW * 2),
-                  desc_kmajor(u + kk * 32, C::UW * 2), idS, 1u);
-      umma_bf16(tS, desc_kmajor(sb + C::OFF_ONES, 32), aug, idS, 1u);  // + (-LSE / s)
+        umma_bf16(tS, desc_add(dW, kk * 32), desc_add(dU, kk * 32), idS, 1u);
+      umma_bf16(tS, dOnesL, aug, idS, 1u);  // + (-LSE / s)
       umma_commit(sdp_full(h));
       return true;
     };
@@ -437,54 +446,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t st = sb + C::OFF_STAGE + (i % NS) * C::STAGE;
       constexpr uint32_t idD = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, false, true);
+      const uint64_t dOmn = desc_mnmajor(st + C::S_DO, D * 2, 128 * D * 2);
 #pragma unroll
       for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
         umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + h * 64 + (kk & 3) * 8,
-                     desc_mnmajor(st + C::S_DO + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+                     desc_add(dOmn, kk * 16 * (D * 2)), idD, acc);
       }
       umma_commit(a_done(h));
-      const uint32_t dsa = ds_buf(i) + h * (kTile * 128);
+      const uint64_t dsa = desc_kmajor(ds_buf(i) + h * (kTile * 128), 128);
+      // [Q | U'] as the MN-major B operand (U' beside Q for d = 64)
+      const uint64_t dQUmn = C::MERGE_KW ? desc_mnmajor(st + C::S_Q, 128, C::S_U - C::S_Q)
+                                         : desc_mnmajor(st + C::S_Q, D * 2, 128 * D * 2);
+      const uint64_t dUmn = desc_mnmajor(st + C::S_U, RP > 0 ? RP * 2 : 32, 128 * (RP > 0 ? RP : 16) * 2);
 #pragma unroll
       for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        const uint64_t ad = desc_kmajor(dsa + (kk & 3) * 32, 128);
+        const uint64_t ad = desc_add(dsa, (kk & 3) * 32);
         if constexpr (C::MERGE_KW) {
           // [dK | dW] += dS^T [Q | U']: one B operand, atoms Q (64 cols) and U'
           // (C::S_U - C::S_Q bytes further), N = D + RP.
           constexpr uint32_t idKW = idesc_bf16_f32(128, D + RP, false, true);
-          umma_bf16(tmem + C::T_DK, ad, desc_mnmajor(st + C::S_Q + kk * 16 * 128, 128, C::S_U - C::S_Q),
-                    idKW, acc);
+          umma_bf16(tmem + C::T_DK, ad, desc_add(dQUmn, kk * 16 * 128), idKW, acc);
         } else {
-          umma_bf16(tmem + C::T_DK, ad,
-                    desc_mnmajor(st + C::S_Q + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD, acc);
+          umma_bf16(tmem + C::T_DK, ad, desc_add(dQUmn, kk * 16 * (D * 2)), idD, acc);
           if constexpr (RP > 0)
-            umma_bf16(tmem + C::T_DW, ad,
-                      desc_mnmajor(st + C::S_U + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR, acc);
+            umma_bf16(tmem + C::T_DW, ad, desc_add(dUmn, kk * 16 * (RP * 2)), idR, acc);
         }
       }
     };
     // dQ = dS K and dU = dS W (A = the dS^T tile read transposed): one chain
     // over [K | W] (N = D + RP) when W is staged beside K, else interleaved.
     auto issue_grad_q = [&](int i) {
-      const uint32_t dsb = ds_buf(i);
+      const uint64_t dsm = desc_mnmajor(ds_buf(i), 128, 128 * 128);
       constexpr uint32_t idD = idesc_bf16_f32(128, D, true, true);
       constexpr uint32_t idR = idesc_bf16_f32(128, RP > 0 ? RP : 16, true, true);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ad = desc_mnmajor(dsb + kk * 16 * 128, 128, 128 * 128);
+        const uint64_t ad = desc_add(dsm, kk * 16 * 128);
         if constexpr (C::MERGE_KW) {
           constexpr uint32_t idQU = idesc_bf16_f32(128, D + RP, true, true);
-          umma_bf16(tmem + C::T_DQ, ad,
-                    desc_mnmajor(sb + C::OFF_K + kk * 16 * 128, 128, C::OFF_W - C::OFF_K), idQU,
-                    kk > 0 ? 1u : 0u);
+          umma_bf16(tmem + C::T_DQ, ad, desc_add(dKWmn, kk * 16 * 128), idQU, kk > 0 ? 1u : 0u);
         } else {
-          umma_bf16(tmem + C::T_DQ, ad,
-                    desc_mnmajor(sb + C::OFF_K + kk * 16 * (D * 2), D * 2, 128 * D * 2), idD,
-                    kk > 0 ? 1u : 0u);
+          umma_bf16(tmem + C::T_DQ, ad, desc_add(dKWmn, kk * 16 * (D * 2)), idD, kk > 0 ? 1u : 0u);
           if constexpr (RP > 0)
-            umma_bf16(tmem + C::T_DQ + D, ad,
-                      desc_mnmajor(sb + C::OFF_W + kk * 16 * (RP * 2), RP * 2, 128 * RP * 2), idR,
+            umma_bf16(tmem + C::T_DQ + D, ad, desc_add(dWmn, kk * 16 * (RP * 2)), idR,
                       kk > 0 ? 1u : 0u);
         }
       }

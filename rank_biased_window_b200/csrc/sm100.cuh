@@ -299,6 +299,14 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, int row_bytes,
                    swizzle_code(row_bytes));
 }
 
+// The descriptor of the operand `bytes` (a multiple of 16) further on in
+// shared memory: one add to the address field, which cannot carry (shared
+// memory ends below 256 KB).  Lets a kernel build each operand's descriptor
+// once and step through its K-steps with constant adds.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (bytes >> 4);
+}
+
 // kind::f16 instruction descriptor: D fp32, A and B bf16, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {
