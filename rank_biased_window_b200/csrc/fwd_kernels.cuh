@@ -181,13 +181,16 @@ template <int D, int RP>
 __device__ __forceinline__ void issue_scores(uint32_t s_tmem, uint32_t q, uint32_t k, uint32_t u,
                                              uint32_t w) {
   constexpr uint32_t id = idesc_bf16_f32(128, 128, false, false);
+  const uint64_t dq = desc_kmajor(q, D * 2), dk = desc_kmajor(k, D * 2);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk)
-    umma_bf16(s_tmem, desc_kmajor(q + kk * 32, D * 2), desc_kmajor(k + kk * 32, D * 2), id,
-              kk > 0 ? 1u : 0u);
+    umma_bf16(s_tmem, desc_add(dq, kk * 32), desc_add(dk, kk * 32), id, kk > 0 ? 1u : 0u);
+  if constexpr (RP > 0) {
+    const uint64_t du = desc_kmajor(u, RP * 2), dw = desc_kmajor(w, RP * 2);
 #pragma unroll
-  for (int kk = 0; kk < RP / 16; ++kk)
-    umma_bf16(s_tmem, desc_kmajor(u + kk * 32, RP * 2), desc_kmajor(w + kk * 32, RP * 2), id, 1u);
+    for (int kk = 0; kk < RP / 16; ++kk)
+      umma_bf16(s_tmem, desc_add(du, kk * 32), desc_add(dw, kk * 32), id, 1u);
+  }
 }
 
 // Issue O(tmem) (+)= P . V for a 128-key tile with P read from TMEM (packed
@@ -196,10 +199,11 @@ template <int D>
 __device__ __forceinline__ void issue_pv_ts(uint32_t o_tmem, uint32_t p_tmem, uint32_t v,
                                             bool accumulate) {
   constexpr uint32_t id = idesc_bf16_f32(128, D, false, true);
+  const uint64_t dv = desc_mnmajor(v, D * 2, 128 * D * 2);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_mnmajor(v + kk * 16 * (D * 2), D * 2, 128 * D * 2),
-                 id, (accumulate || kk > 0) ? 1u : 0u);
+    umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_add(dv, kk * 16 * (D * 2)), id,
+                 (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // O'(tmem) (+)= P . [V | 1] (N = D + 16): the second MN block of B is a
@@ -209,10 +213,11 @@ template <int D>
 __device__ __forceinline__ void issue_pv_ts_ones(uint32_t o_tmem, uint32_t p_tmem, uint32_t v,
                                                  uint32_t ones_off, bool accumulate) {
   constexpr uint32_t id = idesc_bf16_f32(128, D + 16, false, true);
+  const uint64_t dv = desc_mnmajor(v, D * 2, ones_off);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_mnmajor(v + kk * 16 * (D * 2), D * 2, ones_off),
-                 id, (accumulate || kk > 0) ? 1u : 0u);
+    umma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_add(dv, kk * 16 * (D * 2)), id,
+                 (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // ============================================================ window regime
