@@ -261,34 +261,42 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       // columns that these MMAs overwrite.
       if (it > 0 && !wait_warp(grad_full, (it - 1) & 1, g, 53)) break;
       tc_fence_after();
+      // Each operand's descriptor once, stepped through the K-steps by adds.
+      const uint64_t dK = desc_kmajor(st + C::S_K, 64), dQ = desc_kmajor(st + C::S_Q, 64);
+      const uint64_t dV = desc_kmajor(st + C::S_V, 64), dO = desc_kmajor(st + C::S_DO, 64);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        umma_bf16(tmem + C::T_S, desc_kmajor(st + C::S_K + kk * 32, 64),
-                  desc_kmajor(st + C::S_Q + kk * 32, 64), idS, kk > 0 ? 1u : 0u);
-        umma_bf16(tmem + C::T_DP, desc_kmajor(st + C::S_V + kk * 32, 64),
-                  desc_kmajor(st + C::S_DO + kk * 32, 64), idS, kk > 0 ? 1u : 0u);
+        umma_bf16(tmem + C::T_S, desc_add(dK, kk * 32), desc_add(dQ, kk * 32), idS,
+                  kk > 0 ? 1u : 0u);
+        umma_bf16(tmem + C::T_DP, desc_add(dV, kk * 32), desc_add(dO, kk * 32), idS,
+                  kk > 0 ? 1u : 0u);
       }
+      if constexpr (RP > 0) {
+        const uint64_t dW = desc_kmajor(st + C::S_W, 64), dU = desc_kmajor(st + C::S_U, 64);
 #pragma unroll
-      for (int kk = 0; kk < RP / 16; ++kk)
-        umma_bf16(tmem + C::T_S, desc_kmajor(st + C::S_W + kk * 32, 64),
-                  desc_kmajor(st + C::S_U + kk * 32, 64), idS, 1u);
+        for (int kk = 0; kk < RP / 16; ++kk)
+          umma_bf16(tmem + C::T_S, desc_add(dW, kk * 32), desc_add(dU, kk * 32), idS, 1u);
+      }
       umma_commit(sdp_full);
       if (!wait_warp(ds_full, it & 1, g, 54)) break;
       // The previous tile's gradients have been read out of TMEM.
       if (it > 0 && !wait_warp(grad_free, (it - 1) & 1, g, 55)) break;
       tc_fence_after();
+      const uint64_t dOmn = desc_mnmajor(st + C::S_DO, 64, C::TB);
+      const uint64_t dQUmn = desc_mnmajor(st + C::S_Q, 64, C::S_U - C::S_Q);
+      const uint64_t dSmn = desc_mnmajor(dsb, 128, 128 * 128);
+      const uint64_t dKWmn = desc_mnmajor(st + C::S_K, 64, C::S_W - C::S_K);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t acc = kk > 0 ? 1u : 0u;
         // dV = P^T dO
-        umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8,
-                     desc_mnmajor(st + C::S_DO + kk * 16 * 64, 64, C::TB), idV, acc);
+        umma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, desc_add(dOmn, kk * 16 * 64), idV, acc);
         // [dK | dW] = dS^T [Q | U']
-        umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + kk * 8,
-                     desc_mnmajor(st + C::S_Q + kk * 16 * 64, 64, C::S_U - C::S_Q), idKW, acc);
+        umma_bf16_ts(tmem + C::T_DK, tmem + C::T_DP + kk * 8, desc_add(dQUmn, kk * 16 * 64), idKW,
+                     acc);
         // [dQ | dU] = dS [K | W]
-        umma_bf16(tmem + C::T_DQ, desc_mnmajor(dsb + kk * 16 * 128, 128, 128 * 128),
-                  desc_mnmajor(st + C::S_K + kk * 16 * 64, 64, C::S_W - C::S_K), idQU, acc);
+        umma_bf16(tmem + C::T_DQ, desc_add(dSmn, kk * 16 * 128), desc_add(dKWmn, kk * 16 * 64), idQU,
+                  acc);
       }
       umma_commit(grad_full);
       umma_commit(in_empty(s));
