@@ -15,6 +15,8 @@
 #pragma once
 #include <cstdint>
 
+#include "sm100.cuh"
+
 namespace rfb {
 
 constexpr int kProjRows = 128;    // output rows per CTA
@@ -33,6 +35,7 @@ __global__ void __launch_bounds__(kProjThreads) bias_project_kernel(const float*
                                                                    int k) {
   __shared__ float Bs[kProjRows][kProjChunk + 1];
   __shared__ float Xs[kProjChunk][kProjMaxK];
+  grid_dep_wait();
   const int h = blockIdx.y;
   const int r0 = blockIdx.x * kProjRows;
   const float* Bh = B + static_cast<size_t>(h) * N * N;

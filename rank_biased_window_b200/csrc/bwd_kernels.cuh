@@ -92,6 +92,7 @@ struct ImgMoveArgs {
 };
 
 __global__ void __launch_bounds__(256) img_move_kernel(const ImgMoveArgs a) {
+  grid_dep_wait();
   const int G = a.d / 8;  // 16-byte pieces per token row
   const long long total = static_cast<long long>(a.BH) * 64 * G;
   const int nwx = a.img_w / 8, nwy = a.img_h / 8;
@@ -128,6 +129,7 @@ __device__ __forceinline__ void split3_bf16(float x, float (&p)[3]) {
 // ------------------------------------------------------------------ bwd_pre
 // Thread group of G = D/8 lanes per row (16-byte loads); rows grid-strided.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
+  grid_dep_wait();
   const int G = a.D / 8;
   const int rows_per_block = 256 / G;
   const int sub = threadIdx.x % G;
@@ -190,6 +192,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs a) {
 
 // ----------------------------------------------------------------- bwd_post
 __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdArgs a) {
+  grid_dep_wait();
   const int DA = a.D + a.r;
   const int groups = DA / 8;
   const long total = static_cast<long>(a.BH) * a.N * groups;
@@ -365,6 +368,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
+  grid_dep_wait();
+  grid_dep_launch_next();
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer

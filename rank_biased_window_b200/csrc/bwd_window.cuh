@@ -187,6 +187,8 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
+  grid_dep_wait();
+  grid_dep_launch_next();
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -565,6 +567,7 @@ __global__ void __launch_bounds__(256) sum_bias_grads_kernel(const float* du_src
                                                            __nv_bfloat16* du, __nv_bfloat16* dw,
                                                            int B, int H, int N, int r) {
   __shared__ float4 part[256];
+  grid_dep_wait();
   const int hrow = blockIdx.x;            // h * N + n
   const int nv = r / 2;                   // float4 columns: r / 4 of dU, then r / 4 of dW
   const int G = blockDim.x / nv;          // window groups

@@ -349,6 +349,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
+  grid_dep_wait();
+  grid_dep_launch_next();
 
   if (warp >= 8) {
    // Control warpgroup: all four warps shrink their budget at this point.
@@ -822,6 +824,8 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
+  grid_dep_wait();
+  grid_dep_launch_next();
 
   if (warp == 16) {
     // ------------------------------------------------------------ producer

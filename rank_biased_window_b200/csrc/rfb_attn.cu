@@ -291,6 +291,26 @@ int check_shape(int B, int H, int N, int d, int r, float scale, bool* empty) {
   return RFB_OK;
 }
 
+// Launches a kernel with programmatic stream serialisation: it may start while
+// the grid before it in the stream finishes (every kernel launched this way
+// waits for that grid itself before touching global memory, grid_dep_wait()).
+// A launch error is left for launch_status() to read.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RFB_OK : cuda_fail(e, kSiteLaunch);
@@ -371,8 +391,8 @@ int launch_window(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
     }
   }
   LaunchTimer timer(kIdFwd, st);
-  fwd_window_kernel<D, RP, NP><<<grid, kWinThreads, smem, st>>>(m.q, m.k, m.v, m.u, m.w, m.o,
-                                                                 args);
+  launch_pdl(fwd_window_kernel<D, RP, NP>, grid, kWinThreads, smem, st,
+      m.q, m.k, m.v, m.u, m.w, m.o, args);
   return launch_status();
 }
 
@@ -385,7 +405,7 @@ int launch_long(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   const long long units = static_cast<long long>((a.N + 2 * kTile - 1) / (2 * kTile)) * a.BH;
   const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
   LaunchTimer timer(kIdFwd, st);
-  fwd_long_kernel<D, RP><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  launch_pdl(fwd_long_kernel<D, RP>, grid, kLongThreads, C::SMEM, st, m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
 }
 
@@ -402,7 +422,7 @@ int launch_window_img(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st)
   const int tiles = (a.BH + C::NW - 1) / C::NW;
   const int grid = tiles < sms ? tiles : sms;
   LaunchTimer timer(kIdFwd, st);
-  fwd_window_kernel<D, RP, 64, true><<<grid, kWinThreads, static_cast<int>(need), st>>>(
+  launch_pdl(fwd_window_kernel<D, RP, 64, true>, grid, kWinThreads, static_cast<int>(need), st,
       m.q, m.k, m.v, m.u, m.w, m.o, a);
   return launch_status();
 }
@@ -425,7 +445,8 @@ int launch_long_dense(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st)
   const long long units = static_cast<long long>((a.N + 2 * kTile - 1) / (2 * kTile)) * a.BH;
   const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
   LaunchTimer timer(kIdFwd, st);
-  fwd_long_kernel<D, 0, true><<<grid, kLongThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, a);
+  launch_pdl(fwd_long_kernel<D, 0, true>, grid, kLongThreads, C::SMEM, st,
+      m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
 }
 
@@ -476,8 +497,8 @@ int launch_bwd_main(const Maps& m, const BwdArgs& a, cudaStream_t st) {
   if (int rc = ensure_smem(bwd_main_kernel<D, RP>, C::SMEM, done)) return rc;
   const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
   LaunchTimer timer(kIdBwdMain, st);
-  bwd_main_kernel<D, RP><<<grid, kBwdThreads, C::SMEM, st>>>(m.q, m.k, m.v, m.u, m.w, m.g, m.acc,
-                                                              m.aug, a);
+  launch_pdl(bwd_main_kernel<D, RP>, grid, kBwdThreads, C::SMEM, st,
+      m.q, m.k, m.v, m.u, m.w, m.g, m.acc, m.aug, a);
   return launch_status();
 }
 
@@ -503,7 +524,7 @@ int launch_bwd_window(const WinBwdMaps& m, const BwdWinArgs& a, int sms, cudaStr
   const int tiles = (a.BH + C::NW - 1) / C::NW;
   const int grid = tiles < sms ? tiles : sms;
   LaunchTimer timer(kIdBwdMain, st);
-  bwd_window_kernel<RP, NP, IMG><<<grid, kBwdWinThreads, C::SMEM, st>>>(
+  launch_pdl(bwd_window_kernel<RP, NP, IMG>, grid, kBwdWinThreads, C::SMEM, st,
       m.q, m.k, m.v, m.g, m.o, m.u, m.w, m.dq, m.dk, m.dv, a);
   return launch_status();
 }
@@ -675,8 +696,8 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
     if ((rc = dispatch_bwd_window(rp, N, false, wm, a, dev.sms, st))) return rc;
     if (shared && r > 0) {
       LaunchTimer timer(kIdBwdPost, st);
-      sum_bias_grads_kernel<<<H * N, 256, 0, st>>>(a.du_part, r, a.dw_part, r, a.du, a.dw, B, H,
-                                                   N, r);
+      launch_pdl(sum_bias_grads_kernel, H * N, 256, 0, st,
+          a.du_part, r, a.dw_part, r, a.du, a.dw, B, H, N, r);
     }
     return launch_status();
   }
@@ -731,19 +752,19 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* u, co
   const long long rows = static_cast<long long>(BH) * L.npad;
   {
     LaunchTimer timer(kIdBwdPre, st);
-    bwd_pre_kernel<<<grid_for(rows, 256 / (d / 8), dev.sms), 256, 0, st>>>(a);
+    launch_pdl(bwd_pre_kernel, grid_for(rows, 256 / (d / 8), dev.sms), 256, 0, st, a);
   }
   if ((rc = launch_status())) return rc;
   if ((rc = dispatch_bwd_main(d, rp, m, a, st))) return rc;
   const long long groups = static_cast<long long>(BH) * N * ((d + r) / 8);
   {
     LaunchTimer timer(kIdBwdPost, st);
-    bwd_post_kernel<<<grid_for(groups, 256, dev.sms), 256, 0, st>>>(a);
+    launch_pdl(bwd_post_kernel, grid_for(groups, 256, dev.sms), 256, 0, st, a);
     if (shared && r > 0) {
       if ((rc = launch_status())) return rc;
       // dU from the accumulator's dU columns, dW from the per-window fp32 rows
-      sum_bias_grads_kernel<<<H * N, 256, 0, st>>>(a.acc + d, d + r, a.dw_part, r, a.du, a.dw, B,
-                                                   H, N, r);
+      launch_pdl(sum_bias_grads_kernel, H * N, 256, 0, st,
+          a.acc + d, d + r, a.dw_part, r, a.du, a.dw, B, H, N, r);
     }
   }
   return launch_status();
@@ -1030,8 +1051,8 @@ int rfb_attn_bwd_image_windows(const void* q, const void* k, const void* v, cons
     if ((rc = dispatch_bwd_window(rp, 64, true, wm, a, dev.sms, st))) return rc;
     if (r > 0) {
       LaunchTimer timer(kIdBwdPost, st);
-      sum_bias_grads_kernel<<<heads * 64, 256, 0, st>>>(a.du_part, r, a.dw_part, r, a.du, a.dw,
-                                                        nwin, heads, 64, r);
+      launch_pdl(sum_bias_grads_kernel, heads * 64, 256, 0, st,
+          a.du_part, r, a.dw_part, r, a.du, a.dw, nwin, heads, 64, r);
     }
     return launch_status();
   }
@@ -1056,7 +1077,7 @@ int rfb_attn_bwd_image_windows(const void* q, const void* k, const void* v, cons
   g.d = d;
   g.shift = shift;
   g.to_windows = 1;
-  img_move_kernel<<<grid_for(pieces, 256, dev.sms), 256, 0, st>>>(g);
+  launch_pdl(img_move_kernel, grid_for(pieces, 256, dev.sms), 256, 0, st, g);
   if (int rc = launch_status()) return rc;
   // 2. the shared-factor backward on the windows, with the shifted-window mask.
   const int mask[4] = {shift, img_w / 8, img_h / 8, heads};
@@ -1081,7 +1102,7 @@ int rfb_attn_bwd_image_windows(const void* q, const void* k, const void* v, cons
   sc.d = d;
   sc.shift = shift;
   sc.to_windows = 0;
-  img_move_kernel<<<grid_for(pieces, 256, dev.sms), 256, 0, st>>>(sc);
+  launch_pdl(img_move_kernel, grid_for(pieces, 256, dev.sms), 256, 0, st, sc);
   return launch_status();
 }
 
@@ -1118,9 +1139,9 @@ int rfb_bias_project(const float* bias, const float* x, float* out, int H, int N
   const dim3 grid((N + kProjRows - 1) / kProjRows, H);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (transpose)
-    bias_project_kernel<true><<<grid, kProjThreads, 0, st>>>(bias, x, out, N, k);
+    launch_pdl(bias_project_kernel<true>, grid, kProjThreads, 0, st, bias, x, out, N, k);
   else
-    bias_project_kernel<false><<<grid, kProjThreads, 0, st>>>(bias, x, out, N, k);
+    launch_pdl(bias_project_kernel<false>, grid, kProjThreads, 0, st, bias, x, out, N, k);
   return launch_status();
 }
 
