@@ -369,7 +369,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
   grid_dep_wait();
-  grid_dep_launch_next();
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -742,6 +741,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) bulk_wait_all();  // reductions complete before the CTA exits
   }
 
+  // This CTA's work is done: the next grid may start launching (a long
+  // kernel gains nothing from letting it in earlier).
+  grid_dep_launch_next();
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {

@@ -825,7 +825,6 @@ __global__ void __launch_bounds__(kLongThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{abort_flag, args.err, args.timeout_ns, args.fail_site};
   grid_dep_wait();
-  grid_dep_launch_next();
 
   if (warp == 16) {
     // ------------------------------------------------------------ producer
@@ -1119,6 +1118,9 @@ __global__ void __launch_bounds__(kLongThreads, 1)
     }
   }
 
+  // This CTA's work is done: the next grid may start launching (a long
+  // kernel gains nothing from letting it in earlier).
+  grid_dep_launch_next();
   tc_fence_before();
   __syncthreads();
   if (warp == 17) {

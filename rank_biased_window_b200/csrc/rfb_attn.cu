@@ -294,10 +294,12 @@ int check_shape(int B, int H, int N, int d, int r, float scale, bool* empty) {
 // Launches a kernel with programmatic stream serialisation: it may start while
 // the grid before it in the stream finishes (every kernel launched this way
 // waits for that grid itself before touching global memory, grid_dep_wait()).
-// A launch error is left for launch_status() to read.
+// The long kernels (the persistent forward over N > 128, the backward main
+// pass) go without it: for them it hides nothing, and their forwards measured
+// about 1 % slower with it.  A launch error is left for launch_status().
 template <typename... KArgs, typename... Args>
-void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                const Args&... args) {
+void launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              cudaStream_t st, const Args&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -307,8 +309,18 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   (void)cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                const Args&... args) {
+  launch_k(true, kernel, grid, block, smem, st, args...);
+}
+template <typename... KArgs, typename... Args>
+void launch_plain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                  const Args&... args) {
+  launch_k(false, kernel, grid, block, smem, st, args...);
 }
 
 int launch_status() {
@@ -405,7 +417,8 @@ int launch_long(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st) {
   const long long units = static_cast<long long>((a.N + 2 * kTile - 1) / (2 * kTile)) * a.BH;
   const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
   LaunchTimer timer(kIdFwd, st);
-  launch_pdl(fwd_long_kernel<D, RP>, grid, kLongThreads, C::SMEM, st, m.q, m.k, m.v, m.u, m.w, a);
+  launch_plain(fwd_long_kernel<D, RP>, grid, kLongThreads, C::SMEM, st,
+      m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
 }
 
@@ -445,7 +458,7 @@ int launch_long_dense(const Maps& m, const FwdArgs& a, int sms, cudaStream_t st)
   const long long units = static_cast<long long>((a.N + 2 * kTile - 1) / (2 * kTile)) * a.BH;
   const dim3 grid(static_cast<unsigned>(units < sms ? units : sms));
   LaunchTimer timer(kIdFwd, st);
-  launch_pdl(fwd_long_kernel<D, 0, true>, grid, kLongThreads, C::SMEM, st,
+  launch_plain(fwd_long_kernel<D, 0, true>, grid, kLongThreads, C::SMEM, st,
       m.q, m.k, m.v, m.u, m.w, a);
   return launch_status();
 }
@@ -497,7 +510,7 @@ int launch_bwd_main(const Maps& m, const BwdArgs& a, cudaStream_t st) {
   if (int rc = ensure_smem(bwd_main_kernel<D, RP>, C::SMEM, done)) return rc;
   const dim3 grid((a.N + kTile - 1) / kTile, a.BH);
   LaunchTimer timer(kIdBwdMain, st);
-  launch_pdl(bwd_main_kernel<D, RP>, grid, kBwdThreads, C::SMEM, st,
+  launch_plain(bwd_main_kernel<D, RP>, grid, kBwdThreads, C::SMEM, st,
       m.q, m.k, m.v, m.u, m.w, m.g, m.acc, m.aug, a);
   return launch_status();
 }

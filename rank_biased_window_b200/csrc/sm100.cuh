@@ -113,9 +113,11 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const W
 // serialisation: it may start while the grid before it in the stream is still
 // running, so each one waits here before its first global-memory access (the
 // wait returns once that grid has completed and its writes are visible; at
-// once when there is none).  The persistent kernels then let the grid after
-// them start launching, which overlaps that grid's launch and set-up with
-// their own last tiles (its CTAs find room on an SM only as this grid's exit).
+// once when there is none).  The short persistent kernels (window forward and
+// backward) then let the grid after them start launching at once, which
+// overlaps that grid's launch and set-up with their own tiles (its CTAs find
+// room on an SM only as this grid's CTAs exit); the long ones do so when a
+// CTA's work is done.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
