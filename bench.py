@@ -179,7 +179,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:  # noqa: BLE001
                 pass
-            time.sleep(0.05)
+            time.sleep(0.01)
 
     def __enter__(self):
         if self._h is not None:
@@ -196,7 +196,8 @@ class ClockSampler:
         if self._h is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
         busy = [s for s in self.samples] or [0]
-        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": self.max_mhz,
+        return {"sm_mhz": statistics.median(busy), "sm_min_mhz": min(busy),
+                "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
