@@ -36,7 +36,11 @@
  *     allocates no device memory.
  *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
  *     default stream.  Calls are asynchronous on that stream: a return value
- *     of RFB_OK means the work was enqueued, not that it finished.
+ *     of RFB_OK means the work was enqueued, not that it finished.  Stream
+ *     order holds as usual; the short kernels are launched with programmatic
+ *     stream serialisation, so they may begin while the kernel before them
+ *     on the stream finishes, and wait for it before touching memory.  The
+ *     calls may be captured into CUDA graphs.
  *   - Supported shapes: d in {32, 64}; r in {0, 8, 16, ..., 64} (a multiple of
  *     8); B, H, N >= 0.  B*H*N == 0 is a no-op that returns RFB_OK without
  *     touching any pointer.  When r == 0, u / w / du / dw may be NULL.
