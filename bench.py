@@ -567,7 +567,13 @@ def run_configs(rfb, torch, dev, stream, dist, world, peaks, steps, warmup):
             "note": wl.note,
         }
         if wl.B * wl.H > 1:
-            out[name]["graph_stream"] = graph_stream(rfb, torch, dev, wl, g, peaks, dist, world)
+            # a supplementary figure: a failure here is recorded, not fatal
+            try:
+                out[name]["graph_stream"] = graph_stream(rfb, torch, dev, wl, g, peaks, dist,
+                                                         world)
+            except Exception as e:  # noqa: BLE001
+                torch.cuda.synchronize(dev)
+                out[name]["graph_stream"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     return out
 
 
