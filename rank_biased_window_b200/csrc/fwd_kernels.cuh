@@ -302,6 +302,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     wy = (bw / nwx) % nwy;
     b = bw / (nwx * nwy);
   };
+  // v mod size for 0 <= v < 2 size (a window's rows and columns, shifted).
+  auto wrap = [](int v, int size) { return v >= size ? v - size : v; };
   const int res_heads = args.bias_heads + C::NW - 1;
   const uint32_t res_u = sb + C::OFF_RES, res_w = res_u + res_heads * C::HB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NBAR * 8);
@@ -396,8 +398,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           const int i = jj / 12, qd = (jj / 3) % 4, c = jj % 3;
           int b, wy, wx, h;
           window_of(min(w0 + i, args.BH - 1), b, wy, wx, h);
-          const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-          const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+          const int y = wrap(wy * 8 + 4 * (qd >> 1) + args.shift, args.img_h);
+          const int x = wrap(wx * 8 + 4 * (qd & 1) + args.shift, args.img_w);
           const uint32_t off = i * (NP * D * 2) + qd * (16 * D * 2);
           tma_load_5d(st + c * C::QB + off, c == 0 ? &mQ : c == 1 ? &mK : &mV, in_full(s), 0, h, x,
                       y, b);
@@ -538,7 +540,9 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     // O rows go into this warpgroup's staging tile (the TMA store that read
     // the warp's rows two tiles ago must have finished reading them), one TMA
     // store per warp writes its 32 rows, and LSE is written directly.
-    auto epilogue = [&](int t, int it, float m, float l) {
+    // (IMG: wb, wwy, wwx, wh = the row's window, decoded once per tile; the
+    // warp's rows all lie in that window too.)
+    auto epilogue = [&](int t, int it, float m, float l, int wb, int wwy, int wwx, int wh) {
       tc_fence_after();
       uint32_t ov[D];
       tmem_ld_cols<D>(tmem + lane_base + C::T_O + a * D, ov);
@@ -569,12 +573,10 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         if (wwin < args.BH && n0 < N) {
           if constexpr (IMG) {
             // lane k stores quadrant k of the warp's two
-            int b, wy, wx, h;
-            window_of(wwin, b, wy, wx, h);
             const int qd = (n0 >> 4) + lane;
-            const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-            const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
-            tma_store_5d(&mO, ost + (r0 + 16 * lane) * (D * 2), 0, h, x, y, b);
+            const int y = wrap(wwy * 8 + 4 * (qd >> 1) + args.shift, args.img_h);
+            const int x = wrap(wwx * 8 + 4 * (qd & 1) + args.shift, args.img_w);
+            tma_store_5d(&mO, ost + (r0 + 16 * lane) * (D * 2), 0, wh, x, y, wb);
           } else {
             tma_store_3d(&mO, ost + r0 * (D * 2), 0, n0, wwin);
           }
@@ -586,12 +588,10 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         size_t r = static_cast<size_t>(win) * N + n;
         if constexpr (IMG) {
           // the token's place in the unrolled map
-          int b, wy, wx, h;
-          window_of(win, b, wy, wx, h);
           const int qq = n >> 4;
-          const int y = (wy * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift) % args.img_h;
-          const int x = (wx * 8 + 4 * (qq & 1) + (n & 3) + args.shift) % args.img_w;
-          r = ((static_cast<size_t>(b) * args.img_h + y) * args.img_w + x) * args.img_heads + h;
+          const int y = wrap(wwy * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift, args.img_h);
+          const int x = wrap(wwx * 8 + 4 * (qq & 1) + (n & 3) + args.shift, args.img_w);
+          r = ((static_cast<size_t>(wb) * args.img_h + y) * args.img_w + x) * args.img_heads + wh;
         }
         args.lse[r] = (m + __log2f(l)) * kLn2;
       }
@@ -601,6 +601,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     bool ok = true, pending = false;
     int pt = 0, pit = 0;       // the tile whose epilogue is pending
     float pm = 0.f, pl = 1.f;  // its row maximum and row sum
+    int pb = 0, pwy = 0, pwx = 0, ph = 0;  // its window
     int it = a;
     for (int t = blockIdx.x + a * gridDim.x; t < num_tiles; t += 2 * gridDim.x, it += 2) {
       if (!wait_warp(s_full(a), (it >> 1) & 1, g, 5)) { ok = false; break; }
@@ -611,15 +612,15 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty(a));
       if (N < NP) mask_tail<NP>(sv, N);
+      int wb = 0, wwy = 0, wwx = 0, wh = 0;  // this row's window (image windows)
       if constexpr (IMG) {
+        window_of(min(t * C::NW + wl, args.BH - 1), wb, wwy, wwx, wh);
         // Shifted-window mask: in the last window row (column) of the rolled
         // map the two quadrant rows (columns) come from opposite edges of the
         // unrolled map; keys of another region are excluded.
         if (args.shift > 0) {
-          int b, wy, wx, h;
-          window_of(min(t * C::NW + wl, args.BH - 1), b, wy, wx, h);
           const int qq = n >> 4;
-          const bool split_y = wy == nwy - 1, split_x = wx == nwx - 1;
+          const bool split_y = wwy == nwy - 1, split_x = wwx == nwx - 1;
 #pragma unroll
           for (int kq = 0; kq < 4; ++kq) {
             const bool ok_key = (!split_y || (kq >> 1) == (qq >> 1)) &&
@@ -641,14 +642,19 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full(a));
       // The pending tile's O is read now, so this tile's PV may start.
-      if (pending) epilogue(pt, pit, pm, pl);
+      if (pending) epilogue(pt, pit, pm, pl, pb, pwy, pwx, ph);
       pending = true;
       pt = t;
       pit = it;
       pm = m;
       pl = l;
+      pb = wb;
+      pwy = wwy;
+      pwx = wwx;
+      ph = wh;
     }
-    if (ok && pending && wait_warp(o_full(a), (pit >> 1) & 1, g, 6)) epilogue(pt, pit, pm, pl);
+    if (ok && pending && wait_warp(o_full(a), (pit >> 1) & 1, g, 6))
+      epilogue(pt, pit, pm, pl, pb, pwy, pwx, ph);
     // The O stores must have finished before the CTA exits.
     if (lane < kStoreLanes) bulk_wait_all();
   }
