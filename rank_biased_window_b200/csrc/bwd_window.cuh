@@ -147,6 +147,8 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
     wy = (bw / nwx) % nwy;
     b = bw / (nwx * nwy);
   };
+  // v mod size for 0 <= v < 2 size (a window's rows and columns, shifted).
+  auto wrap = [](int v, int size) { return v >= size ? v - size : v; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -217,8 +219,8 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
             tma_load_4d(st + (c == 5 ? C::S_U : C::S_W) + off, c == 5 ? &mU : &mW, in_full(s), 0,
                         4 * (qd & 1), 4 * (qd >> 1), h);
           } else {
-            const int y = (wy * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-            const int x = (wx * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
+            const int y = wrap(wy * 8 + 4 * (qd >> 1) + args.shift, args.img_h);
+            const int x = wrap(wx * 8 + 4 * (qd & 1) + args.shift, args.img_w);
             const CUtensorMap* mp = c == 0 ? &mQ : c == 1 ? &mK : c == 2 ? &mV : c == 3 ? &mDO : &mO;
             const uint32_t so = c == 0 ? C::S_Q : c == 1 ? C::S_K : c == 2 ? C::S_V : c == 3 ? C::S_DO : C::S_O;
             tma_load_5d(st + so + off, mp, in_full(s), 0, h, x, y, b);
@@ -335,17 +337,20 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
     constexpr int kStoreLanes = IMG ? 6 : 3;
     // LSE of this thread's query row of tile tt (0 for padding rows); loaded
     // one tile ahead so that its global-memory latency overlaps a whole tile.
+    // With image windows it also decodes the row's window into nb, nwy_,
+    // nwx_, nh, which the next tile then uses (rows of a missing window keep
+    // stale values: they are masked and not stored).
+    int nb = 0, nwy_ = 0, nwx_ = 0, nh = 0;
     auto load_lse = [&](int tt) -> float {
       const int wn = tt * NW + wl;
       if (tt >= num_tiles || wn >= args.BH || n >= N) return 0.f;
       size_t r = static_cast<size_t>(wn) * N + n;
       if constexpr (IMG) {
-        int b, wy, wx, h;
-        window_of(wn, b, wy, wx, h);
+        window_of(wn, nb, nwy_, nwx_, nh);
         const int qq = n >> 4;
-        const int y = (wy * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift) % args.img_h;
-        const int x = (wx * 8 + 4 * (qq & 1) + (n & 3) + args.shift) % args.img_w;
-        r = ((static_cast<size_t>(b) * args.img_h + y) * args.img_w + x) * args.img_heads + h;
+        const int y = wrap(nwy_ * 8 + 4 * (qq >> 1) + ((n >> 2) & 3) + args.shift, args.img_h);
+        const int x = wrap(nwx_ * 8 + 4 * (qq & 1) + (n & 3) + args.shift, args.img_w);
+        r = ((static_cast<size_t>(nb) * args.img_h + y) * args.img_w + x) * args.img_heads + nh;
       }
       return args.lse[r];
     };
@@ -356,8 +361,8 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
       const uint32_t st = sb + s * C::STAGE;
       const int win = t * NW + wl;
       const bool valid = win < args.BH && n < N;
-      int b = 0, wy = 0, wx = 0, h = 0;
-      if constexpr (IMG) window_of(min(win, args.BH - 1), b, wy, wx, h);
+      // this row's window, decoded by load_lse(t)
+      const int b = nb, wy = nwy_, wx = nwx_, h = nh;
       const float lse_cur = lse_next;
       lse_next = load_lse(t + gridDim.x);
       // ---- -LSE log2(e) and -D of this query row
@@ -486,13 +491,12 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
         const uint32_t src = c == 0 ? stg_q : c == 1 ? stg_k : stg_v;
         if (wwin < args.BH && n0 < N) {
           if constexpr (IMG) {
-            int b2, wy2, wx2, h2;
-            window_of(wwin, b2, wy2, wx2, h2);
+            // the warp's rows lie in this thread's window (b, wy, wx, h)
             const int k = lane / 3;
             const int qd = (n0 >> 4) + k;
-            const int y = (wy2 * 8 + 4 * (qd >> 1) + args.shift) % args.img_h;
-            const int x = (wx2 * 8 + 4 * (qd & 1) + args.shift) % args.img_w;
-            tma_store_5d(mp, src + k * 1024, 0, h2, x, y, b2);
+            const int y = wrap(wy * 8 + 4 * (qd >> 1) + args.shift, args.img_h);
+            const int x = wrap(wx * 8 + 4 * (qd & 1) + args.shift, args.img_w);
+            tma_store_5d(mp, src + k * 1024, 0, h, x, y, b);
           } else {
             tma_store_3d(mp, src, 0, n0, wwin);
           }
