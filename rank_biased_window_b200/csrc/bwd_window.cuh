@@ -412,10 +412,12 @@ __global__ void __launch_bounds__(kBwdWinThreads, 1)
         uint32_t xy[64];
         tmem_ld32x2(tmem + lane_base + C::T_S + c0 + cc, tmem + lane_base + C::T_DP + c0 + cc, xy);
         // Padding keys / queries and masked pairs: a score of -inf gives P = 0, dS = 0.
+        if (!valid || N < cc + 32 || mask_bits != 0) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = cc + e;
-          if (!valid || q >= N || ((n ^ q) & mask_bits) != 0) xy[e] = 0xFF800000u;
+          for (int e = 0; e < 32; ++e) {
+            const int q = cc + e;
+            if (!valid || q >= N || ((n ^ q) & mask_bits) != 0) xy[e] = 0xFF800000u;
+          }
         }
         uint32_t pk[16], dk[16];
 #pragma unroll

@@ -621,13 +621,15 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         if (args.shift > 0) {
           const int qq = n >> 4;
           const bool split_y = wwy == nwy - 1, split_x = wwx == nwx - 1;
+          if (split_y || split_x) {  // windows inside the map need no mask
 #pragma unroll
-          for (int kq = 0; kq < 4; ++kq) {
-            const bool ok_key = (!split_y || (kq >> 1) == (qq >> 1)) &&
-                                (!split_x || (kq & 1) == (qq & 1));
-            if (!ok_key) {
+            for (int kq = 0; kq < 4; ++kq) {
+              const bool ok_key = (!split_y || (kq >> 1) == (qq >> 1)) &&
+                                  (!split_x || (kq & 1) == (qq & 1));
+              if (!ok_key) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) sv[kq * 16 + e] = 0xFF800000u;
+                for (int e = 0; e < 16; ++e) sv[kq * 16 + e] = 0xFF800000u;
+              }
             }
           }
         }
