@@ -99,3 +99,48 @@ def test_graph_captured_chain_matches_eager(rfb_lib, cuda_dev):
         for i, (a, b) in enumerate(zip(_flat(cap), _flat(eager))):
             assert torch.equal(a, b), f"output {i} of the replayed chain differs"
     del graph
+
+
+def test_concurrent_streams_match_sequential(rfb_lib, cuda_dev):
+    """Calls on two streams at once share no device state: a window forward
+    and a long forward with its backward (own workspace) on one stream, the
+    same on other inputs on a second stream, repeated, give what each gives
+    alone.  dQ, dU come from reductions whose order varies and are compared
+    with a tolerance of their fp32 rounding; the rest bit for bit."""
+    shapes = [(300, 1, 64, 32, 8), (2, 3, 640, 64, 16)]
+    sets = []
+    for j in range(2):
+        for B, H, N, d, r in shapes:
+            g = _dev(make_inputs(B, H, N, d, r, seed=7300 + 10 * j + N, with_dout=True), cuda_dev)
+            sets.append((g, (B, H, N, d, r), _bufs(rfb_lib, g, B, H, N, d, r, cuda_dev)))
+
+    def run(items, stream):
+        with torch.cuda.stream(stream):
+            for g, (B, H, N, d, r), b in items:
+                s = 1.0 / math.sqrt(d)
+                o, lse = rfb_lib.attn_fwd(g["q"], g["k"], g["v"], g["u"], g["w"], s,
+                                          out=b["o"], lse=b["lse"])
+                rfb_lib.attn_bwd(g["q"], g["k"], g["v"], g["u"], g["w"], o, lse, g["dout"], s,
+                                 workspace=b["ws"], grads=b["grads"])
+
+    s0 = torch.cuda.current_stream(cuda_dev)
+    run(sets, s0)
+    torch.cuda.synchronize()
+    ref = [[t.clone() for t in (b["o"], b["lse"], *b["grads"])] for _, _, b in sets]
+    sa, sb = torch.cuda.Stream(cuda_dev), torch.cuda.Stream(cuda_dev)
+    for _ in range(3):
+        for _, _, b in sets:
+            for t in (b["o"], b["lse"], *b["grads"]):
+                t.zero_()
+        torch.cuda.synchronize()
+        run(sets[:2] * 2, sa)   # the first input set twice on stream a
+        run(sets[2:] * 2, sb)   # the second on stream b, concurrently
+        torch.cuda.synchronize()
+        assert rfb_lib.last_device_error() == 0
+        for (_, shape, b), want in zip(sets, ref):
+            got = [b["o"], b["lse"], *b["grads"]]
+            for i, (x, y) in enumerate(zip(got, want)):
+                if i in (2, 5) and shape[2] > 128:  # dQ, dU of the long backward
+                    assert torch.allclose(x.float(), y.float(), rtol=1e-2, atol=1e-3), (shape, i)
+                else:
+                    assert torch.equal(x, y), (shape, i)
